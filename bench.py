@@ -1,0 +1,353 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the fused MiMo-V2 preprocessing path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload c5] [--dtype f32|bf16]
+
+A step is one call of the C-ABI entry point mimo_preprocess_batch over the
+whole batch of the workload (default: 256 images 1080x1920, half RGB / half
+RGBA -> 1088x1920, fp32 rows + column-order permutation), with the packed
+uint8 inputs already resident in HBM. Timing: W untimed warm-up steps, then K
+steps bracketed by barrier + synchronize, CUDA events on the launching stream,
+max over ranks. Inputs (1.86 GB) and outputs (12.8 GB fp32) are far larger
+than the 126 MB L2, so no flush is needed between steps.
+
+Under torchrun each rank processes its own batch (different seed), with no
+collective on the data path: weak scaling.
+
+Also reported on the same JSON line:
+  roofline     algorithmic bytes of the kernel (uint8 read + rows written +
+               permutation written) / its average event-timed duration,
+               against the measured HBM copy bandwidth;
+  e2e          the same metric through mimo_preprocess_batch_host: pinned
+               host images in, pinned host rows out, copies inside the timing;
+  cpu_baseline the CPU oracle timed on a bounded sample of the same workload
+               on this host's cores (rank 0, N=1 only);
+  clocks       SM clock and throttle reasons sampled through NVML during the
+               timed region.
+
+--impl reference times the CPU oracle alone (rank 0; other ranks exit).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "images/s and output HBM GB/s (% of B200 peak) for fused MiMo preprocess"
+UNIT = "images/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c5", choices=["c2", "c3", "c4", "c5"])
+    ap.add_argument("--dtype", default=None, choices=["f32", "bf16"])
+    ap.add_argument("--images", type=int, default=None, help="override the workload's image count")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    for rel in ("vision_lm_image_b200/csrc/mimo_preprocess.cu", "vision_lm_image_b200/csrc/mimo_internal.h"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, dtype: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    entry = d.get(f"{workload}_{dtype}")
+    if not entry or entry.get("kernel_digest") != kernel_source_digest():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.handle, self.nv.NVML_CLOCK_SM))
+            bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+            for b, name in self.REASONS.items():
+                if bits & b:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+            self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        s = sorted(self.samples)
+        return {"sm_mhz": s[len(s) // 2], "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(s)}
+
+
+def algorithmic_bytes(packed, total_rows, dtype_bytes, perm: bool) -> dict:
+    read = int(sum(int(h) * int(w) * int(c) for h, w, c in zip(packed.heights, packed.widths, packed.channels)))
+    write_rows = int(total_rows) * 1536 * dtype_bytes
+    write_perm = int(total_rows) * 4 if perm else 0
+    return {"read": read, "write_rows": write_rows, "write_perm": write_perm,
+            "total": read + write_rows + write_perm}
+
+
+def cpu_baseline(w, sample_images: int, threads: int):
+    import oracle
+
+    imgs = w["images"][:sample_images]
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.preprocess(imgs, w["mean"], w["std"], column_perm=w["column_perm"], threads=threads)
+    dt = time.perf_counter() - t0
+    return len(imgs) / dt, dt
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    import workloads
+
+    if rank != 0:
+        return
+    w = workloads.workload(args.workload, n_images=args.images)
+    if args.dtype:
+        w["dtype"] = args.dtype
+    cores = host_cores()
+    per_step = max(1, min(len(w["images"]), 2 * cores, 16))
+    sample = f"{per_step} of the workload's {len(w['images'])} images per step, oracle on {cores} threads"
+    for _ in range(args.warmup):
+        cpu_baseline(w, per_step, cores)
+    t = 0.0
+    for _ in range(args.steps):
+        _, dt = cpu_baseline(w, per_step, cores)
+        t += dt
+    value = per_step * args.steps / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "description": w["description"], "images": len(w["images"]),
+                   "out_dtype": w["dtype"], "column_perm": w["column_perm"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import workloads
+    from vision_lm_image_b200 import build as _build
+    from vision_lm_image_b200 import mimo
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    if not os.path.exists(_build.LIB_PATH):
+        _build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = workloads.workload(args.workload, seed_offset=7919 * rank, n_images=args.images)
+    out_dtype = args.dtype or w["dtype"]
+    tdtype = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+    dbytes = 2 if out_dtype == "bf16" else 4
+    params = mimo.make_params(w["mean"], w["std"])
+    host = mimo.pack_images(w["images"], device="cpu", pin_memory=True)
+    packed = host.to(dev)
+    grid, offs = mimo.plan_batch(host.heights, host.widths, params)
+    total = int(offs[-1])
+    out = torch.empty((total, 1536), dtype=tdtype, device=dev)
+    perm = torch.empty(total, dtype=torch.int32, device=dev) if w["column_perm"] else None
+    n_img = host.n
+    launches_per_step = (n_img + 511) // 512
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mimo.preprocess_batch(params, packed, out, perm, stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        ev[0].record(stream)
+        for k in range(K):
+            step()
+            ev[k + 1].record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    per_launch_ms = [ev[k].elapsed_time(ev[k + 1]) for k in range(K)]
+    elapsed_ms = ev[0].elapsed_time(ev[K])
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    nbytes = algorithmic_bytes(host, total, dbytes, perm is not None)
+    avg_launch_ms = sum(per_launch_ms) / K / launches_per_step
+    peak, peak_kind = measured_hbm_peak()
+    achieved = nbytes["total"] / (avg_launch_ms * 1e-3) / 1e9
+    value = world * n_img * K / (max_ms * 1e-3)
+    out_gbs = nbytes["write_rows"] / (max_ms / K * 1e-3) / 1e9
+
+    # e2e: host images in, host rows out, through the host-buffer entry point
+    e2e = None
+    if not args.no_e2e and args.e2e_steps > 0:
+        out_h = torch.empty((total, 1536), dtype=tdtype, pin_memory=True)
+        perm_h = torch.empty(total, dtype=torch.int32, pin_memory=True) if perm is not None else None
+        mimo.preprocess_batch_host(params, host, out_h, perm_h, packed.buffer, out, perm, stream)  # warm-up
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(args.e2e_steps):
+            mimo.preprocess_batch_host(params, host, out_h, perm_h, packed.buffer, out, perm, stream)
+        torch.cuda.synchronize()
+        e2e_s = time.perf_counter() - t0
+        te = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.barrier()
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * n_img * args.e2e_steps / float(te.item()), "unit": UNIT,
+               "h2d_bytes_per_step": int(host.buffer.numel()),
+               "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()
+                                         + (perm_h.numel() * 4 if perm_h is not None else 0)),
+               "timing": "host wall clock around the synchronous host-to-host call"}
+        del out_h, perm_h
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = host_cores()
+        sample_n = max(1, min(n_img, 2 * cores, 64))
+        v, dt = cpu_baseline(w, sample_n, cores)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"first {sample_n} of the {n_img} workload images, one pass, {dt:.1f} s"}
+
+    if dist is not None:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "description": w["description"], "images_per_gpu": n_img,
+                       "out_dtype": out_dtype, "column_perm": perm is not None, "rows_per_gpu": total,
+                       "l2": "inputs and outputs larger than L2 (no flush)", "parallelism": f"dp{world}"},
+            "output_gbs": out_gbs,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "traffic": ncu_traffic(args.workload, out_dtype),
+                         "algorithmic_bytes_per_launch": nbytes["total"] // launches_per_step,
+                         "kernel": "preprocess_kernel", "avg_launch_ms": avg_launch_ms},
+            "gpu_launches": K * launches_per_step,
+            "clocks": clocks.summary(),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.impl == "reference" else 1)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,178 @@
+/*
+ * mimo.h -- C ABI of the B200 MiMo-V2 image preprocessing library.
+ *
+ * The library turns decoded 8-bit images into the patch rows the MiMo-V2
+ * vision tower consumes, on the GPU, in one fused kernel per batch. The
+ * operation is the pixel path of MimoV2ImageProcessor (NeMo Automodel page
+ * "nemo_automodel.components.models.mimo_v2_flash.processing", class
+ * MimoV2ImageProcessor and its __call__; restated on docs.rs
+ * "cortiq_engine::mimo_vision", conventions list and prepare_image):
+ *
+ *   smart_resize geometry (factor = patch_size * merge_size = 32)
+ *   -> RGBA composited onto white (function _to_rgb), alpha dropped
+ *   -> uint8 to float on the 0..255 scale
+ *   -> bilinear resize, align_corners=False, no antialias, no 8-bit rounding
+ *   -> (x - 255*mean_c) / (255*std_c)
+ *   -> the frame duplicated to temporal_patch_size = 2 frames
+ *   -> rows of 3*2*16*16 = 1536 values laid out (c, tt, py, px),
+ *      rows ordered (t, block row, block col, mh, mw) (merge-block order)
+ *   -> optionally the column-order row permutation (column_permutation:
+ *      merge units listed by (t, block col, block row), perm[dst] = src).
+ *
+ * Conventions for every entry point:
+ *   - Return value: a mimo_status (0 = MIMO_OK). Every argument problem the
+ *     host can see is reported before anything is launched or copied; the
+ *     device code contains no traps and no waits.
+ *   - Ownership: the caller owns every buffer. The library never allocates
+ *     or frees device memory and keeps no state between calls.
+ *   - "d_" pointers are device pointers, "h_" pointers host pointers; the
+ *     other arrays (sizes, offsets) are host arrays read during the call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Device work is asynchronous on it unless stated otherwise.
+ *   - Only the geometry knobs patch_size = 16, temporal_patch_size = 2 and
+ *     merge_size = 2 are implemented on the GPU (the processor's defaults);
+ *     other values return MIMO_EUNSUPPORTED.
+ */
+#ifndef MIMO_H_
+#define MIMO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MIMO_OK = 0,
+    MIMO_EINVAL = 1,        /* null pointer, negative count, non-positive size, bad knob */
+    MIMO_EASPECT = 2,       /* long/short side above 200 with the short side >= factor   */
+    MIMO_EDEGENERATE = 3,   /* the max_pixels shrink rounds a side down to zero          */
+    MIMO_ECHANNELS = 4,     /* channels other than 3 (RGB) or 4 (RGBA)                  */
+    MIMO_EUNSUPPORTED = 5,  /* patch/temporal/merge other than 16/2/2, or std <= 0       */
+    MIMO_EALIGN = 6,        /* a source offset or output pointer is not 16-byte aligned  */
+    MIMO_ECAPACITY = 7,     /* an output or staging buffer is too small for the batch    */
+    MIMO_EOVERFLOW = 8,     /* a size does not fit the index types (see each call)       */
+    MIMO_ECUDA = 9,         /* a CUDA runtime call failed (launch or copy)               */
+    MIMO_ERANGE = 10        /* an image reaches past the end of the source buffer        */
+} mimo_status;
+
+typedef enum {
+    MIMO_F32 = 0,   /* float32 patch values (the processor's own output type)   */
+    MIMO_BF16 = 1   /* bfloat16, rounded to nearest-even from the float32 value */
+} mimo_dtype;
+
+/*
+ * Processor knobs (class MimoV2ImageProcessor constructor; per-call
+ * min_pixels / max_pixels overrides of __call__ are expressed by passing a
+ * struct with other bounds). Statistics are always caller-supplied: the page
+ * reads them from the checkpoint (ImageNet for MiMo-V2.6, CLIP for V2.5).
+ */
+typedef struct {
+    int32_t patch_size;           /* 16 */
+    int32_t temporal_patch_size;  /* 2  */
+    int32_t merge_size;           /* 2  */
+    int32_t reserved;             /* must be 0 */
+    int64_t min_pixels;           /* 8192    (lower bound on resized area) */
+    int64_t max_pixels;           /* 8388608 (upper bound on resized area) */
+    float image_mean[3];          /* per-channel mean on the 0..1 scale    */
+    float image_std[3];           /* per-channel std on the 0..1 scale, > 0 */
+} mimo_params;
+
+/* Fills the constructor defaults: 16/2/2, 8192, 8388608, ImageNet
+ * mean (0.485, 0.456, 0.406) and std (0.229, 0.224, 0.225). */
+void mimo_params_default(mimo_params *p);
+
+/*
+ * smart_resize (processing page, function smart_resize; cortiq page,
+ * smart_resize). Resized (height, width), both multiples of `factor`:
+ *  - a side below `factor` first scales both sides so the short side equals
+ *    `factor`; that branch skips the aspect guard;
+ *  - otherwise long/short > 200 -> MIMO_EASPECT;
+ *  - each side rounds to the nearest multiple of factor (exact halves to
+ *    even); an area above max_pixels shrinks by sqrt(area/max_pixels) with
+ *    floor (a zero side -> MIMO_EDEGENERATE), an area below min_pixels grows
+ *    by sqrt(min_pixels/area) with ceil.
+ * Host only. Errors: MIMO_EINVAL for non-positive sizes/factor, null outputs.
+ */
+int mimo_smart_resize(int64_t height, int64_t width, int64_t factor,
+                      int64_t min_pixels, int64_t max_pixels,
+                      int64_t *out_height, int64_t *out_width);
+
+/*
+ * get_number_of_image_patches (processing page): grid_h * grid_w of the
+ * resized image, before the merge_size**2 reduction (vision tokens =
+ * *out_patches / 4). Host only.
+ */
+int mimo_num_patches(int64_t height, int64_t width, const mimo_params *p, int64_t *out_patches);
+
+/*
+ * Batch plan (the __call__ batch assembly: per-image rows concatenated,
+ * image_grid_thw of shape [n, 3]). Host only.
+ *   heights/widths: [n] source sizes.
+ *   grid_thw:       out, [n*3] int64, rows (1, H'/16, W'/16).
+ *   row_offsets:    out, [n+1] int64, first output row of each image; the
+ *                   last entry is the total number of rows.
+ * The first image whose geometry fails decides the returned status.
+ */
+int mimo_plan_batch(int32_t n, const int32_t *heights, const int32_t *widths,
+                    const mimo_params *p, int64_t *grid_thw, int64_t *row_offsets);
+
+/*
+ * The fused pixel path for a batch, on the GPU.
+ *   d_src:        device, packed interleaved HWC uint8 images.
+ *   src_bytes:    size of the d_src buffer; every image must lie inside it
+ *                 (MIMO_ERANGE otherwise).
+ *   src_offsets:  host [n], byte offset of image i in d_src, a multiple of 16.
+ *   heights, widths, channels: host [n]; channels 3 (RGB) or 4 (RGBA).
+ *   out_dtype:    MIMO_F32 or MIMO_BF16.
+ *   d_out:        device [out_rows_capacity, 1536] of out_dtype, 16-byte
+ *                 aligned; rows [row_offsets[i], row_offsets[i+1]) belong
+ *                 to image i, in the order of mimo_plan_batch.
+ *   d_column_perm: device int32 [total_rows] or NULL. When given, receives
+ *                 the column-order permutation of every image, as indices
+ *                 into the whole batch (pixel_values[perm] works directly);
+ *                 16-byte aligned; total_rows must fit int32
+ *                 (MIMO_EOVERFLOW otherwise).
+ * Every output row and permutation entry in [0, total_rows) is written
+ * exactly once; nothing past total_rows is touched. Asynchronous on
+ * `stream`; launch errors come back as MIMO_ECUDA.
+ */
+int mimo_preprocess_batch(const mimo_params *p, int32_t n,
+                          const uint8_t *d_src, size_t src_bytes, const int64_t *src_offsets,
+                          const int32_t *heights, const int32_t *widths, const int32_t *channels,
+                          int32_t out_dtype, void *d_out, int64_t out_rows_capacity,
+                          int32_t *d_column_perm, void *stream);
+
+/*
+ * The same path from host memory to host memory (inputs copied in, rows and
+ * permutation copied back), for callers whose images and results live on
+ * the host. The caller supplies device staging buffers of at least the batch
+ * size (d_src_stage >= src_bytes; d_out_stage >= total_rows rows of
+ * out_dtype; d_perm_stage >= total_rows int32 when h_column_perm is not
+ * NULL), so the call allocates nothing. Host buffers should be page-locked
+ * for full copy bandwidth. The batch is cut into chunks of images whose
+ * upload, kernel and download overlap on the caller's stream plus library-
+ * created streams that live only for the call. Synchronous: returns after
+ * the last copy to h_out has completed.
+ */
+int mimo_preprocess_batch_host(const mimo_params *p, int32_t n,
+                               const uint8_t *h_src, size_t src_bytes, const int64_t *src_offsets,
+                               const int32_t *heights, const int32_t *widths, const int32_t *channels,
+                               int32_t out_dtype, void *h_out, int64_t out_rows_capacity,
+                               int32_t *h_column_perm,
+                               uint8_t *d_src_stage, size_t d_src_stage_bytes,
+                               void *d_out_stage, int64_t d_out_stage_rows,
+                               int32_t *d_perm_stage, void *stream);
+
+/* Static description of a status code. */
+const char *mimo_status_string(int status);
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+int mimo_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MIMO_H_ */

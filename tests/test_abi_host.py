@@ -1,0 +1,152 @@
+"""Host-side checks of the C ABI (no GPU needed, nothing is launched).
+
+- the library loads and exports every function include/mimo.h declares;
+- the library's own smart_resize / plan agree bit for bit with the oracle's;
+- argument validation returns the documented status before any device work.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from vision_lm_image_b200 import build, mimo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(mimo_[a-z_0-9]+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert {"mimo_smart_resize", "mimo_preprocess_batch", "mimo_plan_batch"} <= names
+    L = ctypes.CDLL(mimo.library_path())
+    for name in sorted(names):
+        assert hasattr(L, name), name
+    assert set(mimo.EXPORTED) == names
+
+
+def test_version_and_status_strings():
+    L = mimo.lib()
+    assert L.mimo_version() >= 10000
+    for s in range(11):
+        assert L.mimo_status_string(s) and L.mimo_status_string(s) != b"unknown status"
+
+
+def test_defaults_match_processor_constructor():
+    p = mimo.make_params()
+    assert (p.patch_size, p.temporal_patch_size, p.merge_size) == (16, 2, 2)
+    assert (p.min_pixels, p.max_pixels) == (8192, 8388608)
+    assert np.allclose(list(p.image_mean), workloads.IMAGENET_MEAN)
+    assert np.allclose(list(p.image_std), workloads.IMAGENET_STD)
+
+
+def test_smart_resize_matches_oracle_exhaustive():
+    for h in range(1, 200):
+        for w in range(1, 200, 7):
+            assert mimo.smart_resize_status(h, w) == oracle.smart_resize_status(h, w)
+            if oracle.smart_resize_status(h, w) == oracle.OK:
+                assert mimo.smart_resize(h, w) == oracle.smart_resize(h, w), (h, w)
+
+
+@pytest.mark.parametrize("bounds", [(8192, 8388608), (50_000, 200_000), (0, 1 << 40), (8192, 30_000)])
+def test_smart_resize_matches_oracle_random(bounds):
+    mn, mx = bounds
+    rng = np.random.Generator(np.random.PCG64(21))
+    for _ in range(5000):
+        h = int(np.exp(rng.uniform(0, np.log(60000))))
+        w = int(np.exp(rng.uniform(0, np.log(60000))))
+        for factor in (32, 28):
+            so = oracle.smart_resize_status(h, w, factor, mn, mx)
+            assert mimo.smart_resize_status(h, w, factor, mn, mx) == so, (h, w, factor)
+            if so == oracle.OK:
+                assert mimo.smart_resize(h, w, factor, mn, mx) == oracle.smart_resize(h, w, factor, mn, mx)
+
+
+def test_plan_batch_matches_oracle():
+    imgs = workloads.random_small_batch(77, 40, max_side=400)
+    H = [im.shape[0] for im in imgs]
+    W = [im.shape[1] for im in imgs]
+    grid, offs = mimo.plan_batch(H, W)
+    assert offs[0] == 0
+    for i, (h, w) in enumerate(zip(H, W)):
+        oh, ow = oracle.smart_resize(h, w)
+        assert tuple(grid[i]) == (1, oh // 16, ow // 16)
+        assert offs[i + 1] - offs[i] == oracle.get_number_of_image_patches(h, w)
+    assert mimo.get_number_of_image_patches(1080, 1920) == 8160
+
+
+def test_plan_batch_errors():
+    with pytest.raises(mimo.MimoError) as e:
+        mimo.plan_batch([32], [6401])
+    assert e.value.status == 2
+    with pytest.raises(mimo.MimoError) as e:
+        mimo.plan_batch([16], [300000])
+    assert e.value.status == 3
+    with pytest.raises(mimo.MimoError) as e:
+        mimo.plan_batch([0], [5])
+    assert e.value.status == 1
+    with pytest.raises(mimo.MimoError) as e:
+        mimo.plan_batch([64], [64], mimo.make_params(patch_size=14))
+    assert e.value.status == 5
+    g, o = mimo.plan_batch([], [])
+    assert g.shape == (0, 3) and list(o) == [0]
+
+
+# Validation-only calls: every call below must fail before launching. They are
+# run only where no GPU is present, so a validation bug cannot send a bogus
+# pointer to a real device.
+no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(), reason="host-validation test uses fake device pointers")
+
+FAKE = 1 << 20  # 16-byte aligned, never dereferenced
+
+
+def _call(p=None, n=1, src=FAKE, src_bytes=1 << 30, offsets=(0,), H=(64,), W=(48,), C=(3,), dtype=0,
+          out=FAKE, cap=1 << 20, perm=0):
+    p = p or mimo.make_params()
+    offs = np.asarray(offsets, np.int64)
+    h = np.asarray(H, np.int32)
+    w = np.asarray(W, np.int32)
+    c = np.asarray(C, np.int32)
+    return mimo.lib().mimo_preprocess_batch(ctypes.byref(p), n, ctypes.c_void_p(src), src_bytes, offs.ctypes.data,
+                                            h.ctypes.data, w.ctypes.data, c.ctypes.data, dtype,
+                                            ctypes.c_void_p(out), cap, ctypes.c_void_p(perm), None)
+
+
+@no_gpu_only
+def test_validation_statuses():
+    assert _call(n=0) == 0                                  # empty batch: nothing to do
+    assert _call(C=(2,)) == 4                               # channels
+    assert _call(offsets=(8,)) == 6                         # misaligned offset
+    assert _call(src=FAKE + 4) == 6                         # misaligned base
+    assert _call(out=FAKE + 8) == 6                         # misaligned output
+    assert _call(perm=FAKE + 4) == 6                        # misaligned permutation
+    assert _call(cap=47) == 7                               # 64x48 -> 48 rows
+    assert _call(src_bytes=64 * 48 * 3 - 1) == 10           # image past the end of the buffer
+    assert _call(offsets=(16,), src_bytes=64 * 48 * 3) == 10
+    assert _call(H=(32,), W=(6401,)) == 2                   # aspect
+    assert _call(H=(16,), W=(300000,)) == 3                 # degenerate shrink
+    assert _call(dtype=7) == 1                              # dtype
+    assert _call(n=-1) == 1
+    assert _call(out=0) == 1
+    p = mimo.make_params(std=(0.2, 0.0, 0.2))
+    assert _call(p=p) == 5                                  # std must be > 0
+    p = mimo.make_params(merge_size=1)
+    assert _call(p=p) == 5

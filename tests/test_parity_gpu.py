@@ -1,0 +1,254 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle, element by element.
+
+Bars (from the method's definition and the arithmetic of both sides):
+- geometry, image_grid_thw, row offsets and the column permutation: bit-exact;
+- fp32 patch values: |gpu - oracle| <= 1e-4 in normalised units;
+- bf16 patch values: within one bf16 ulp of the oracle value rounded to bf16, with the ulp taken no
+  smaller than 2**-19 (below |v| ~ 2**-12 the fp32 rounding noise of the GPU arithmetic, ~1e-6, is
+  larger than a bf16 ulp and may move the rounding by more than one step).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from vision_lm_image_b200 import build, mimo
+
+pytestmark = pytest.mark.gpu
+
+FP32_ATOL = 1e-4
+BF16_ULP_FLOOR = 2.0 ** -19
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+    oracle.build()
+
+
+def gpu_run(images, mean, std, dtype=torch.float32, column_perm=False, min_pixels=None, max_pixels=None):
+    pv, grid, perm = mimo.preprocess(images, mean, std, min_pixels=min_pixels, max_pixels=max_pixels,
+                                     dtype=dtype, column_perm=column_perm)
+    torch.cuda.synchronize()
+    return pv, grid.numpy(), perm
+
+
+def assert_fp32_close(gpu: np.ndarray, ref: np.ndarray, what=""):
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    assert np.isfinite(gpu).all(), what
+    err = np.abs(gpu.astype(np.float64) - ref.astype(np.float64))
+    worst = float(err.max()) if err.size else 0.0
+    assert worst <= FP32_ATOL, f"{what}: max |gpu - oracle| = {worst:.3e}"
+    return worst
+
+
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    a = np.abs(v.astype(np.float64))
+    e = np.floor(np.log2(np.maximum(a, 1e-30)))
+    return np.maximum(2.0 ** (e - 7), BF16_ULP_FLOOR)
+
+
+def assert_bf16_close(gpu_bf16: torch.Tensor, ref_f32: np.ndarray, what=""):
+    g = gpu_bf16.float().cpu().numpy().astype(np.float64)
+    r = oracle.bf16_bits_to_f32(oracle.round_to_bf16(ref_f32)).astype(np.float64)
+    assert g.shape == r.shape
+    bad = np.abs(g - r) > bf16_ulp(r)
+    assert not bad.any(), f"{what}: {int(bad.sum())} values beyond 1 bf16 ulp"
+
+
+def check_against_oracle(images, mean, std, threads=8, min_pixels=8192, max_pixels=8388608, perm=True):
+    pv, grid, gperm = gpu_run(images, mean, std, column_perm=perm, min_pixels=min_pixels, max_pixels=max_pixels)
+    ref, rgrid, rperm = oracle.preprocess(images, mean, std, min_pixels=min_pixels, max_pixels=max_pixels,
+                                          column_perm=perm, threads=threads)
+    assert np.array_equal(grid, rgrid)
+    worst = assert_fp32_close(pv.cpu().numpy(), ref)
+    if perm:
+        assert np.array_equal(gperm.cpu().numpy(), rperm)
+    return worst
+
+
+# ---------------------------------------------------------------- the five workloads
+def test_c1_single_upscaled_image():
+    w = workloads.workload("c1")
+    check_against_oracle(w["images"], w["mean"], w["std"])
+
+
+def test_c2_rgba_identity_batch():
+    w = workloads.workload("c2")
+    check_against_oracle(w["images"], w["mean"], w["std"])
+
+
+def test_c3_mixed_sizes_clip():
+    w = workloads.workload("c3")
+    check_against_oracle(w["images"], w["mean"], w["std"], threads=16)
+
+
+def test_c4_max_pixels_downscale():
+    w = workloads.workload("c4")
+    check_against_oracle(w["images"], w["mean"], w["std"], perm=False)
+
+
+def test_c5_full_size_sampled():
+    """Full 256-image batch in the launch the benchmark times: exact permutation, two whole images
+    against the oracle, random samples across all images, both temporal copies identical."""
+    w = workloads.workload("c5")
+    imgs = w["images"]
+    pv, grid, perm = gpu_run(imgs, w["mean"], w["std"], column_perm=True)
+    assert pv.shape == (256 * 8160, 1536)
+    assert (grid == np.array([1, 68, 120])).all()
+    # permutation: bit-exact for the whole batch
+    rperm = np.concatenate([oracle.column_permutation(68, 120, 2, 8160 * i) for i in range(256)])
+    assert np.array_equal(perm.cpu().numpy(), rperm)
+    # both frames identical everywhere
+    v = pv.view(-1, 3, 2, 256)
+    assert torch.equal(v[:, :, 0], v[:, :, 1])
+    # two whole images: one RGB (index 2), one RGBA (index 255)
+    for i in (2, 255):
+        ref, g = oracle.preprocess_image(imgs[i], w["mean"], w["std"])
+        assert_fp32_close(pv[8160 * i:8160 * (i + 1)].cpu().numpy(), ref, f"image {i}")
+    # samples across the whole batch
+    rng = np.random.Generator(np.random.PCG64(55))
+    n = 3000
+    img_idx = rng.integers(0, 256, n)
+    rows = rng.integers(0, 8160, n)
+    cols = rng.integers(0, 1536, n)
+    flat = (torch.from_numpy(img_idx * 8160 + rows) * 1536 + torch.from_numpy(cols)).cuda()
+    got = pv.view(-1).index_select(0, flat).cpu().numpy()
+    want = np.array([oracle.patch_value(imgs[i], (1088, 1920), int(r), int(c), w["mean"], w["std"])
+                     for i, r, c in zip(img_idx, rows, cols)], np.float32)
+    assert_fp32_close(got, want, "samples")
+
+
+def test_c5_bf16_subset():
+    w = workloads.workload("c5", n_images=6)
+    pv, grid, perm = gpu_run(w["images"], w["mean"], w["std"], dtype=torch.bfloat16, column_perm=True)
+    ref, rgrid, rperm = oracle.preprocess(w["images"], w["mean"], w["std"], column_perm=True, threads=6)
+    assert np.array_equal(grid, rgrid) and np.array_equal(perm.cpu().numpy(), rperm)
+    assert_bf16_close(pv, ref, "c5 bf16")
+
+
+def test_c3_bf16():
+    w = workloads.workload("c3", n_images=12)
+    pv, _, _ = gpu_run(w["images"], w["mean"], w["std"], dtype=torch.bfloat16)
+    ref, _, _ = oracle.preprocess(w["images"], w["mean"], w["std"], threads=8)
+    assert_bf16_close(pv, ref, "c3 bf16")
+
+
+# ---------------------------------------------------------------- sweeps and edge cases
+@pytest.mark.parametrize("seed", range(5))
+def test_random_small_batches(seed):
+    imgs = workloads.random_small_batch(900 + seed, 24, max_side=300, min_side=1)
+    check_against_oracle(imgs, workloads.CLIP_MEAN, workloads.CLIP_STD)
+
+
+def test_flatten_exhaustive_identity_image():
+    # every (c, a) pair once: 256x256 RGBA is a multiple of 32 inside the bounds -> identity resize
+    c = np.tile(np.arange(256, dtype=np.uint8), 256).reshape(256, 256)
+    a = np.repeat(np.arange(256, dtype=np.uint8), 256).reshape(256, 256)
+    img = np.stack([c, 255 - c, c // 2 + 7, a], axis=-1)
+    check_against_oracle([img], workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+
+
+def test_gathered_taps_strong_downscale():
+    # a per-call max_pixels override makes the shrink factor > 2, so the kernel gathers taps
+    rng = workloads.rng_for(5)
+    imgs = [workloads.uniform_image(rng, 2000, 2000, 3), workloads.rgba_image(rng, 1500, 3000),
+            workloads.uniform_image(rng, 3000, 700, 3)]
+    check_against_oracle(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD, max_pixels=200_000)
+
+
+def test_extreme_shapes():
+    rng = workloads.rng_for(6)
+    imgs = [workloads.uniform_image(rng, 1, 1, 3), workloads.rgba_image(rng, 1, 200),
+            workloads.uniform_image(rng, 32, 6400, 3), workloads.rgba_image(rng, 6400, 32),
+            workloads.uniform_image(rng, 31, 33, 3), workloads.uniform_image(rng, 33, 4001, 3)]
+    check_against_oracle(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+
+
+def test_more_images_than_one_launch():
+    # more than 512 images: the host cuts the batch into several launches
+    rng = workloads.rng_for(7)
+    imgs = [workloads.uniform_image(rng, int(rng.integers(20, 70)), int(rng.integers(20, 70)), 3 + i % 2)
+            for i in range(1100)]
+    check_against_oracle(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+
+
+def test_coverage_sentinels():
+    """Every row and permutation entry of the batch is written; nothing past the batch is."""
+    imgs = workloads.random_small_batch(13, 9, max_side=250)
+    params = mimo.make_params(workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    packed = mimo.pack_images(imgs, device="cuda")
+    grid, offs = mimo.plan_batch(packed.heights, packed.widths, params)
+    total = int(offs[-1])
+    for dtype in (torch.float32, torch.bfloat16):
+        out = torch.full((total + 37, 1536), float("nan"), dtype=dtype, device="cuda")
+        perm = torch.full((total + 37,), -7, dtype=torch.int32, device="cuda")
+        mimo.preprocess_batch(params, packed, out, perm)
+        torch.cuda.synchronize()
+        assert not torch.isnan(out[:total]).any()
+        assert torch.isnan(out[total:]).all()
+        assert (perm[total:] == -7).all()
+        assert torch.equal(torch.sort(perm[:total]).values, torch.arange(total, device="cuda", dtype=torch.int32))
+
+
+def test_empty_batch():
+    pv, grid, perm = mimo.preprocess([], workloads.IMAGENET_MEAN, workloads.IMAGENET_STD, column_perm=True)
+    assert pv.shape == (0, 1536) and grid.shape == (0, 3) and perm.shape == (0,)
+
+
+def test_nested_input_flattens_one_level():
+    imgs = workloads.random_small_batch(14, 3, max_side=120)
+    a, ga, _ = gpu_run(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    b, gb, _ = gpu_run([[imgs[0]], [imgs[1], imgs[2]]], workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    assert torch.equal(a, b) and np.array_equal(ga, gb)
+
+
+def test_device_resident_inputs_and_streams():
+    imgs = workloads.random_small_batch(15, 5, max_side=200)
+    ref, _, _ = gpu_run(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        dev_imgs = [torch.from_numpy(im).cuda() for im in imgs]
+        out, _, _ = mimo.preprocess(dev_imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    s.synchronize()
+    assert torch.equal(out, ref)
+
+
+def test_host_buffer_entry_point_matches_device_path():
+    w = workloads.workload("c5", n_images=5)
+    params = mimo.make_params(w["mean"], w["std"])
+    for dtype in (torch.float32, torch.bfloat16):
+        ref, _, rperm = gpu_run(w["images"], w["mean"], w["std"], dtype=dtype, column_perm=True)
+        host = mimo.pack_images(w["images"], device="cpu", pin_memory=True)
+        _, offs = mimo.plan_batch(host.heights, host.widths, params)
+        total = int(offs[-1])
+        out_h = torch.empty((total, 1536), dtype=dtype, pin_memory=True)
+        perm_h = torch.empty(total, dtype=torch.int32, pin_memory=True)
+        src_d = torch.empty_like(host.buffer, device="cuda")
+        out_d = torch.empty((total, 1536), dtype=dtype, device="cuda")
+        perm_d = torch.empty(total, dtype=torch.int32, device="cuda")
+        mimo.preprocess_batch_host(params, host, out_h, perm_h, src_d, out_d, perm_d)
+        assert torch.equal(out_h, ref.cpu()) and torch.equal(perm_h, rperm.cpu())
+
+
+def test_device_validation_errors():
+    imgs = workloads.random_small_batch(16, 2, max_side=100)
+    params = mimo.make_params()
+    packed = mimo.pack_images(imgs, device="cuda")
+    _, offs = mimo.plan_batch(packed.heights, packed.widths, params)
+    total = int(offs[-1])
+    out = torch.empty((total, 1536), device="cuda")
+    with pytest.raises(mimo.MimoError) as e:
+        mimo.preprocess_batch(params, packed, out[: total - 1])
+    assert e.value.status == 7
+    bad = mimo.PackedBatch(packed.buffer[: packed.buffer.numel() - 16], packed.offsets, packed.heights,
+                           packed.widths, packed.channels)
+    with pytest.raises(mimo.MimoError) as e:
+        mimo.preprocess_batch(params, bad, out)
+    assert e.value.status == 10
+    wide = torch.empty((total + 1) * 1536 + 1, device="cuda")
+    shifted = wide[1:1 + total * 1536].view(total, 1536)  # starts 4 bytes past a 16-byte boundary
+    with pytest.raises(mimo.MimoError) as e:
+        mimo.preprocess_batch(params, packed, shifted)
+    assert e.value.status == 6

@@ -1,0 +1,417 @@
+// mimo_api.cpp -- host side of the C ABI declared in include/mimo.h:
+// geometry (smart_resize), batch planning, argument validation, per-launch
+// descriptor blocks and the host-memory pipeline. All pixel work happens in
+// the CUDA kernel (mimo_preprocess.cu).
+#include "mimo.h"
+
+#include <cuda_runtime_api.h>
+
+#include <algorithm>
+#include <cfenv>
+#include <cmath>
+#include <cstring>
+#include <limits>
+#include <vector>
+
+#include "mimo_internal.h"
+
+namespace {
+
+constexpr int64_t kFactor = mimo::kBlock;  // patch 16 x merge 2
+
+bool supported_knobs(const mimo_params *p) {
+    return p->patch_size == 16 && p->temporal_patch_size == 2 && p->merge_size == 2 && p->reserved == 0;
+}
+
+int check_params(const mimo_params *p) {
+    if (!p) return MIMO_EINVAL;
+    if (p->min_pixels < 0 || p->max_pixels <= 0) return MIMO_EINVAL;
+    if (!supported_knobs(p)) return MIMO_EUNSUPPORTED;
+    for (int c = 0; c < 3; ++c) {
+        if (!std::isfinite(p->image_mean[c]) || !std::isfinite(p->image_std[c]) || !(p->image_std[c] > 0.f))
+            return MIMO_EUNSUPPORTED;
+    }
+    return MIMO_OK;
+}
+
+// Nearest integer with ties to even (the default IEEE rounding mode), the
+// behaviour of Python's round() on the processor's float quotients.
+double round_ties_even(double v) {
+    const int saved = std::fegetround();
+    if (saved != FE_TONEAREST) std::fesetround(FE_TONEAREST);
+    const double r = std::nearbyint(v);
+    if (saved != FE_TONEAREST) std::fesetround(saved);
+    return r;
+}
+
+// smart_resize of the processing page: sub-factor upscale first (no aspect
+// guard in that branch), else the HF aspect guard; round to the factor; then
+// the max_pixels shrink (floor, zero side rejected) or min_pixels growth (ceil).
+int smart_resize_impl(int64_t height, int64_t width, int64_t factor, int64_t min_px, int64_t max_px,
+                      int64_t *oh, int64_t *ow) {
+    if (height <= 0 || width <= 0 || factor <= 0 || min_px < 0 || max_px <= 0 || !oh || !ow) return MIMO_EINVAL;
+    // sizes whose products could overflow the exact-integer steps below
+    const int64_t lim = int64_t(1) << 31;
+    if (height >= lim || width >= lim || factor >= lim) return MIMO_EOVERFLOW;
+
+    const double f = static_cast<double>(factor);
+    double h, w;
+    const int64_t short_side = std::min(height, width);
+    if (short_side < factor) {
+        // both sides scaled by factor/short: the short side lands exactly on the factor
+        if (height == short_side) {
+            h = f;
+            w = static_cast<double>(width * factor) / static_cast<double>(height);
+        } else {
+            w = f;
+            h = static_cast<double>(height * factor) / static_cast<double>(width);
+        }
+    } else {
+        const double ratio = static_cast<double>(std::max(height, width)) / static_cast<double>(short_side);
+        if (ratio > 200.0) return MIMO_EASPECT;
+        h = static_cast<double>(height);
+        w = static_cast<double>(width);
+    }
+
+    double hb = round_ties_even(h / f) * f;
+    double wb = round_ties_even(w / f) * f;
+    const double area = hb * wb;
+    if (area > static_cast<double>(max_px)) {
+        const double beta = std::sqrt((h * w) / static_cast<double>(max_px));
+        hb = std::floor(h / beta / f) * f;
+        wb = std::floor(w / beta / f) * f;
+        if (hb <= 0.0 || wb <= 0.0) return MIMO_EDEGENERATE;
+    } else if (area < static_cast<double>(min_px)) {
+        const double beta = std::sqrt(static_cast<double>(min_px) / (h * w));
+        hb = std::ceil(h * beta / f) * f;
+        wb = std::ceil(w * beta / f) * f;
+    }
+    if (hb > 9.0e15 || wb > 9.0e15) return MIMO_EOVERFLOW;
+    *oh = static_cast<int64_t>(hb);
+    *ow = static_cast<int64_t>(wb);
+    return MIMO_OK;
+}
+
+// Geometry of one image for the kernel, or a status.
+struct ImagePlan {
+    int64_t Hr, Wr, rows, blocks;
+    int32_t flags;
+    int32_t tile_rows, tile_cols;
+};
+
+int64_t axis_max_span(int64_t in, int64_t out) {
+    int64_t span = 0;
+    for (int64_t b = 0; b < out / mimo::kBlock; ++b) span = std::max(span, mimo::block_span(b, in, out));
+    return span;
+}
+
+int plan_image(int64_t H, int64_t W, const mimo_params *p, ImagePlan *ip) {
+    int64_t Hr = 0, Wr = 0;
+    const int st = smart_resize_impl(H, W, kFactor, p->min_pixels, p->max_pixels, &Hr, &Wr);
+    if (st != MIMO_OK) return st;
+    if (Hr > INT32_MAX || Wr > INT32_MAX) return MIMO_EOVERFLOW;
+    ip->Hr = Hr;
+    ip->Wr = Wr;
+    ip->rows = (Hr / 16) * (Wr / 16);
+    ip->blocks = (Hr / mimo::kBlock) * (Wr / mimo::kBlock);
+    if (ip->blocks > INT32_MAX / 2) return MIMO_EOVERFLOW;
+    ip->flags = 0;
+    const int64_t rs = axis_max_span(H, Hr), cs = axis_max_span(W, Wr);
+    if (rs > mimo::kMaxTile) {
+        ip->flags |= mimo::kGatherRows;
+        ip->tile_rows = mimo::kMaxTile;
+    } else {
+        ip->tile_rows = static_cast<int32_t>(rs);
+    }
+    if (cs > mimo::kMaxTile) {
+        ip->flags |= mimo::kGatherCols;
+        ip->tile_cols = mimo::kMaxTile;
+    } else {
+        ip->tile_cols = static_cast<int32_t>(cs);
+    }
+    return MIMO_OK;
+}
+
+struct BatchPlan {
+    std::vector<ImagePlan> img;
+    std::vector<int64_t> row0;  // n + 1
+};
+
+int plan_all(int32_t n, const int32_t *heights, const int32_t *widths, const mimo_params *p, BatchPlan *bp) {
+    bp->img.resize(static_cast<size_t>(n));
+    bp->row0.assign(static_cast<size_t>(n) + 1, 0);
+    for (int32_t i = 0; i < n; ++i) {
+        if (heights[i] <= 0 || widths[i] <= 0) return MIMO_EINVAL;
+        const int st = plan_image(heights[i], widths[i], p, &bp->img[i]);
+        if (st != MIMO_OK) return st;
+        if (bp->row0[i] > std::numeric_limits<int64_t>::max() / 2) return MIMO_EOVERFLOW;
+        bp->row0[i + 1] = bp->row0[i] + bp->img[i].rows;
+    }
+    return MIMO_OK;
+}
+
+bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+struct Validated {
+    BatchPlan plan;
+    int64_t total_rows = 0;
+};
+
+// Shared argument checks of the two batch entry points (device or host
+// buffers); `src`/`out`/`perm` are whatever the call will read and write.
+int validate_batch(const mimo_params *p, int32_t n, const void *src, size_t src_bytes, const int64_t *src_offsets,
+                   const int32_t *heights, const int32_t *widths, const int32_t *channels, int32_t out_dtype,
+                   const void *out, int64_t out_rows_capacity, const void *perm, Validated *v) {
+    int st = check_params(p);
+    if (st != MIMO_OK) return st;
+    if (n < 0) return MIMO_EINVAL;
+    if (out_dtype != MIMO_F32 && out_dtype != MIMO_BF16) return MIMO_EINVAL;
+    if (n == 0) return MIMO_OK;
+    if (!src || !src_offsets || !heights || !widths || !channels) return MIMO_EINVAL;
+    for (int32_t i = 0; i < n; ++i) {
+        if (channels[i] != 3 && channels[i] != 4) return MIMO_ECHANNELS;
+        if (src_offsets[i] < 0) return MIMO_EINVAL;
+        if ((src_offsets[i] & 15) != 0) return MIMO_EALIGN;
+    }
+    if (!aligned16(src)) return MIMO_EALIGN;
+    st = plan_all(n, heights, widths, p, &v->plan);
+    if (st != MIMO_OK) return st;
+    for (int32_t i = 0; i < n; ++i) {
+        const uint64_t bytes = static_cast<uint64_t>(heights[i]) * static_cast<uint64_t>(widths[i]) *
+                               static_cast<uint64_t>(channels[i]);
+        const uint64_t off = static_cast<uint64_t>(src_offsets[i]);
+        if (off > src_bytes || bytes > src_bytes - off) return MIMO_ERANGE;
+    }
+    v->total_rows = v->plan.row0[n];
+    if (v->total_rows > out_rows_capacity) return MIMO_ECAPACITY;
+    if (!out) return MIMO_EINVAL;
+    if (!aligned16(out)) return MIMO_EALIGN;
+    if (perm) {
+        if (!aligned16(perm)) return MIMO_EALIGN;
+        if (v->total_rows > INT32_MAX) return MIMO_EOVERFLOW;
+    }
+    return MIMO_OK;
+}
+
+void fold_normalisation(const mimo_params *p, mimo::LaunchParams *lp) {
+    for (int c = 0; c < 3; ++c) {
+        const double s = 255.0 * static_cast<double>(p->image_std[c]);
+        const double m = 255.0 * static_cast<double>(p->image_mean[c]);
+        lp->k[c] = static_cast<float>(1.0 / s);
+        lp->b[c] = static_cast<float>(-m / s);
+    }
+}
+
+// Launches images [first, last) of a validated batch, cut into launches of at
+// most kMaxImagesPerLaunch images and INT32_MAX blocks. Output rows and
+// source offsets stay batch-global.
+int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_t last, const uint8_t *d_src,
+                 const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
+                 const int32_t *channels, int32_t out_dtype, void *d_out, int32_t *d_perm, void *stream) {
+    static thread_local mimo::LaunchParams lp;  // 23 KB: kept off the stack
+    int32_t i = first;
+    while (i < last) {
+        std::memset(&lp, 0, sizeof(lp));
+        lp.src = d_src;
+        lp.out = d_out;
+        lp.perm = d_perm;
+        fold_normalisation(p, &lp);
+        int64_t blocks = 0;
+        int32_t tr = 1, tc = 1, k = 0;
+        while (i < last && k < mimo::kMaxImagesPerLaunch &&
+               blocks + v.plan.img[i].blocks <= static_cast<int64_t>(INT32_MAX)) {
+            const ImagePlan &ip = v.plan.img[i];
+            mimo::ImageDesc &d = lp.img[k];
+            d.src_off = src_offsets[i];
+            d.row0 = v.plan.row0[i];
+            d.H = heights[i];
+            d.W = widths[i];
+            d.Hr = static_cast<int32_t>(ip.Hr);
+            d.Wr = static_cast<int32_t>(ip.Wr);
+            d.C = channels[i];
+            d.flags = ip.flags;
+            lp.block_start[k] = static_cast<int32_t>(blocks);
+            blocks += ip.blocks;
+            tr = std::max(tr, ip.tile_rows);
+            tc = std::max(tc, ip.tile_cols);
+            ++k;
+            ++i;
+        }
+        lp.block_start[k] = static_cast<int32_t>(blocks);
+        lp.n = k;
+        lp.tile_rows = tr;
+        lp.tile_stride = tc | 1;  // odd stride: consecutive tile rows start in different banks
+        const size_t smem = sizeof(float) * 3u * static_cast<size_t>(tr) * static_cast<size_t>(lp.tile_stride);
+        const int st = mimo::launch_preprocess(lp, blocks, out_dtype, smem, stream);
+        if (st != MIMO_OK) return st;
+    }
+    return MIMO_OK;
+}
+
+size_t dtype_bytes(int32_t out_dtype) { return out_dtype == MIMO_BF16 ? 2u : 4u; }
+
+}  // namespace
+
+extern "C" {
+
+void mimo_params_default(mimo_params *p) {
+    if (!p) return;
+    std::memset(p, 0, sizeof(*p));
+    p->patch_size = 16;
+    p->temporal_patch_size = 2;
+    p->merge_size = 2;
+    p->min_pixels = 8192;
+    p->max_pixels = 8388608;
+    const float mean[3] = {0.485f, 0.456f, 0.406f};
+    const float stdv[3] = {0.229f, 0.224f, 0.225f};
+    for (int c = 0; c < 3; ++c) {
+        p->image_mean[c] = mean[c];
+        p->image_std[c] = stdv[c];
+    }
+}
+
+int mimo_smart_resize(int64_t height, int64_t width, int64_t factor, int64_t min_pixels, int64_t max_pixels,
+                      int64_t *out_height, int64_t *out_width) {
+    return smart_resize_impl(height, width, factor, min_pixels, max_pixels, out_height, out_width);
+}
+
+int mimo_num_patches(int64_t height, int64_t width, const mimo_params *p, int64_t *out_patches) {
+    if (!p || !out_patches) return MIMO_EINVAL;
+    if (p->patch_size <= 0 || p->merge_size <= 0) return MIMO_EINVAL;
+    int64_t oh = 0, ow = 0;
+    const int64_t factor = static_cast<int64_t>(p->patch_size) * p->merge_size;
+    const int st = smart_resize_impl(height, width, factor, p->min_pixels, p->max_pixels, &oh, &ow);
+    if (st != MIMO_OK) return st;
+    *out_patches = (oh / p->patch_size) * (ow / p->patch_size);
+    return MIMO_OK;
+}
+
+int mimo_plan_batch(int32_t n, const int32_t *heights, const int32_t *widths, const mimo_params *p,
+                    int64_t *grid_thw, int64_t *row_offsets) {
+    const int st0 = check_params(p);
+    if (st0 != MIMO_OK) return st0;
+    if (n < 0 || !row_offsets) return MIMO_EINVAL;
+    if (n > 0 && (!heights || !widths || !grid_thw)) return MIMO_EINVAL;
+    BatchPlan bp;
+    const int st = plan_all(n, heights, widths, p, &bp);
+    if (st != MIMO_OK) return st;
+    for (int32_t i = 0; i < n; ++i) {
+        grid_thw[3 * i + 0] = 1;
+        grid_thw[3 * i + 1] = bp.img[i].Hr / 16;
+        grid_thw[3 * i + 2] = bp.img[i].Wr / 16;
+    }
+    std::memcpy(row_offsets, bp.row0.data(), sizeof(int64_t) * (static_cast<size_t>(n) + 1));
+    return MIMO_OK;
+}
+
+int mimo_preprocess_batch(const mimo_params *p, int32_t n, const uint8_t *d_src, size_t src_bytes,
+                          const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
+                          const int32_t *channels, int32_t out_dtype, void *d_out, int64_t out_rows_capacity,
+                          int32_t *d_column_perm, void *stream) {
+    Validated v;
+    const int st = validate_batch(p, n, d_src, src_bytes, src_offsets, heights, widths, channels, out_dtype, d_out,
+                                  out_rows_capacity, d_column_perm, &v);
+    if (st != MIMO_OK || n == 0) return st;
+    return launch_range(p, v, 0, n, d_src, src_offsets, heights, widths, channels, out_dtype, d_out,
+                        d_column_perm, stream);
+}
+
+int mimo_preprocess_batch_host(const mimo_params *p, int32_t n, const uint8_t *h_src, size_t src_bytes,
+                               const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
+                               const int32_t *channels, int32_t out_dtype, void *h_out, int64_t out_rows_capacity,
+                               int32_t *h_column_perm, uint8_t *d_src_stage, size_t d_src_stage_bytes,
+                               void *d_out_stage, int64_t d_out_stage_rows, int32_t *d_perm_stage, void *stream) {
+    Validated v;
+    int st = validate_batch(p, n, h_src, src_bytes, src_offsets, heights, widths, channels, out_dtype, h_out,
+                            out_rows_capacity, h_column_perm, &v);
+    if (st != MIMO_OK || n == 0) return st;
+    if (!d_src_stage || !d_out_stage) return MIMO_EINVAL;
+    if (!aligned16(d_src_stage) || !aligned16(d_out_stage)) return MIMO_EALIGN;
+    if (d_src_stage_bytes < src_bytes || d_out_stage_rows < v.total_rows) return MIMO_ECAPACITY;
+    if (h_column_perm && (!d_perm_stage || !aligned16(d_perm_stage))) return d_perm_stage ? MIMO_EALIGN : MIMO_EINVAL;
+
+    const size_t row_bytes = static_cast<size_t>(mimo::kRowWidth) * dtype_bytes(out_dtype);
+    cudaStream_t caller = static_cast<cudaStream_t>(stream);
+
+    // Chunks of whole images of roughly equal output size; each chunk's
+    // upload -> kernel -> download runs in order on one of two streams, so
+    // one chunk's download overlaps the next chunk's upload and kernel.
+    const int64_t target_chunks = std::min<int64_t>(n, 8);
+    const int64_t rows_per_chunk = std::max<int64_t>(1, (v.total_rows + target_chunks - 1) / target_chunks);
+
+    cudaStream_t ss[2] = {nullptr, nullptr};
+    cudaEvent_t start = nullptr;
+    int result = MIMO_OK;
+    auto fail = [&](cudaError_t e) {
+        if (e != cudaSuccess && result == MIMO_OK) result = MIMO_ECUDA;
+        return e != cudaSuccess;
+    };
+    if (fail(cudaStreamCreateWithFlags(&ss[0], cudaStreamNonBlocking)) ||
+        fail(cudaStreamCreateWithFlags(&ss[1], cudaStreamNonBlocking)) ||
+        fail(cudaEventCreateWithFlags(&start, cudaEventDisableTiming)) || fail(cudaEventRecord(start, caller)) ||
+        fail(cudaStreamWaitEvent(ss[0], start, 0)) || fail(cudaStreamWaitEvent(ss[1], start, 0))) {
+        // fall through to cleanup
+    } else {
+        int32_t i = 0;
+        int chunk = 0;
+        while (i < n && result == MIMO_OK) {
+            const int32_t first = i;
+            int64_t rows = 0;
+            uint64_t lo = UINT64_MAX, hi = 0;
+            while (i < n && (rows == 0 || rows + v.plan.img[i].rows <= rows_per_chunk)) {
+                rows += v.plan.img[i].rows;
+                const uint64_t off = static_cast<uint64_t>(src_offsets[i]);
+                lo = std::min(lo, off);
+                hi = std::max(hi, off + static_cast<uint64_t>(heights[i]) * widths[i] * channels[i]);
+                ++i;
+            }
+            cudaStream_t s = ss[chunk & 1];
+            const int64_t r0 = v.plan.row0[first];
+            if (fail(cudaMemcpyAsync(d_src_stage + lo, h_src + lo, hi - lo, cudaMemcpyHostToDevice, s))) break;
+            const int lst = launch_range(p, v, first, i, d_src_stage, src_offsets, heights, widths, channels,
+                                         out_dtype, d_out_stage, h_column_perm ? d_perm_stage : nullptr, s);
+            if (lst != MIMO_OK) {
+                result = lst;
+                break;
+            }
+            if (fail(cudaMemcpyAsync(static_cast<char *>(h_out) + static_cast<size_t>(r0) * row_bytes,
+                                     static_cast<char *>(d_out_stage) + static_cast<size_t>(r0) * row_bytes,
+                                     static_cast<size_t>(rows) * row_bytes, cudaMemcpyDeviceToHost, s)))
+                break;
+            if (h_column_perm &&
+                fail(cudaMemcpyAsync(h_column_perm + r0, d_perm_stage + r0, sizeof(int32_t) * rows,
+                                     cudaMemcpyDeviceToHost, s)))
+                break;
+            ++chunk;
+        }
+    }
+    for (cudaStream_t s : ss) {
+        if (s) {
+            fail(cudaStreamSynchronize(s));
+            cudaStreamDestroy(s);
+        }
+    }
+    if (start) cudaEventDestroy(start);
+    return result;
+}
+
+const char *mimo_status_string(int status) {
+    switch (status) {
+        case MIMO_OK: return "ok";
+        case MIMO_EINVAL: return "invalid argument";
+        case MIMO_EASPECT: return "absolute aspect ratio must be at most 200";
+        case MIMO_EDEGENERATE: return "max_pixels shrink rounds a side down to zero";
+        case MIMO_ECHANNELS: return "channels must be 3 (RGB) or 4 (RGBA)";
+        case MIMO_EUNSUPPORTED: return "unsupported processor knobs (patch 16, temporal 2, merge 2, std > 0)";
+        case MIMO_EALIGN: return "source offsets and output pointers must be 16-byte aligned";
+        case MIMO_ECAPACITY: return "output or staging buffer too small for the batch";
+        case MIMO_EOVERFLOW: return "size exceeds the supported index range";
+        case MIMO_ECUDA: return "CUDA runtime error";
+        case MIMO_ERANGE: return "an image lies outside the source buffer";
+        default: return "unknown status";
+    }
+}
+
+int mimo_version(void) { return 10000; }
+
+}  // extern "C"

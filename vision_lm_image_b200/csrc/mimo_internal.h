@@ -1,0 +1,91 @@
+// mimo_internal.h -- types shared by the host planner (mimo_api.cpp) and the
+// sm_100a kernel (mimo_preprocess.cu). Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#if defined(__CUDACC__)
+#define MIMO_HD __host__ __device__ __forceinline__
+#else
+#define MIMO_HD inline
+#endif
+
+namespace mimo {
+
+// One 32x32 output merge block per CTA; the source samples it needs are
+// staged in shared memory as planar fp32 tiles of at most kMaxTile rows and
+// columns (2 taps x 32 outputs).
+constexpr int kBlock = 32;             // merge block side in resized pixels (patch 16 x merge 2)
+constexpr int kRowWidth = 1536;        // 3 channels x 2 frames x 16 x 16
+constexpr int kMaxTile = 64;           // 32 outputs x 2 taps
+constexpr int kThreads = 256;
+constexpr int kMaxImagesPerLaunch = 512;
+
+// Per-axis staging mode of an image, decided on the host from the scale:
+// contiguous = the block's source span (first tap to last tap) fits in
+// kMaxTile rows/cols and is staged whole; gathered = only the two taps of
+// each of the 32 outputs are staged (tile index 2*d and 2*d+1).
+enum : int32_t { kGatherRows = 1, kGatherCols = 2 };
+
+struct ImageDesc {
+    int64_t src_off;  // byte offset of the image in the packed source buffer
+    int64_t row0;     // first output row of the image in the batch
+    int32_t H, W;     // source size
+    int32_t Hr, Wr;   // resized size, multiples of 32
+    int32_t C;        // 3 or 4
+    int32_t flags;    // kGatherRows | kGatherCols
+};
+static_assert(sizeof(ImageDesc) == 40, "descriptor layout");
+
+// Everything one launch needs travels by value as the kernel's parameter
+// block (__grid_constant__), so a launch needs no device-side table and no
+// host-to-device copy.
+struct LaunchParams {
+    const uint8_t *src;
+    void *out;
+    int32_t *perm;       // may be null
+    float k[3], b[3];    // normalisation folded: v = x*k[c] + b[c]
+    int32_t n;           // images in this launch
+    int32_t tile_rows;   // rows of the shared-memory tile (max over images)
+    int32_t tile_stride; // odd row stride (floats) of the tile
+    int32_t pad_;
+    int32_t block_start[kMaxImagesPerLaunch + 1];  // prefix sum of merge blocks
+    ImageDesc img[kMaxImagesPerLaunch];
+};
+static_assert(sizeof(LaunchParams) <= 32764 - 64, "kernel parameter limit");
+
+// Bilinear taps of output index d along an axis of size in -> out under the
+// align_corners=False rule, computed exactly: the source coordinate is the
+// rational ((2d+1)*in - out) / (2*out), clamped at 0 from below.
+struct Taps {
+    int64_t i0, i1;
+    int64_t rem, den;  // weight of the second tap = rem / den
+};
+
+MIMO_HD Taps axis_taps(int64_t d, int64_t in, int64_t out) {
+    Taps t;
+    const int64_t num = (2 * d + 1) * in - out;
+    t.den = 2 * out;
+    if (num <= 0) {
+        t.i0 = 0;
+        t.rem = 0;
+    } else {
+        t.i0 = num / t.den;
+        t.rem = num - t.i0 * t.den;
+    }
+    t.i1 = (t.i0 + 1 < in) ? t.i0 + 1 : in - 1;
+    return t;
+}
+
+// Number of source rows (or columns) a merge block touches when staged
+// contiguously: last tap of output 32b+31 minus first tap of output 32b, + 1.
+MIMO_HD int64_t block_span(int64_t b, int64_t in, int64_t out) {
+    const Taps first = axis_taps(b * kBlock, in, out);
+    const Taps last = axis_taps(b * kBlock + kBlock - 1, in, out);
+    return last.i1 - first.i0 + 1;
+}
+
+int launch_preprocess(const LaunchParams &lp, int64_t blocks, int out_dtype, size_t smem_bytes, void *stream);
+
+}  // namespace mimo

@@ -1,0 +1,303 @@
+"""Python binding of the C ABI in include/mimo.h (argument marshalling only).
+
+Every step of the pixel path runs in the CUDA library ``libmimo_b200.so``;
+this module only packs images into one buffer, allocates outputs with torch
+on the caller's device and stream, and passes pointers and sizes. If the
+library is missing, every call raises :class:`MimoLibraryMissing`: there is
+no CPU fallback.
+
+The user-level call mirrors ``MimoV2ImageProcessor.__call__`` (NeMo Automodel,
+"mimo_v2_flash.processing"): images (HWC uint8, RGB or RGBA; one nesting level
+is flattened) go in, ``pixel_values [total_patches, 1536]`` and
+``image_grid_thw [n, 3]`` come out, plus the optional column-order
+permutation (docs.rs "cortiq_engine::mimo_vision", column_permutation).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Iterable, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+OK = 0
+F32, BF16 = 0, 1
+ROW_WIDTH = 1536
+ALIGN = 16
+
+STATUS_NAMES = {
+    0: "MIMO_OK", 1: "MIMO_EINVAL", 2: "MIMO_EASPECT", 3: "MIMO_EDEGENERATE", 4: "MIMO_ECHANNELS",
+    5: "MIMO_EUNSUPPORTED", 6: "MIMO_EALIGN", 7: "MIMO_ECAPACITY", 8: "MIMO_EOVERFLOW", 9: "MIMO_ECUDA",
+    10: "MIMO_ERANGE",
+}
+EXPORTED = ("mimo_params_default", "mimo_smart_resize", "mimo_num_patches", "mimo_plan_batch",
+            "mimo_preprocess_batch", "mimo_preprocess_batch_host", "mimo_status_string", "mimo_version")
+
+
+class MimoLibraryMissing(RuntimeError):
+    pass
+
+
+class MimoError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        msg = _lib_status_string(status)
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}{(' (' + what + ')') if what else ''}")
+        self.status = status
+
+
+class MimoParams(ctypes.Structure):
+    _fields_ = [
+        ("patch_size", ctypes.c_int32),
+        ("temporal_patch_size", ctypes.c_int32),
+        ("merge_size", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("min_pixels", ctypes.c_int64),
+        ("max_pixels", ctypes.c_int64),
+        ("image_mean", ctypes.c_float * 3),
+        ("image_std", ctypes.c_float * 3),
+    ]
+
+
+_i32, _i64, _p, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+_lib = None
+_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = library_path()
+            if not os.path.exists(path):
+                raise MimoLibraryMissing(
+                    f"{path} is missing: build it with `python -m vision_lm_image_b200.build` "
+                    "(or __graft_entry__.build()); there is no fallback path")
+            L = ctypes.CDLL(path)
+            L.mimo_params_default.argtypes = [ctypes.POINTER(MimoParams)]
+            L.mimo_params_default.restype = None
+            L.mimo_smart_resize.argtypes = [_i64, _i64, _i64, _i64, _i64, ctypes.POINTER(_i64), ctypes.POINTER(_i64)]
+            L.mimo_smart_resize.restype = ctypes.c_int
+            L.mimo_num_patches.argtypes = [_i64, _i64, ctypes.POINTER(MimoParams), ctypes.POINTER(_i64)]
+            L.mimo_num_patches.restype = ctypes.c_int
+            L.mimo_plan_batch.argtypes = [_i32, _p, _p, ctypes.POINTER(MimoParams), _p, _p]
+            L.mimo_plan_batch.restype = ctypes.c_int
+            L.mimo_preprocess_batch.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p, _i32,
+                                                _p, _i64, _p, _p]
+            L.mimo_preprocess_batch.restype = ctypes.c_int
+            L.mimo_preprocess_batch_host.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p,
+                                                     _i32, _p, _i64, _p, _p, _sz, _p, _i64, _p, _p]
+            L.mimo_preprocess_batch_host.restype = ctypes.c_int
+            L.mimo_status_string.argtypes = [ctypes.c_int]
+            L.mimo_status_string.restype = ctypes.c_char_p
+            L.mimo_version.argtypes = []
+            L.mimo_version.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _lib_status_string(status: int) -> str:
+    try:
+        return lib().mimo_status_string(status).decode()
+    except MimoLibraryMissing:
+        return "library missing"
+
+
+def _check(status: int, what: str = ""):
+    if status != OK:
+        raise MimoError(status, what)
+
+
+# ----------------------------------------------------------------- knobs
+def make_params(mean=None, std=None, min_pixels: int | None = None, max_pixels: int | None = None,
+                patch_size: int = 16, temporal_patch_size: int = 2, merge_size: int = 2) -> MimoParams:
+    p = MimoParams()
+    lib().mimo_params_default(ctypes.byref(p))
+    p.patch_size, p.temporal_patch_size, p.merge_size = patch_size, temporal_patch_size, merge_size
+    if min_pixels is not None:
+        p.min_pixels = int(min_pixels)
+    if max_pixels is not None:
+        p.max_pixels = int(max_pixels)
+    if mean is not None:
+        for c in range(3):
+            p.image_mean[c] = float(mean[c])
+    if std is not None:
+        for c in range(3):
+            p.image_std[c] = float(std[c])
+    return p
+
+
+# ----------------------------------------------------------------- host-only geometry
+def smart_resize(height: int, width: int, factor: int = 32, min_pixels: int = 8192,
+                 max_pixels: int = 8388608) -> tuple[int, int]:
+    oh, ow = _i64(), _i64()
+    _check(lib().mimo_smart_resize(height, width, factor, min_pixels, max_pixels, ctypes.byref(oh),
+                                   ctypes.byref(ow)), f"smart_resize({height}, {width})")
+    return oh.value, ow.value
+
+
+def smart_resize_status(height: int, width: int, factor: int = 32, min_pixels: int = 8192,
+                        max_pixels: int = 8388608) -> int:
+    oh, ow = _i64(), _i64()
+    return lib().mimo_smart_resize(height, width, factor, min_pixels, max_pixels, ctypes.byref(oh), ctypes.byref(ow))
+
+
+def get_number_of_image_patches(height: int, width: int, params: MimoParams | None = None) -> int:
+    p = params if params is not None else make_params()
+    out = _i64()
+    _check(lib().mimo_num_patches(height, width, ctypes.byref(p), ctypes.byref(out)))
+    return out.value
+
+
+def plan_batch(heights: Sequence[int], widths: Sequence[int], params: MimoParams | None = None):
+    """(grid_thw int64 [n, 3], row_offsets int64 [n + 1])."""
+    p = params if params is not None else make_params()
+    n = len(heights)
+    h = np.ascontiguousarray(heights, dtype=np.int32)
+    w = np.ascontiguousarray(widths, dtype=np.int32)
+    grid = np.zeros((n, 3), np.int64)
+    offs = np.zeros(n + 1, np.int64)
+    _check(lib().mimo_plan_batch(n, h.ctypes.data, w.ctypes.data, ctypes.byref(p), grid.ctypes.data,
+                                 offs.ctypes.data), "plan_batch")
+    return grid, offs
+
+
+# ----------------------------------------------------------------- packing
+def _flatten_one_level(images):
+    flat = []
+    for item in images:
+        if isinstance(item, (list, tuple)):
+            flat.extend(item)
+        else:
+            flat.append(item)
+    return flat
+
+
+def packed_layout(shapes: Iterable[tuple[int, int, int]]):
+    """Byte offsets (16-byte aligned) of HWC images packed back to back, and the total size."""
+    offsets, pos = [], 0
+    for (h, w, c) in shapes:
+        offsets.append(pos)
+        pos += h * w * c
+        pos = (pos + ALIGN - 1) // ALIGN * ALIGN
+    return np.asarray(offsets, np.int64), max(pos, ALIGN)
+
+
+class PackedBatch:
+    """Images packed into one uint8 buffer (host or device) with their sizes."""
+
+    def __init__(self, buffer, offsets, heights, widths, channels):
+        self.buffer = buffer  # torch uint8 tensor
+        self.offsets = np.ascontiguousarray(offsets, np.int64)
+        self.heights = np.ascontiguousarray(heights, np.int32)
+        self.widths = np.ascontiguousarray(widths, np.int32)
+        self.channels = np.ascontiguousarray(channels, np.int32)
+
+    @property
+    def n(self) -> int:
+        return int(self.heights.shape[0])
+
+    def to(self, device, non_blocking: bool = False) -> "PackedBatch":
+        return PackedBatch(self.buffer.to(device, non_blocking=non_blocking), self.offsets, self.heights,
+                           self.widths, self.channels)
+
+
+def pack_images(images, device="cpu", pin_memory: bool = False) -> PackedBatch:
+    import torch
+
+    imgs = _flatten_one_level(images)
+    shapes = []
+    for im in imgs:
+        if im.ndim != 3:
+            raise ValueError("images must be HWC uint8 arrays")
+        shapes.append(tuple(int(s) for s in im.shape))
+    offsets, total = packed_layout(shapes)
+    dev = torch.device(device)
+    buf = torch.empty(total, dtype=torch.uint8, device=dev,
+                      pin_memory=(pin_memory and dev.type == "cpu"))
+    for im, off, (h, w, c) in zip(imgs, offsets.tolist(), shapes):
+        t = im if isinstance(im, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(im, dtype=np.uint8))
+        if t.dtype != torch.uint8:
+            raise ValueError("images must be uint8")
+        buf[off:off + h * w * c].copy_(t.reshape(-1), non_blocking=True)
+    return PackedBatch(buf, offsets, [s[0] for s in shapes], [s[1] for s in shapes], [s[2] for s in shapes])
+
+
+# ----------------------------------------------------------------- device path
+def _stream_handle(stream, device):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def preprocess_batch(params: MimoParams, packed: PackedBatch, out, perm=None, stream=None) -> None:
+    """Raw ABI call on device buffers (``packed.buffer``, ``out`` and ``perm`` on the same CUDA device)."""
+    buf = packed.buffer
+    st = lib().mimo_preprocess_batch(
+        ctypes.byref(params), packed.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
+        packed.offsets.ctypes.data, packed.heights.ctypes.data, packed.widths.ctypes.data,
+        packed.channels.ctypes.data, _dtype_code(out.dtype), ctypes.c_void_p(out.data_ptr()),
+        out.shape[0] if out.ndim == 2 else 0, ctypes.c_void_p(perm.data_ptr() if perm is not None else 0),
+        _stream_handle(stream, buf.device))
+    _check(st, "preprocess_batch")
+
+
+def _dtype_code(dtype) -> int:
+    import torch
+
+    if dtype == torch.float32:
+        return F32
+    if dtype == torch.bfloat16:
+        return BF16
+    raise ValueError(f"unsupported output dtype {dtype}")
+
+
+def preprocess(images, mean=None, std=None, min_pixels: int | None = None, max_pixels: int | None = None,
+               dtype=None, column_perm: bool = False, device="cuda", stream=None):
+    """The processor call on the GPU: returns (pixel_values, image_grid_thw, perm | None).
+
+    ``images``: HWC uint8 numpy arrays or torch tensors (CPU or CUDA), RGB or
+    RGBA, or a list of such lists (flattened one level). ``pixel_values`` is a
+    CUDA tensor [total_patches, 1536] (float32 by default, bfloat16 on
+    request); ``image_grid_thw`` a CPU int64 tensor [n, 3].
+    """
+    import torch
+
+    dtype = torch.float32 if dtype is None else dtype
+    dev = torch.device(device)
+    if dev.type != "cuda":
+        raise ValueError("the MiMo preprocessing library runs on CUDA devices only")
+    params = make_params(mean, std, min_pixels, max_pixels)
+    packed = pack_images(images, device=dev)
+    grid, offs = plan_batch(packed.heights, packed.widths, params)
+    total = int(offs[-1])
+    out = torch.empty((total, ROW_WIDTH), dtype=dtype, device=dev)
+    perm = torch.empty(total, dtype=torch.int32, device=dev) if column_perm else None
+    preprocess_batch(params, packed, out, perm, stream)
+    return out, torch.from_numpy(grid), perm
+
+
+# ----------------------------------------------------------------- host-to-host path
+def preprocess_batch_host(params: MimoParams, packed_host: PackedBatch, out_host, perm_host, src_stage,
+                          out_stage, perm_stage=None, stream=None) -> None:
+    """Raw ABI call of mimo_preprocess_batch_host: host input and output buffers (pinned for full
+    bandwidth), caller-provided device staging buffers. Returns when ``out_host`` is filled."""
+    buf = packed_host.buffer
+    st = lib().mimo_preprocess_batch_host(
+        ctypes.byref(params), packed_host.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
+        packed_host.offsets.ctypes.data, packed_host.heights.ctypes.data, packed_host.widths.ctypes.data,
+        packed_host.channels.ctypes.data, _dtype_code(out_host.dtype), ctypes.c_void_p(out_host.data_ptr()),
+        out_host.shape[0], ctypes.c_void_p(perm_host.data_ptr() if perm_host is not None else 0),
+        ctypes.c_void_p(src_stage.data_ptr()), src_stage.numel(), ctypes.c_void_p(out_stage.data_ptr()),
+        out_stage.shape[0], ctypes.c_void_p(perm_stage.data_ptr() if perm_stage is not None else 0),
+        _stream_handle(stream, src_stage.device))
+    _check(st, "preprocess_batch_host")
