@@ -1,0 +1,80 @@
+"""Multi-rank sharding on CPU (gloo, world size 2): every image is taken by exactly one rank, the
+ranks agree on the assignment without exchanging it, row offsets stay batch-global, and the load
+is balanced within the LPT bound."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import workloads
+from vision_lm_image_b200 import build, shard
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, sizes, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        H = [h for h, _ in sizes]
+        W = [w for _, w in sizes]
+        assign, grid, offs = shard.shard_plan(H, W, world)
+        mine = assign[rank]
+        gathered = [None] * world
+        dist.all_gather_object(gathered, (rank, mine, offs.tolist()))
+        q.put(gathered if rank == 0 else None)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_lpt_two_ranks_gloo():
+    build.build()
+    rng = workloads.rng_for(99)
+    sizes = workloads.random_sizes(rng, 37) + [(16, 192), (4096, 4096), (1080, 1920)]
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, sizes, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = None
+    for _ in range(world):
+        item = q.get(timeout=120)
+        if item is not None:
+            res = item
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res is not None
+    sets = [set(m) for _, m, _ in res]
+    assert sets[0].isdisjoint(sets[1])
+    assert sets[0] | sets[1] == set(range(len(sizes)))
+    assert res[0][2] == res[1][2]  # identical global row offsets on both ranks
+    offs = np.array(res[0][2])
+    rows = np.diff(offs)
+    loads = [int(rows[list(s)].sum()) for s in sets]
+    assert max(loads) - min(loads) <= rows.max()  # LPT: imbalance below the largest item
+
+
+def test_lpt_properties():
+    rng = np.random.Generator(np.random.PCG64(3))
+    for world in (1, 2, 3, 8):
+        costs = rng.integers(1, 1000, size=50).tolist()
+        a = shard.lpt_assign(costs, world)
+        flat = sorted(i for part in a for i in part)
+        assert flat == list(range(50))
+        loads = [sum(costs[i] for i in part) for part in a]
+        assert max(loads) <= sum(costs) / world + max(costs)
+    assert shard.lpt_assign([], 4) == [[], [], [], []]
+    with pytest.raises(ValueError):
+        shard.lpt_assign([1], 0)

@@ -116,18 +116,31 @@ int plan_image(int64_t H, int64_t W, const mimo_params *p, ImagePlan *ip) {
     ip->blocks = (Hr / mimo::kBlock) * (Wr / mimo::kBlock);
     if (ip->blocks > INT32_MAX / 2) return MIMO_EOVERFLOW;
     ip->flags = 0;
-    const int64_t rs = axis_max_span(H, Hr), cs = axis_max_span(W, Wr);
-    if (rs > mimo::kMaxTile) {
-        ip->flags |= mimo::kGatherRows;
-        ip->tile_rows = mimo::kMaxTile;
+    // rows
+    if (Hr == H) {
+        ip->flags |= mimo::kIdentityRows;  // every weight is 0: only the first tap is staged
+        ip->tile_rows = mimo::kBlock;
     } else {
-        ip->tile_rows = static_cast<int32_t>(rs);
+        const int64_t rs = axis_max_span(H, Hr);
+        if (rs > mimo::kMaxTile) {
+            ip->flags |= mimo::kGatherRows;
+            ip->tile_rows = mimo::kMaxTile;
+        } else {
+            ip->tile_rows = static_cast<int32_t>(rs);
+        }
     }
-    if (cs > mimo::kMaxTile) {
-        ip->flags |= mimo::kGatherCols;
-        ip->tile_cols = mimo::kMaxTile;
+    // columns
+    if (Wr == W) {
+        ip->flags |= mimo::kIdentityCols;
+        ip->tile_cols = mimo::kBlock;
     } else {
-        ip->tile_cols = static_cast<int32_t>(cs);
+        const int64_t cs = axis_max_span(W, Wr);
+        if (cs > mimo::kMaxTile) {
+            ip->flags |= mimo::kGatherCols;
+            ip->tile_cols = mimo::kMaxTile;
+        } else {
+            ip->tile_cols = static_cast<int32_t>(cs);
+        }
     }
     return MIMO_OK;
 }
@@ -206,7 +219,7 @@ void fold_normalisation(const mimo_params *p, mimo::LaunchParams *lp) {
 // most kMaxImagesPerLaunch images and INT32_MAX blocks. Output rows and
 // source offsets stay batch-global.
 int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_t last, const uint8_t *d_src,
-                 const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
+                 size_t src_bytes, const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
                  const int32_t *channels, int32_t out_dtype, void *d_out, int32_t *d_perm, void *stream) {
     static thread_local mimo::LaunchParams lp;  // 23 KB: kept off the stack
     int32_t i = first;
@@ -218,6 +231,7 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
         fold_normalisation(p, &lp);
         int64_t blocks = 0;
         int32_t tr = 1, tc = 1, k = 0;
+        bool hpass = false;
         while (i < last && k < mimo::kMaxImagesPerLaunch &&
                blocks + v.plan.img[i].blocks <= static_cast<int64_t>(INT32_MAX)) {
             const ImagePlan &ip = v.plan.img[i];
@@ -230,6 +244,11 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
             d.Wr = static_cast<int32_t>(ip.Wr);
             d.C = channels[i];
             d.flags = ip.flags;
+            // aligned 32-bit reads may round the image's last byte up to a word
+            // boundary; allow that only inside the caller's buffer
+            const int64_t bytes = static_cast<int64_t>(heights[i]) * widths[i] * channels[i];
+            d.readable = std::min<int64_t>((bytes + 3) & ~int64_t(3), static_cast<int64_t>(src_bytes) - src_offsets[i]);
+            hpass = hpass || (ip.flags & mimo::kIdentityCols) == 0;
             lp.block_start[k] = static_cast<int32_t>(blocks);
             blocks += ip.blocks;
             tr = std::max(tr, ip.tile_rows);
@@ -240,8 +259,11 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
         lp.block_start[k] = static_cast<int32_t>(blocks);
         lp.n = k;
         lp.tile_rows = tr;
-        lp.tile_stride = tc | 1;  // odd stride: consecutive tile rows start in different banks
-        const size_t smem = sizeof(float) * 3u * static_cast<size_t>(tr) * static_cast<size_t>(lp.tile_stride);
+        lp.tile_stride = (tc + 3) & ~3;  // 16-byte rows: whole-float4 staging stores and loads
+        const size_t tile_floats = 3u * static_cast<size_t>(tr) * static_cast<size_t>(lp.tile_stride);
+        lp.hbuf = hpass ? static_cast<int32_t>(tile_floats) : 0;
+        const size_t hbuf_floats = hpass ? 3u * static_cast<size_t>(tr) * mimo::kBlock : 0u;
+        const size_t smem = sizeof(float) * (tile_floats + hbuf_floats);
         const int st = mimo::launch_preprocess(lp, blocks, out_dtype, smem, stream);
         if (st != MIMO_OK) return st;
     }
@@ -312,7 +334,7 @@ int mimo_preprocess_batch(const mimo_params *p, int32_t n, const uint8_t *d_src,
     const int st = validate_batch(p, n, d_src, src_bytes, src_offsets, heights, widths, channels, out_dtype, d_out,
                                   out_rows_capacity, d_column_perm, &v);
     if (st != MIMO_OK || n == 0) return st;
-    return launch_range(p, v, 0, n, d_src, src_offsets, heights, widths, channels, out_dtype, d_out,
+    return launch_range(p, v, 0, n, d_src, src_bytes, src_offsets, heights, widths, channels, out_dtype, d_out,
                         d_column_perm, stream);
 }
 
@@ -368,7 +390,7 @@ int mimo_preprocess_batch_host(const mimo_params *p, int32_t n, const uint8_t *h
             cudaStream_t s = ss[chunk & 1];
             const int64_t r0 = v.plan.row0[first];
             if (fail(cudaMemcpyAsync(d_src_stage + lo, h_src + lo, hi - lo, cudaMemcpyHostToDevice, s))) break;
-            const int lst = launch_range(p, v, first, i, d_src_stage, src_offsets, heights, widths, channels,
+            const int lst = launch_range(p, v, first, i, d_src_stage, src_bytes, src_offsets, heights, widths, channels,
                                          out_dtype, d_out_stage, h_column_perm ? d_perm_stage : nullptr, s);
             if (lst != MIMO_OK) {
                 result = lst;

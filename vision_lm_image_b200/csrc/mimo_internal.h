@@ -22,21 +22,24 @@ constexpr int kMaxTile = 64;           // 32 outputs x 2 taps
 constexpr int kThreads = 256;
 constexpr int kMaxImagesPerLaunch = 512;
 
-// Per-axis staging mode of an image, decided on the host from the scale:
-// contiguous = the block's source span (first tap to last tap) fits in
-// kMaxTile rows/cols and is staged whole; gathered = only the two taps of
-// each of the 32 outputs are staged (tile index 2*d and 2*d+1).
-enum : int32_t { kGatherRows = 1, kGatherCols = 2 };
+// Per-axis staging mode of an image, decided on the host:
+//  - gathered: the block's source span does not fit kMaxTile, so only the
+//    two taps of each of the 32 outputs are staged (tile index 2d, 2d+1);
+//  - identity: the axis is not resized (in == out), every weight is 0 and
+//    only the first tap of each output is staged (32 entries);
+//  - otherwise the span from the first to the last tap is staged whole.
+enum : int32_t { kGatherRows = 1, kGatherCols = 2, kIdentityRows = 4, kIdentityCols = 8 };
 
 struct ImageDesc {
-    int64_t src_off;  // byte offset of the image in the packed source buffer
-    int64_t row0;     // first output row of the image in the batch
-    int32_t H, W;     // source size
-    int32_t Hr, Wr;   // resized size, multiples of 32
-    int32_t C;        // 3 or 4
-    int32_t flags;    // kGatherRows | kGatherCols
+    int64_t src_off;   // byte offset of the image in the packed source buffer
+    int64_t row0;      // first output row of the image in the batch
+    int64_t readable;  // bytes from src_off that may be read with aligned words
+    int32_t H, W;      // source size
+    int32_t Hr, Wr;    // resized size, multiples of 32
+    int32_t C;         // 3 or 4
+    int32_t flags;     // kGather* | kIdentity*
 };
-static_assert(sizeof(ImageDesc) == 40, "descriptor layout");
+static_assert(sizeof(ImageDesc) == 48, "descriptor layout");
 
 // Everything one launch needs travels by value as the kernel's parameter
 // block (__grid_constant__), so a launch needs no device-side table and no
@@ -48,8 +51,8 @@ struct LaunchParams {
     float k[3], b[3];    // normalisation folded: v = x*k[c] + b[c]
     int32_t n;           // images in this launch
     int32_t tile_rows;   // rows of the shared-memory tile (max over images)
-    int32_t tile_stride; // odd row stride (floats) of the tile
-    int32_t pad_;
+    int32_t tile_stride; // row stride (floats, multiple of 4) of the tile
+    int32_t hbuf;        // float offset of the horizontal-pass buffer, 0 if unused
     int32_t block_start[kMaxImagesPerLaunch + 1];  // prefix sum of merge blocks
     ImageDesc img[kMaxImagesPerLaunch];
 };

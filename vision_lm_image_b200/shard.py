@@ -1,0 +1,54 @@
+"""Data-parallel sharding of a preprocessing batch across ranks (one process per GPU).
+
+Images are independent and every output row has exactly one producer, so the
+path needs no exchange step: each rank runs the fused kernel on its own
+images. This module only decides which images a rank takes. Images go to
+ranks by longest-processing-time-first greedy assignment, with the cost of an
+image taken as its output bytes (resized pixels; the kernel is bound by HBM
+writes). Ties break by image index and then by rank, so every rank computes
+the same assignment from the same sizes without communicating.
+
+The batch plan (image_grid_thw, row offsets) stays global: a rank's rows for
+image i are rows [row_offsets[i], row_offsets[i+1]) of the batch, so shards
+can be reassembled, or consumed in place, without renumbering.
+"""
+from __future__ import annotations
+
+import heapq
+from typing import Sequence
+
+import numpy as np
+
+from . import mimo
+
+
+def lpt_assign(costs: Sequence[int], world: int) -> list[list[int]]:
+    """Greedy LPT: images by decreasing cost, each to the currently least-loaded rank."""
+    if world <= 0:
+        raise ValueError("world must be positive")
+    order = sorted(range(len(costs)), key=lambda i: (-int(costs[i]), i))
+    heap = [(0, r) for r in range(world)]
+    out: list[list[int]] = [[] for _ in range(world)]
+    for i in order:
+        load, r = heapq.heappop(heap)
+        out[r].append(i)
+        heapq.heappush(heap, (load + int(costs[i]), r))
+    for r in range(world):
+        out[r].sort()
+    return out
+
+
+def shard_plan(heights: Sequence[int], widths: Sequence[int], world: int, params=None):
+    """Returns (assignment per rank, grid_thw [n, 3], row_offsets [n + 1]) for a batch."""
+    grid, offs = mimo.plan_batch(heights, widths, params)
+    rows = np.diff(offs)
+    return lpt_assign(rows.tolist(), world), grid, offs
+
+
+def rank_images(images, rank: int, world: int, params=None):
+    """The images (in batch order) that ``rank`` processes, with their batch indices."""
+    heights = [int(im.shape[0]) for im in images]
+    widths = [int(im.shape[1]) for im in images]
+    assign, grid, offs = shard_plan(heights, widths, world, params)
+    mine = assign[rank]
+    return [images[i] for i in mine], mine, grid, offs
