@@ -244,10 +244,9 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
             d.Wr = static_cast<int32_t>(ip.Wr);
             d.C = channels[i];
             d.flags = ip.flags;
-            // aligned 32-bit reads may round the image's last byte up to a word
-            // boundary; allow that only inside the caller's buffer
-            const int64_t bytes = static_cast<int64_t>(heights[i]) * widths[i] * channels[i];
-            d.readable = std::min<int64_t>((bytes + 3) & ~int64_t(3), static_cast<int64_t>(src_bytes) - src_offsets[i]);
+            // staging copies are 16-byte chunks that may run up to 15 bytes past
+            // the image; they read nothing past the end of the caller's buffer
+            d.limit = static_cast<int64_t>(src_bytes) - src_offsets[i];
             hpass = hpass || (ip.flags & mimo::kIdentityCols) == 0;
             lp.block_start[k] = static_cast<int32_t>(blocks);
             blocks += ip.blocks;
@@ -263,7 +262,12 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
         const size_t tile_floats = 3u * static_cast<size_t>(tr) * static_cast<size_t>(lp.tile_stride);
         lp.hbuf = hpass ? static_cast<int32_t>(tile_floats) : 0;
         const size_t hbuf_floats = hpass ? 3u * static_cast<size_t>(tr) * mimo::kBlock : 0u;
-        const size_t smem = sizeof(float) * (tile_floats + hbuf_floats);
+        // raw staging rows: a row segment of up to 4*tc bytes at any 16-byte
+        // misalignment, plus the word a 12-byte RGB read may touch past it
+        lp.raw_stride = ((32 + 4 * tc) + 15) & ~15;
+        const size_t raw_floats = static_cast<size_t>(tr) * static_cast<size_t>(lp.raw_stride) / 4u;
+        lp.raw = static_cast<int32_t>(tile_floats + hbuf_floats);
+        const size_t smem = sizeof(float) * (tile_floats + hbuf_floats + raw_floats);
         const int st = mimo::launch_preprocess(lp, blocks, out_dtype, smem, stream);
         if (st != MIMO_OK) return st;
     }

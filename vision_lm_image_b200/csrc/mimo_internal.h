@@ -13,9 +13,9 @@
 
 namespace mimo {
 
-// One 32x32 output merge block per CTA; the source samples it needs are
-// staged in shared memory as planar fp32 tiles of at most kMaxTile rows and
-// columns (2 taps x 32 outputs).
+// One 32x32 output merge block at a time per CTA; the source samples it
+// needs are staged in shared memory as planar fp32 tiles of at most kMaxTile
+// rows and columns (2 taps x 32 outputs).
 constexpr int kBlock = 32;             // merge block side in resized pixels (patch 16 x merge 2)
 constexpr int kRowWidth = 1536;        // 3 channels x 2 frames x 16 x 16
 constexpr int kMaxTile = 64;           // 32 outputs x 2 taps
@@ -33,7 +33,7 @@ enum : int32_t { kGatherRows = 1, kGatherCols = 2, kIdentityRows = 4, kIdentityC
 struct ImageDesc {
     int64_t src_off;   // byte offset of the image in the packed source buffer
     int64_t row0;      // first output row of the image in the batch
-    int64_t readable;  // bytes from src_off that may be read with aligned words
+    int64_t limit;     // bytes of the caller's source buffer from src_off on
     int32_t H, W;      // source size
     int32_t Hr, Wr;    // resized size, multiples of 32
     int32_t C;         // 3 or 4
@@ -53,6 +53,8 @@ struct LaunchParams {
     int32_t tile_rows;   // rows of the shared-memory tile (max over images)
     int32_t tile_stride; // row stride (floats, multiple of 4) of the tile
     int32_t hbuf;        // float offset of the horizontal-pass buffer, 0 if unused
+    int32_t raw;         // float offset of the raw staging rows
+    int32_t raw_stride;  // bytes per raw staging row (multiple of 16)
     int32_t block_start[kMaxImagesPerLaunch + 1];  // prefix sum of merge blocks
     ImageDesc img[kMaxImagesPerLaunch];
 };

@@ -1,26 +1,29 @@
 // mimo_preprocess.cu -- the fused MiMo-V2 pixel path for sm_100a.
 //
-// One CTA owns one 32x32 merge block of one resized image (4 output rows of
-// 1536 values) and does every step of the path for it:
-//   0. exact bilinear taps of its 32 output rows (warp 0) and 32 output
-//      columns (warp 1) under align_corners=False (NeMo Automodel
-//      "mimo_v2_flash.processing", class MimoV2ImageProcessor: F.interpolate
-//      bilinear; docs.rs "cortiq_engine::mimo_vision", resize_bilinear);
-//   1. stages the source samples those taps touch into shared memory as
-//      planar fp32 on the 0..255 scale, compositing RGBA onto white on the
-//      way in (function _to_rgb); each lane moves 4 source pixels with
-//      aligned 32-bit loads and 16-byte shared stores;
-//   2. interpolates along W for every staged row (skipped when the width is
-//      not resized), then along H with packed f32x2 arithmetic, applies
-//      (x - 255*mean)/(255*std) folded to x*k + b (module docstring), and
-//      writes each 16-pixel row segment twice, once per temporal frame, laid
-//      out (c, tt, py, px) in merge-block row order (cortiq page, conventions);
-//   3. writes the column-order permutation entries of its merge unit
-//      (cortiq page, column_permutation).
-// The kernel has no inter-CTA communication, no atomics and no waits; every
+// The unit of work is one 32x32 merge block of one resized image (4 output
+// rows of 1536 values). For each block the kernel
+//   - computes the exact bilinear taps of its 32 output rows (warp 0) and 32
+//     output columns (warp 1) under align_corners=False (NeMo Automodel
+//     "mimo_v2_flash.processing", class MimoV2ImageProcessor: F.interpolate
+//     bilinear; docs.rs "cortiq_engine::mimo_vision", resize_bilinear);
+//   - copies the source row segments those taps touch into shared memory
+//     with 16-byte cp.async, then converts them to planar fp32 on the 0..255
+//     scale, compositing RGBA onto white on the way (function _to_rgb);
+//   - interpolates along W for every staged row (skipped when the width is
+//     not resized), then along H with packed f32x2 arithmetic, applies
+//     (x - 255*mean)/(255*std) folded to x*k + b (module docstring), and
+//     writes each 16-pixel row segment twice, once per temporal frame, laid
+//     out (c, tt, py, px) in merge-block row order (cortiq page, conventions);
+//   - writes the column-order permutation entries of its merge unit (cortiq
+//     page, column_permutation).
+// CTAs are persistent: each takes a contiguous range of blocks and overlaps
+// the source copies of the next blocks with the stores of the current one.
+// There is no inter-CTA communication, no atomics and no global wait; every
 // output element has exactly one writer.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "mimo.h"
 #include "mimo_internal.h"
@@ -29,20 +32,17 @@ namespace mimo {
 namespace {
 
 constexpr float kTwo23 = 8388608.0f;
+constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
 
-// Byte k of w as an exact float: PRMT builds the bit pattern 0x4B0000bb
-// (= 2^23 + b) and one subtraction removes 2^23.
+// Byte k of w as the float 2^23 + byte: PRMT builds the bit pattern
+// 0x4B0000bb; subtracting 2^23 afterwards gives the byte value exactly.
+template <int k>
+__device__ __forceinline__ float byte_bits(uint32_t w) {
+    return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u + k));
+}
 template <int k>
 __device__ __forceinline__ float byte_f(uint32_t w) {
-    return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u + k)) - kTwo23;
-}
-
-// Composite one RGBA channel value onto white: nearest integer of
-// (c*a + 255*(255-a)) / 255, as an exact float. 255 is odd, so there are no
-// ties, and floor((t + 127.5) / 255) equals floor((t + 127) / 255).
-__device__ __forceinline__ float on_white(uint32_t c, uint32_t a, uint32_t white) {
-    const uint32_t t = c * a + white;  // white = 255 * (255 - a)
-    return __uint_as_float(0x4B000000u | ((t + 127u) / 255u)) - kTwo23;
+    return byte_bits<k>(w) - kTwo23;
 }
 
 __device__ __forceinline__ uint64_t pack2(float a, float b) {
@@ -66,6 +66,18 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
     return r;
 }
 
+// Composite channel pairs onto white: nearest integer of (c*a + 255*(255-a))
+// / 255 per lane of the pair. c*a + white is an exact integer below 2^24;
+// t/255 is never within 1/510 of a half-integer (255 is odd) while the
+// product with fl(1/255) is within 1e-5 of it, so one FMA with the 1.5*2^23
+// constant rounds it exactly.
+__device__ __forceinline__ uint64_t on_white2(uint64_t c2, uint64_t a2, uint64_t white2) {
+    const uint64_t t = fma2(c2, a2, white2);
+    const uint64_t inv = pack2(1.0f / 255.0f, 1.0f / 255.0f);
+    const uint64_t rnd = pack2(kRound, kRound);
+    return sub2(fma2(t, inv, rnd), rnd);
+}
+
 // last i with block_start[i] <= blk
 __device__ __forceinline__ int find_image(const LaunchParams &P, int blk) {
     int lo = 0, hi = P.n - 1;
@@ -77,75 +89,113 @@ __device__ __forceinline__ int find_image(const LaunchParams &P, int blk) {
     return lo;
 }
 
-// One 32-bit word of the image at word index a (byte 4a), or, for the last
-// partial word of an image that ends unaligned at the end of the caller's
-// buffer, its bytes below `size` (the rest zero).
-__device__ __forceinline__ uint32_t load_word(const uint8_t *img, int64_t a, int64_t readable, int64_t size) {
-    if (4 * a + 4 <= readable) return __ldg(reinterpret_cast<const uint32_t *>(img) + a);
-    uint32_t w = 0;
-#pragma unroll
-    for (int b = 0; b < 4; ++b)
-        if (4 * a + b < size) w |= static_cast<uint32_t>(__ldg(img + 4 * a + b)) << (8 * b);
-    return w;
-}
+// Taps, staging geometry and output addresses of one merge block (double-
+// buffered in shared memory: the pipeline holds the current block and the
+// next one). Every later phase reads the block's constants from here.
+struct TapSet {
+    int32_t ty[2][kBlock];   // tile row of each output row's two taps
+    int32_t tx[2][kBlock];   // tile column of each output column's two taps
+    float ly[kBlock];        // weight of the second row tap
+    float lx[kBlock];        // weight of the second column tap
+    int32_t srow[kMaxTile];  // source row of each tile row (gathered rows)
+    int32_t scol[kMaxTile];  // source column of each tile column (gathered columns)
+    int32_t y_first, nrows;  // first source row / staged rows (contiguous rows)
+    int32_t x_first, ncols;  // first source column / staged columns
+    int32_t flags, W, C, CQ; // image flags, width, channels, 16-byte chunks per staged row
+    int32_t gw2, gh2, bh, bw;
+    int64_t src_off;         // image offset in the source buffer
+    int64_t limit;           // bytes readable from src_off (caller's buffer end)
+    int64_t row_base;        // first output row of the block
+};
 
-template <bool kBF16>
-__global__ void __launch_bounds__(kThreads) preprocess_kernel(const __grid_constant__ LaunchParams P) {
-    extern __shared__ float4 smem4[];
-    float *const tile = reinterpret_cast<float *>(smem4);  // [3][tile_rows][tile_stride] (+ hbuf)
-    __shared__ int32_t s_img;
-    __shared__ int32_t s_ty[2][kBlock];
-    __shared__ int32_t s_tx[2][kBlock];
-    __shared__ float s_ly[kBlock];
-    __shared__ float s_lx[kBlock];
-    __shared__ int32_t s_srow[kMaxTile];
-    __shared__ int32_t s_scol[kMaxTile];
-    __shared__ int32_t s_span[4];  // first row, rows, first col, cols
+// Per-lane state of a tap warp across the blocks of a CTA: the exact floor
+// quotient q and remainder r of ((2d+1)*in - out) / (2*out) for the lane's
+// output index d in the last block seen along the warp's axis, and the
+// change of both from one block to the next.
+struct AxisCursor {
+    int img = -1, b = -2;
+    int64_t q = 0, r = 0;
+    int64_t den = 1, step_q = 0, step_r = 0;
+    double inv_den = 1.0;
+};
 
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int blk = blockIdx.x;
+// Warps 0 (rows) and 1 (columns): taps of block blk into T. `prev` holds the
+// taps of the block before blk in this CTA's order.
+__device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, const TapSet &prev, int blk, int &ii,
+                                             AxisCursor &cur, int warp, int lane) {
+    while (ii + 1 < P.n && P.block_start[ii + 1] <= blk) ++ii;
+    const ImageDesc &D = P.img[ii];
+    const int32_t H = D.H, W = D.W, Hr = D.Hr, Wr = D.Wr, flags = D.flags, C = D.C;
+    const int local = blk - P.block_start[ii];
+    const int gw2 = Wr / kBlock;
+    const int bh = local / gw2;
+    const int bw = local - bh * gw2;
+    const bool is_col = warp == 1;
+    const int64_t in = is_col ? W : H;
+    const int64_t out = is_col ? Wr : Hr;
+    const int b = is_col ? bw : bh;
 
-    // ---- 0. taps: warp 0 -> the block's 32 output rows, warp 1 -> columns
-    if (warp < 2) {
-        const int ii = find_image(P, blk);
-        const ImageDesc &D = P.img[ii];
-        const int local = blk - P.block_start[ii];
-        const int gw2 = D.Wr / kBlock;
-        const int bh = local / gw2;
-        const int bw = local - bh * gw2;
-        const bool is_col = warp == 1;
-        const int64_t in = is_col ? D.W : D.H;
-        const int64_t out = is_col ? D.Wr : D.Hr;
-        const bool gather = (D.flags & (is_col ? kGatherCols : kGatherRows)) != 0;
-        const bool ident = (D.flags & (is_col ? kIdentityCols : kIdentityRows)) != 0;
-        const int64_t d = static_cast<int64_t>(is_col ? bw : bh) * kBlock + lane;
-        // source coordinate ((2d+1)*in - out) / (2*out): fp64 quotient, exact
-        // integer correction
-        const int64_t num = (2 * d + 1) * in - out;
-        const int64_t den = 2 * out;
-        int64_t q = 0, r = 0;
-        if (num > 0) {
-            q = static_cast<int64_t>(static_cast<double>(num) / static_cast<double>(den));
-            r = num - q * den;
-            if (r < 0) {
-                --q;
-                r += den;
-            } else if (r >= den) {
-                ++q;
-                r -= den;
-            }
+    if (!is_col && ii == cur.img && b == cur.b) {
+        // same block row as the previous block: row taps unchanged
+        T.ty[0][lane] = prev.ty[0][lane];
+        T.ty[1][lane] = prev.ty[1][lane];
+        T.ly[lane] = prev.ly[lane];
+        T.srow[lane] = prev.srow[lane];
+        T.srow[lane + 32] = prev.srow[lane + 32];
+        if (lane == 0) {
+            T.y_first = prev.y_first;
+            T.nrows = prev.nrows;
         }
-        const int32_t i0 = static_cast<int32_t>(q);
-        const int32_t i1 = (q + 1 < in) ? i0 + 1 : static_cast<int32_t>(in - 1);
-        const float lam = __fdiv_rn(static_cast<float>(r), static_cast<float>(den));
+    } else {
+        if (ii != cur.img) {
+            cur.img = ii;
+            cur.b = -2;
+            cur.den = 2 * out;
+            cur.inv_den = 1.0 / static_cast<double>(cur.den);
+            const int64_t step = 2 * kBlock * in;  // numerator change between blocks
+            cur.step_q = step / cur.den;
+            cur.step_r = step - cur.step_q * cur.den;
+        }
+        if (b == cur.b + 1) {
+            cur.q += cur.step_q;
+            cur.r += cur.step_r;
+            if (cur.r >= cur.den) {
+                cur.r -= cur.den;
+                ++cur.q;
+            }
+        } else {
+            // floor division of the (possibly negative) numerator: fp64
+            // estimate, exact integer correction
+            const int64_t d = static_cast<int64_t>(b) * kBlock + lane;
+            const int64_t num = (2 * d + 1) * in - out;
+            int64_t q = static_cast<int64_t>(floor(static_cast<double>(num) * cur.inv_den));
+            int64_t r = num - q * cur.den;
+            while (r < 0) {
+                --q;
+                r += cur.den;
+            }
+            while (r >= cur.den) {
+                ++q;
+                r -= cur.den;
+            }
+            cur.q = q;
+            cur.r = r;
+        }
+        cur.b = b;
+        // source coordinate clamped at 0: negative quotient -> first pixel, weight 0
+        const bool clamp = cur.q < 0;
+        const int32_t i0 = clamp ? 0 : static_cast<int32_t>(cur.q);
+        const int32_t i1 = (static_cast<int64_t>(i0) + 1 < in) ? i0 + 1 : static_cast<int32_t>(in - 1);
+        const float lam = clamp ? 0.0f : __fdiv_rn(static_cast<float>(cur.r), static_cast<float>(cur.den));
+        const bool gather = (flags & (is_col ? kGatherCols : kGatherRows)) != 0;
+        const bool ident = (flags & (is_col ? kIdentityCols : kIdentityRows)) != 0;
         const int32_t first = __shfl_sync(0xffffffffu, i0, 0);
         const int32_t last = __shfl_sync(0xffffffffu, i1, 31);
         int32_t j0, j1, count;
         if (gather) {
             j0 = 2 * lane;
             j1 = 2 * lane + 1;
-            int32_t *src_idx = is_col ? s_scol : s_srow;
+            int32_t *src_idx = is_col ? T.scol : T.srow;
             src_idx[j0] = i0;
             src_idx[j1] = i1;
             count = kMaxTile;
@@ -155,125 +205,188 @@ __global__ void __launch_bounds__(kThreads) preprocess_kernel(const __grid_const
             count = ident ? kBlock : last - first + 1;
         }
         if (is_col) {
-            s_tx[0][lane] = j0;
-            s_tx[1][lane] = j1;
-            s_lx[lane] = lam;
+            T.tx[0][lane] = j0;
+            T.tx[1][lane] = j1;
+            T.lx[lane] = lam;
         } else {
-            s_ty[0][lane] = j0;
-            s_ty[1][lane] = j1;
-            s_ly[lane] = lam;
+            T.ty[0][lane] = j0;
+            T.ty[1][lane] = j1;
+            T.ly[lane] = lam;
         }
         if (lane == 0) {
-            s_span[is_col ? 2 : 0] = gather ? 0 : first;
-            s_span[is_col ? 3 : 1] = count;
-            if (!is_col) s_img = ii;
+            if (is_col) {
+                T.x_first = gather ? 0 : first;
+                T.ncols = count;
+                T.CQ = (30 + C * count) >> 4;  // chunks covering a row segment at any 16-byte offset
+            } else {
+                T.y_first = gather ? 0 : first;
+                T.nrows = count;
+            }
         }
     }
-    __syncthreads();
+    if (!is_col && lane == 0) {
+        T.flags = flags;
+        T.W = W;
+        T.C = C;
+        T.gw2 = gw2;
+        T.gh2 = Hr / kBlock;
+        T.bh = bh;
+        T.bw = bw;
+        T.src_off = D.src_off;
+        T.limit = D.limit;
+        T.row_base = D.row0 + 4LL * (static_cast<int64_t>(bh) * gw2 + bw);
+    }
+}
 
-    const int ii = s_img;
-    const ImageDesc &D = P.img[ii];
-    const int flags = D.flags;
-    const int TS = P.tile_stride;
-    const int plane = P.tile_rows * TS;
-    const int y_first = s_span[0], nrows = s_span[1];
-    const int x_first = s_span[2], ncols = s_span[3];
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, int nbytes) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(src), "r"(nbytes) : "memory");
+}
 
-    // ---- 1. stage source samples as planar fp32, RGBA composited onto white
-    {
-        const uint8_t *img = P.src + D.src_off;
-        const int64_t W = D.W;
+// Starts the asynchronous copy of block T's source row segments into the
+// raw buffer: row j's bytes [rs, rs + C*ncols) are covered by 16-byte aligned
+// chunks stored at raw + j*raw_stride. A chunk reaching past the caller's
+// buffer is zero-filled there.
+__device__ __forceinline__ void issue_stage(const LaunchParams &P, const TapSet &T, uint8_t *raw, int tid) {
+    const int flags = T.flags;
+    if ((flags & kGatherCols) == 0) {
+        const uint8_t *img = P.src + T.src_off;
+        const int64_t limit = T.limit;
+        const int W = T.W, C = T.C, CQ = T.CQ;
+        const int y_first = T.y_first, x_first = T.x_first;
+        const int L = C * T.ncols;
         const bool grow = (flags & kGatherRows) != 0;
-        if ((flags & kGatherCols) == 0) {
-            // a job = 4 consecutive staged pixels of one tile row
-            const int Q = (ncols + 3) >> 2;
-            const uint32_t qmagic = (65536u + Q - 1) / Q;  // job / Q exact for job < 1024, Q <= 16
-            const int jobs = nrows * Q;
-            for (int job = tid; job < jobs; job += kThreads) {
-                const int j = static_cast<int>((static_cast<uint32_t>(job) * qmagic) >> 16);
-                const int px0 = (job - j * Q) * 4;
-                const int sy = grow ? s_srow[j] : y_first + j;
-                const int64_t pix0 = static_cast<int64_t>(sy) * W + x_first + px0;  // first source pixel
-                float4 c0, c1, c2;
-                if (D.C == 4) {
-                    const int nv = min(4, ncols - px0);
-                    uint32_t w[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        w[k] = (k < nv) ? __ldg(reinterpret_cast<const uint32_t *>(img) + pix0 + k) : 0xFF000000u;
-                    float o[3][4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t a = w[k] >> 24;
-                        const uint32_t white = 255u * (255u - a);
-                        o[0][k] = on_white(w[k] & 0xFFu, a, white);
-                        o[1][k] = on_white((w[k] >> 8) & 0xFFu, a, white);
-                        o[2][k] = on_white((w[k] >> 16) & 0xFFu, a, white);
-                    }
-                    c0 = make_float4(o[0][0], o[0][1], o[0][2], o[0][3]);
-                    c1 = make_float4(o[1][0], o[1][1], o[1][2], o[1][3]);
-                    c2 = make_float4(o[2][0], o[2][1], o[2][2], o[2][3]);
-                } else {
-                    // 12 bytes from byte 3*pix0: up to 4 aligned words, realigned
-                    const int64_t b0 = 3 * pix0;
-                    const int64_t a0 = b0 >> 2;
-                    const int sh = static_cast<int>(b0 & 3) * 8;
-                    const int64_t bend = 3 * (pix0 + min(4, ncols - px0));  // end of the bytes needed
-                    uint32_t w[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        w[k] = (4 * (a0 + k) < bend) ? load_word(img, a0 + k, D.readable, 3 * (int64_t)D.H * W) : 0u;
-                    const uint32_t r0 = __funnelshift_r(w[0], w[1], sh);
-                    const uint32_t r1 = __funnelshift_r(w[1], w[2], sh);
-                    const uint32_t r2 = __funnelshift_r(w[2], w[3], sh);
-                    // bytes: r0 = R0 G0 B0 R1 | r1 = G1 B1 R2 G2 | r2 = B2 R3 G3 B3
-                    c0 = make_float4(byte_f<0>(r0), byte_f<3>(r0), byte_f<2>(r1), byte_f<1>(r2));
-                    c1 = make_float4(byte_f<1>(r0), byte_f<0>(r1), byte_f<3>(r1), byte_f<2>(r2));
-                    c2 = make_float4(byte_f<2>(r0), byte_f<1>(r1), byte_f<0>(r2), byte_f<3>(r2));
-                }
-                float *t = tile + j * TS + px0;
-                *reinterpret_cast<float4 *>(t) = c0;
-                *reinterpret_cast<float4 *>(t + plane) = c1;
-                *reinterpret_cast<float4 *>(t + 2 * plane) = c2;
-            }
-        } else {
-            // gathered columns: 64 single pixels per tile row
-            const int total = nrows * kMaxTile;
-            for (int e = tid; e < total; e += kThreads) {
-                const int j = e >> 6;
-                const int i = e & (kMaxTile - 1);
-                const int sy = grow ? s_srow[j] : y_first + j;
-                const int64_t pix = static_cast<int64_t>(sy) * W + s_scol[i];
-                float r, g, b;
-                if (D.C == 4) {
-                    const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(img) + pix);
-                    const uint32_t a = v >> 24;
-                    const uint32_t white = 255u * (255u - a);
-                    r = on_white(v & 0xFFu, a, white);
-                    g = on_white((v >> 8) & 0xFFu, a, white);
-                    b = on_white((v >> 16) & 0xFFu, a, white);
-                } else {
-                    const uint8_t *px = img + 3 * pix;
-                    r = static_cast<float>(__ldg(px));
-                    g = static_cast<float>(__ldg(px + 1));
-                    b = static_cast<float>(__ldg(px + 2));
-                }
-                float *t = tile + j * TS + i;
-                t[0] = r;
-                t[plane] = g;
-                t[2 * plane] = b;
+        const int jobs = T.nrows * CQ;
+        const uint32_t cmagic = (65536u + CQ - 1) / CQ;  // job / CQ for job < 64 * 18
+        for (int job = tid; job < jobs; job += kThreads) {
+            const int j = static_cast<int>((static_cast<uint32_t>(job) * cmagic) >> 16);
+            const int c = job - j * CQ;
+            const int sy = grow ? T.srow[j] : y_first + j;
+            const int64_t rs = (static_cast<int64_t>(sy) * W + x_first) * C;
+            const int64_t cs = (rs & ~int64_t(15)) + 16 * c;
+            if (cs < rs + L) {
+                const int64_t left = limit - cs;
+                const int nb = left < 16 ? static_cast<int>(left) : 16;
+                cp_async16(raw + j * P.raw_stride + 16 * c, img + cs, nb);
             }
         }
     }
-    __syncthreads();
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
 
-    // ---- 2a. horizontal pass (resized widths only): hbuf[c][j][dx]
+// Converts block T's staged bytes to planar fp32 in the tile (RGBA
+// composited onto white): a job = 4 consecutive pixels of one tile row.
+// Gathered columns are loaded here directly from global memory.
+__device__ __forceinline__ void finish_stage(const LaunchParams &P, const TapSet &T, const uint8_t *raw, float *tile,
+                                             int TS, int plane, int tid) {
+    const int flags = T.flags;
+    const int nrows = T.nrows, ncols = T.ncols;
+    const int C = T.C;
+    const uint64_t two23 = pack2(kTwo23, kTwo23);
+    if ((flags & kGatherCols) == 0) {
+        const int W = T.W, y_first = T.y_first, x_first = T.x_first;
+        const bool grow = (flags & kGatherRows) != 0;
+        const int Q = (ncols + 3) >> 2;
+        const int jobs = nrows * Q;
+        const uint32_t qmagic = (65536u + Q - 1) / Q;  // job / Q for job < 1024
+        for (int job = tid; job < jobs; job += kThreads) {
+            const int j = static_cast<int>((static_cast<uint32_t>(job) * qmagic) >> 16);
+            const int px0 = (job - j * Q) * 4;
+            const int sy = grow ? T.srow[j] : y_first + j;
+            // low 4 bits of the row segment's byte offset (exact under 32-bit wraparound)
+            const uint32_t mis = ((static_cast<uint32_t>(sy) * static_cast<uint32_t>(W) + x_first) *
+                                  static_cast<uint32_t>(C)) & 15u;
+            const uint32_t o = mis + static_cast<uint32_t>(C * px0);
+            const uint32_t *rw = reinterpret_cast<const uint32_t *>(raw + j * P.raw_stride) + (o >> 2);
+            const uint32_t w0 = rw[0], w1 = rw[1], w2 = rw[2], w3 = rw[3];
+            float4 c0, c1, c2;
+            if (C == 4) {
+                // o is a multiple of 4: 4 whole RGBA pixels
+                const uint64_t A01 = sub2(pack2(byte_bits<3>(w0), byte_bits<3>(w1)), two23);
+                const uint64_t A23 = sub2(pack2(byte_bits<3>(w2), byte_bits<3>(w3)), two23);
+                // white = 255 * (255 - a) = 65025 - 255 a
+                const uint64_t m255 = pack2(-255.0f, -255.0f), k65025 = pack2(65025.0f, 65025.0f);
+                const uint64_t wh01 = fma2(A01, m255, k65025), wh23 = fma2(A23, m255, k65025);
+                const float2 R0 = unpack2(on_white2(sub2(pack2(byte_bits<0>(w0), byte_bits<0>(w1)), two23), A01, wh01));
+                const float2 R1 = unpack2(on_white2(sub2(pack2(byte_bits<0>(w2), byte_bits<0>(w3)), two23), A23, wh23));
+                const float2 G0 = unpack2(on_white2(sub2(pack2(byte_bits<1>(w0), byte_bits<1>(w1)), two23), A01, wh01));
+                const float2 G1 = unpack2(on_white2(sub2(pack2(byte_bits<1>(w2), byte_bits<1>(w3)), two23), A23, wh23));
+                const float2 B0 = unpack2(on_white2(sub2(pack2(byte_bits<2>(w0), byte_bits<2>(w1)), two23), A01, wh01));
+                const float2 B1 = unpack2(on_white2(sub2(pack2(byte_bits<2>(w2), byte_bits<2>(w3)), two23), A23, wh23));
+                c0 = make_float4(R0.x, R0.y, R1.x, R1.y);
+                c1 = make_float4(G0.x, G0.y, G1.x, G1.y);
+                c2 = make_float4(B0.x, B0.y, B1.x, B1.y);
+            } else {
+                // 12 bytes from o, realigned by the byte offset within the word
+                const int sh = static_cast<int>(o & 3u) * 8;
+                const uint32_t r0 = __funnelshift_r(w0, w1, sh);
+                const uint32_t r1 = __funnelshift_r(w1, w2, sh);
+                const uint32_t r2 = __funnelshift_r(w2, w3, sh);
+                // bytes: r0 = R0 G0 B0 R1 | r1 = G1 B1 R2 G2 | r2 = B2 R3 G3 B3
+                const float2 R0 = unpack2(sub2(pack2(byte_bits<0>(r0), byte_bits<3>(r0)), two23));
+                const float2 R1 = unpack2(sub2(pack2(byte_bits<2>(r1), byte_bits<1>(r2)), two23));
+                const float2 G0 = unpack2(sub2(pack2(byte_bits<1>(r0), byte_bits<0>(r1)), two23));
+                const float2 G1 = unpack2(sub2(pack2(byte_bits<3>(r1), byte_bits<2>(r2)), two23));
+                const float2 B0 = unpack2(sub2(pack2(byte_bits<2>(r0), byte_bits<1>(r1)), two23));
+                const float2 B1 = unpack2(sub2(pack2(byte_bits<0>(r2), byte_bits<3>(r2)), two23));
+                c0 = make_float4(R0.x, R0.y, R1.x, R1.y);
+                c1 = make_float4(G0.x, G0.y, G1.x, G1.y);
+                c2 = make_float4(B0.x, B0.y, B1.x, B1.y);
+            }
+            float *t = tile + j * TS + px0;
+            *reinterpret_cast<float4 *>(t) = c0;
+            *reinterpret_cast<float4 *>(t + plane) = c1;
+            *reinterpret_cast<float4 *>(t + 2 * plane) = c2;
+        }
+    } else {
+        const uint8_t *img = P.src + T.src_off;
+        const int64_t W = T.W;
+        const bool grow = (flags & kGatherRows) != 0;
+        const int total = nrows * kMaxTile;
+        for (int e = tid; e < total; e += kThreads) {
+            const int j = e >> 6;
+            const int i = e & (kMaxTile - 1);
+            const int sy = grow ? T.srow[j] : T.y_first + j;
+            const int64_t pix = static_cast<int64_t>(sy) * W + T.scol[i];
+            float r, g, b;
+            if (C == 4) {
+                const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(img) + pix);
+                const float a = byte_f<3>(v);
+                const float wh = fmaf(a, -255.0f, 65025.0f);
+                const uint64_t a2 = pack2(a, a), wh2 = pack2(wh, wh);
+                const float2 rg = unpack2(on_white2(sub2(pack2(byte_bits<0>(v), byte_bits<1>(v)), two23), a2, wh2));
+                const float2 bx = unpack2(on_white2(sub2(pack2(byte_bits<2>(v), byte_bits<2>(v)), two23), a2, wh2));
+                r = rg.x;
+                g = rg.y;
+                b = bx.x;
+            } else {
+                const uint8_t *px = img + 3 * pix;
+                r = static_cast<float>(__ldg(px));
+                g = static_cast<float>(__ldg(px + 1));
+                b = static_cast<float>(__ldg(px + 2));
+            }
+            float *t = tile + j * TS + i;
+            t[0] = r;
+            t[plane] = g;
+            t[2 * plane] = b;
+        }
+    }
+}
+
+// Interpolation, normalisation and stores of one staged block.
+template <bool kBF16>
+__device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &T, float *tile, int TS, int plane,
+                                           int tid, int warp, int lane) {
+    const int flags = T.flags;
+    const int nrows = T.nrows;
+
+    // horizontal pass (resized widths only): hbuf[c][j][dx]
     const bool hpass = (flags & kIdentityCols) == 0;
     if (hpass) {
         float *hb = tile + P.hbuf;
         const int hplane = P.tile_rows * kBlock;
-        const int x0 = s_tx[0][lane], x1 = s_tx[1][lane];
-        const float lx = s_lx[lane];
+        const int x0 = T.tx[0][lane], x1 = T.tx[1][lane];
+        const float lx = T.lx[lane];
         for (int j = warp; j < nrows; j += kThreads / 32) {
             const float *t = tile + j * TS;
 #pragma unroll
@@ -286,69 +399,112 @@ __global__ void __launch_bounds__(kThreads) preprocess_kernel(const __grid_const
         __syncthreads();
     }
 
-    // ---- 2b. vertical pass + normalisation + both temporal copies
-    // warp w covers output rows dy = 4w..4w+3 of the block; a lane covers 4
-    // consecutive columns. For fixed mw the 16 lanes write 4 consecutive
-    // 16-float segments of one output row: 256 contiguous bytes (fp32).
-    {
-        const int mh = warp >> 2;
-        const int py = ((warp & 3) << 2) | (lane >> 3);
-        const int mw = (lane >> 2) & 1;
-        const int q = lane & 3;
-        const int dy = (mh << 4) | py;
-        const int dx0 = (mw << 4) | (q << 2);
-        const float *buf = hpass ? tile + P.hbuf : tile;
-        const int stride = hpass ? kBlock : TS;
-        const int vplane = hpass ? P.tile_rows * kBlock : plane;
-        const bool yident = (flags & kIdentityRows) != 0;
-        const int r0 = s_ty[0][dy] * stride + dx0;
-        const int r1 = s_ty[1][dy] * stride + dx0;
-        const float ly = s_ly[dy];
-        const uint64_t ly2 = pack2(ly, ly);
-
-        const int local = blk - P.block_start[ii];
-        const int gw2 = D.Wr / kBlock;
-        const int bh = local / gw2;
-        const int bw = local - bh * gw2;
-        const int64_t row = D.row0 + 4LL * (static_cast<int64_t>(bh) * gw2 + bw) + (mh * 2 + mw);
-        const int col = py * 16 + q * 4;
+    // vertical pass + normalisation + both temporal copies. Warp w covers
+    // output rows dy = 4w..4w+3 of the block; a lane covers 4 consecutive
+    // columns. For fixed mw the 16 lanes write 4 consecutive 16-float
+    // segments of one output row: 256 contiguous bytes (fp32).
+    const int mh = warp >> 2;
+    const int py = ((warp & 3) << 2) | (lane >> 3);
+    const int mw = (lane >> 2) & 1;
+    const int q = lane & 3;
+    const int dy = (mh << 4) | py;
+    const int dx0 = (mw << 4) | (q << 2);
+    const float *buf = hpass ? tile + P.hbuf : tile;
+    const int stride = hpass ? kBlock : TS;
+    const int vplane = hpass ? P.tile_rows * kBlock : plane;
+    const bool yident = (flags & kIdentityRows) != 0;
+    const int r0 = T.ty[0][dy] * stride + dx0;
+    const int r1 = T.ty[1][dy] * stride + dx0;
+    const float ly = T.ly[dy];
+    const uint64_t ly2 = pack2(ly, ly);
+    const int64_t row = T.row_base + (mh * 2 + mw);
+    const int col = py * 16 + q * 4;
 #pragma unroll
-        for (int c = 0; c < 3; ++c) {
-            const float4 A = *reinterpret_cast<const float4 *>(buf + c * vplane + r0);
-            uint64_t v01 = pack2(A.x, A.y), v23 = pack2(A.z, A.w);
-            if (!yident) {
-                const float4 B = *reinterpret_cast<const float4 *>(buf + c * vplane + r1);
-                v01 = fma2(ly2, sub2(pack2(B.x, B.y), v01), v01);
-                v23 = fma2(ly2, sub2(pack2(B.z, B.w), v23), v23);
-            }
-            const uint64_t k2 = pack2(P.k[c], P.k[c]), b2 = pack2(P.b[c], P.b[c]);
-            const float2 n01 = unpack2(fma2(v01, k2, b2));
-            const float2 n23 = unpack2(fma2(v23, k2, b2));
-            if constexpr (!kBF16) {
-                float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col;
-                const float4 f4 = make_float4(n01.x, n01.y, n23.x, n23.y);
-                __stcs(reinterpret_cast<float4 *>(o), f4);        // tt = 0
-                __stcs(reinterpret_cast<float4 *>(o + 256), f4);  // tt = 1
-            } else {
-                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col;
-                const __nv_bfloat162 lo2 = __floats2bfloat162_rn(n01.x, n01.y);
-                const __nv_bfloat162 hi2 = __floats2bfloat162_rn(n23.x, n23.y);
-                uint2 u;
-                u.x = *reinterpret_cast<const uint32_t *>(&lo2);
-                u.y = *reinterpret_cast<const uint32_t *>(&hi2);
-                __stcs(reinterpret_cast<uint2 *>(o), u);
-                __stcs(reinterpret_cast<uint2 *>(o + 256), u);
-            }
+    for (int c = 0; c < 3; ++c) {
+        const float4 A = *reinterpret_cast<const float4 *>(buf + c * vplane + r0);
+        uint64_t v01 = pack2(A.x, A.y), v23 = pack2(A.z, A.w);
+        if (!yident) {
+            const float4 B = *reinterpret_cast<const float4 *>(buf + c * vplane + r1);
+            v01 = fma2(ly2, sub2(pack2(B.x, B.y), v01), v01);
+            v23 = fma2(ly2, sub2(pack2(B.z, B.w), v23), v23);
         }
+        const uint64_t k2 = pack2(P.k[c], P.k[c]), b2 = pack2(P.b[c], P.b[c]);
+        const float2 n01 = unpack2(fma2(v01, k2, b2));
+        const float2 n23 = unpack2(fma2(v23, k2, b2));
+        if constexpr (!kBF16) {
+            float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col;
+            const float4 f4 = make_float4(n01.x, n01.y, n23.x, n23.y);
+            __stcs(reinterpret_cast<float4 *>(o), f4);        // tt = 0
+            __stcs(reinterpret_cast<float4 *>(o + 256), f4);  // tt = 1
+        } else {
+            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col;
+            const __nv_bfloat162 lo2 = __floats2bfloat162_rn(n01.x, n01.y);
+            const __nv_bfloat162 hi2 = __floats2bfloat162_rn(n23.x, n23.y);
+            uint2 u;
+            u.x = *reinterpret_cast<const uint32_t *>(&lo2);
+            u.y = *reinterpret_cast<const uint32_t *>(&hi2);
+            __stcs(reinterpret_cast<uint2 *>(o), u);
+            __stcs(reinterpret_cast<uint2 *>(o + 256), u);
+        }
+    }
 
-        // ---- 3. column-order permutation: unit (bh, bw) is listed at (bw, bh)
-        if (P.perm != nullptr && tid == 0) {
-            const int gh2 = D.Hr / kBlock;
-            const int64_t src_unit = static_cast<int64_t>(bh) * gw2 + bw;
-            const int64_t dst_unit = static_cast<int64_t>(bw) * gh2 + bh;
-            const int32_t s0 = static_cast<int32_t>(D.row0 + 4 * src_unit);
-            __stcs(reinterpret_cast<int4 *>(P.perm + D.row0 + 4 * dst_unit), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
-        }
+    // column-order permutation: unit (bh, bw) is listed at (bw, bh)
+    if (P.perm != nullptr && tid == 0) {
+        const int64_t unit_row0 = T.row_base - 4LL * (static_cast<int64_t>(T.bh) * T.gw2 + T.bw);
+        const int64_t dst = unit_row0 + 4LL * (static_cast<int64_t>(T.bw) * T.gh2 + T.bh);
+        const int32_t s0 = static_cast<int32_t>(T.row_base);
+        __stcs(reinterpret_cast<int4 *>(P.perm + dst), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
+    }
+}
+
+// Persistent CTAs: CTA c takes the contiguous block range
+// [c*B/G, (c+1)*B/G) of the launch and pipelines it. While block k is
+// interpolated and stored, the source bytes of block k+1 are already in
+// shared memory and those of block k+2 are in flight (cp.async), and warps
+// 0-1 compute the taps of the block after.
+template <bool kBF16>
+__global__ void __launch_bounds__(kThreads, 6) preprocess_kernel(const __grid_constant__ LaunchParams P) {
+    extern __shared__ float4 smem4[];
+    float *const tile = reinterpret_cast<float *>(smem4);  // [3][rows][stride] | hbuf | raw bytes
+    uint8_t *const raw = reinterpret_cast<uint8_t *>(tile + P.raw);
+    __shared__ TapSet S[2];
+    __shared__ AxisCursor s_cur[64];  // one per lane of the two tap warps
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int TS = P.tile_stride;
+    const int plane = P.tile_rows * TS;
+    const int64_t B = P.block_start[P.n];
+    const int begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * B / gridDim.x);
+    const int end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * B / gridDim.x);
+    if (begin >= end) return;
+
+    int ii = 0;  // image cursor of warps 0-1
+    AxisCursor &cur = s_cur[tid & 63];
+    if (warp < 2) {
+        cur = AxisCursor();
+        ii = find_image(P, begin);
+        compute_taps(P, S[0], S[1], begin, ii, cur, warp, lane);
+    }
+    __syncthreads();
+    if (warp < 2 && begin + 1 < end) compute_taps(P, S[1], S[0], begin + 1, ii, cur, warp, lane);
+    issue_stage(P, S[0], raw, tid);
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    finish_stage(P, S[0], raw, tile, TS, plane, tid);
+    __syncthreads();
+    if (begin + 1 < end) issue_stage(P, S[1], raw, tid);
+
+    int slot = 0;
+    for (int blk = begin; blk < end; ++blk) {
+        emit_block<kBF16>(P, S[slot], tile, TS, plane, tid, warp, lane);
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncthreads();  // tile, hbuf and S[slot] free; raw holds block blk+1
+        if (blk + 1 < end) finish_stage(P, S[slot ^ 1], raw, tile, TS, plane, tid);
+        if (warp < 2 && blk + 2 < end) compute_taps(P, S[slot], S[slot ^ 1], blk + 2, ii, cur, warp, lane);
+        __syncthreads();  // tile holds block blk+1, S[slot] the taps of blk+2, raw is free
+        if (blk + 2 < end) issue_stage(P, S[slot], raw, tid);
+        slot ^= 1;
     }
 }
 
@@ -360,7 +516,15 @@ int launch_typed(const LaunchParams &lp, int64_t blocks, size_t smem_bytes, cuda
             cudaSuccess)
             return MIMO_ECUDA;
     }
-    kern<<<static_cast<unsigned>(blocks), kThreads, smem_bytes, stream>>>(lp);
+    // persistent grid: as many CTAs as can be resident at once
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem_bytes) != cudaSuccess ||
+        per_sm <= 0)
+        return MIMO_ECUDA;
+    const int64_t grid = std::min<int64_t>(blocks, static_cast<int64_t>(sms) * per_sm);
+    kern<<<static_cast<unsigned>(grid), kThreads, smem_bytes, stream>>>(lp);
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
 }
 
