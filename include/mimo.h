@@ -24,7 +24,8 @@
  *     host can see is reported before anything is launched or copied; the
  *     device code contains no traps and no waits.
  *   - Ownership: the caller owns every buffer. The library never allocates
- *     or frees device memory and keeps no state between calls.
+ *     or frees device memory at run time. Apart from the fixed staging area
+ *     of mimo_preprocess_batch_host_noalloc it keeps no state between calls.
  *   - "d_" pointers are device pointers, "h_" pointers host pointers; the
  *     other arrays (sizes, offsets) are host arrays read during the call.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
@@ -54,7 +55,8 @@ typedef enum {
     MIMO_ECAPACITY = 7,     /* an output or staging buffer is too small for the batch    */
     MIMO_EOVERFLOW = 8,     /* a size does not fit the index types (see each call)       */
     MIMO_ECUDA = 9,         /* a CUDA runtime call failed (launch or copy)               */
-    MIMO_ERANGE = 10        /* an image reaches past the end of the source buffer        */
+    MIMO_ERANGE = 10,       /* an image reaches past the end of the source buffer        */
+    MIMO_ELIMIT = 11        /* an image does not fit the fixed no-allocation staging area */
 } mimo_status;
 
 typedef enum {
@@ -164,6 +166,38 @@ int mimo_preprocess_batch_host(const mimo_params *p, int32_t n,
                                uint8_t *d_src_stage, size_t d_src_stage_bytes,
                                void *d_out_stage, int64_t d_out_stage_rows,
                                int32_t *d_perm_stage, void *stream);
+
+/*
+ * Host memory to host memory like mimo_preprocess_batch_host, for callers
+ * that cannot allocate device memory (no cudaMalloc, no caching-allocator
+ * call): images and rows are staged in a fixed area that the library itself
+ * defines, MIMO_NOALLOC_STAGING_BYTES of device memory held by every GPU
+ * that loads the library until the process exits. No counterpart on the
+ * reference pages: it is an interface choice of this library.
+ *   - Arguments and results are those of mimo_preprocess_batch_host without
+ *     the three device staging buffers. The call runs on the current device;
+ *     `stream` must belong to it. Synchronous: returns after the last copy
+ *     to h_out has completed.
+ *   - The batch is processed in chunks of whole images. An image whose
+ *     uint8 bytes plus output rows (plus permutation entries when asked for)
+ *     exceed the area, rounded up as the staging layout needs, is rejected
+ *     with MIMO_ELIMIT before anything is copied or launched. With fp32 rows
+ *     (24 bytes per resized pixel) an image of about 2.4 million resized
+ *     pixels fits; a 1080x1920 RGBA image resized to 1088x1920 does.
+ *   - The first call on a device looks the area's device address up
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call shares the one area and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero: each call writes every staged
+ *     byte it reads. Calls that overlap on the GPU (from several host
+ *     threads or streams at once) race on the area; serialise them.
+ * Allocates no device or page-locked memory.
+ */
+#define MIMO_NOALLOC_STAGING_BYTES (64u << 20)
+int mimo_preprocess_batch_host_noalloc(const mimo_params *p, int32_t n,
+                                       const uint8_t *h_src, size_t src_bytes, const int64_t *src_offsets,
+                                       const int32_t *heights, const int32_t *widths, const int32_t *channels,
+                                       int32_t out_dtype, void *h_out, int64_t out_rows_capacity,
+                                       int32_t *h_column_perm, void *stream);
 
 /* Static description of a status code. */
 const char *mimo_status_string(int status);

@@ -421,6 +421,83 @@ int mimo_preprocess_batch_host(const mimo_params *p, int32_t n, const uint8_t *h
     return result;
 }
 
+int mimo_preprocess_batch_host_noalloc(const mimo_params *p, int32_t n, const uint8_t *h_src, size_t src_bytes,
+                                       const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
+                                       const int32_t *channels, int32_t out_dtype, void *h_out,
+                                       int64_t out_rows_capacity, int32_t *h_column_perm, void *stream) {
+    Validated v;
+    const int st = validate_batch(p, n, h_src, src_bytes, src_offsets, heights, widths, channels, out_dtype, h_out,
+                                  out_rows_capacity, h_column_perm, &v);
+    if (st != MIMO_OK || n == 0) return st;
+
+    const size_t row_bytes = static_cast<size_t>(mimo::kRowWidth) * dtype_bytes(out_dtype);
+    const bool perm = h_column_perm != nullptr;
+    auto up = [](size_t x, size_t a) { return (x + a - 1) / a * a; };
+    // staged footprint of one image: its bytes (16-byte slots), rows, permutation entries
+    auto image_src = [&](int32_t i) {
+        return up(static_cast<size_t>(heights[i]) * widths[i] * channels[i], 16);
+    };
+    auto image_out = [&](int32_t i) {
+        const size_t rows = static_cast<size_t>(v.plan.img[i].rows);
+        return up(rows * row_bytes, 256) + (perm ? up(rows * sizeof(int32_t), 256) : 0);
+    };
+    const size_t cap = MIMO_NOALLOC_STAGING_BYTES;
+    for (int32_t i = 0; i < n; ++i)
+        if (up(image_src(i), 256) + image_out(i) > cap) return MIMO_ELIMIT;
+
+    void *stage = nullptr;
+    size_t stage_bytes = 0;
+    int rc = mimo::noalloc_staging(&stage, &stage_bytes);
+    if (rc != MIMO_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uintptr_t base = reinterpret_cast<uintptr_t>(stage);
+
+    // the launch helper reads source offsets by batch index: chunk-local
+    // positions go into a batch-sized table
+    std::vector<int64_t> local_off(static_cast<size_t>(n), 0);
+    int32_t i = 0;
+    while (i < n) {
+        const int32_t first = i;
+        size_t src_used = 0, out_used = 0;
+        while (i < n) {
+            const size_t s_add = image_src(i), o_add = image_out(i);
+            if (i > first && up(src_used + s_add, 256) + out_used + o_add > stage_bytes) break;
+            local_off[i] = static_cast<int64_t>(src_used);
+            src_used += s_add;
+            out_used += o_add;
+            ++i;
+        }
+        const int64_t row0 = v.plan.row0[first];
+        const int64_t rows = v.plan.row0[i] - row0;
+        const uintptr_t out_at = base + up(src_used, 256);
+        const uintptr_t perm_at = out_at + up(static_cast<size_t>(rows) * row_bytes, 256);
+        for (int32_t k = first; k < i; ++k) {
+            const size_t bytes = static_cast<size_t>(heights[k]) * widths[k] * channels[k];
+            if (cudaMemcpyAsync(reinterpret_cast<void *>(base + static_cast<uintptr_t>(local_off[k])),
+                                h_src + src_offsets[k], bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return MIMO_ECUDA;
+        }
+        // The kernel addresses rows and permutation entries by batch-global
+        // row index; shifting the bases down by the chunk's first row puts
+        // this chunk's rows at the start of its staging slots.
+        void *out_base = reinterpret_cast<void *>(out_at - static_cast<uintptr_t>(row0) * row_bytes);
+        int32_t *perm_base =
+            perm ? reinterpret_cast<int32_t *>(perm_at - static_cast<uintptr_t>(row0) * sizeof(int32_t)) : nullptr;
+        rc = launch_range(p, v, first, i, reinterpret_cast<const uint8_t *>(base), src_used, local_off.data(),
+                          heights, widths, channels, out_dtype, out_base, perm_base, s);
+        if (rc != MIMO_OK) return rc;
+        if (cudaMemcpyAsync(static_cast<char *>(h_out) + static_cast<size_t>(row0) * row_bytes,
+                            reinterpret_cast<void *>(out_at), static_cast<size_t>(rows) * row_bytes,
+                            cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return MIMO_ECUDA;
+        if (perm && cudaMemcpyAsync(h_column_perm + row0, reinterpret_cast<void *>(perm_at),
+                                    static_cast<size_t>(rows) * sizeof(int32_t), cudaMemcpyDeviceToHost,
+                                    s) != cudaSuccess)
+            return MIMO_ECUDA;
+    }
+    return cudaStreamSynchronize(s) == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
+}
+
 const char *mimo_status_string(int status) {
     switch (status) {
         case MIMO_OK: return "ok";
@@ -434,6 +511,7 @@ const char *mimo_status_string(int status) {
         case MIMO_EOVERFLOW: return "size exceeds the supported index range";
         case MIMO_ECUDA: return "CUDA runtime error";
         case MIMO_ERANGE: return "an image lies outside the source buffer";
+        case MIMO_ELIMIT: return "an image does not fit the fixed staging area of the no-allocation entry point";
         default: return "unknown status";
     }
 }

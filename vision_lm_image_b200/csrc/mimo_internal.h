@@ -93,4 +93,8 @@ MIMO_HD int64_t block_span(int64_t b, int64_t in, int64_t out) {
 
 int launch_preprocess(const LaunchParams &lp, int64_t blocks, int out_dtype, size_t smem_bytes, void *stream);
 
+// Device address and size of the library's fixed staging area on the
+// current device (mimo_noalloc.cu).
+int noalloc_staging(void **dev_ptr, size_t *bytes);
+
 }  // namespace mimo

@@ -31,10 +31,12 @@ ALIGN = 16
 STATUS_NAMES = {
     0: "MIMO_OK", 1: "MIMO_EINVAL", 2: "MIMO_EASPECT", 3: "MIMO_EDEGENERATE", 4: "MIMO_ECHANNELS",
     5: "MIMO_EUNSUPPORTED", 6: "MIMO_EALIGN", 7: "MIMO_ECAPACITY", 8: "MIMO_EOVERFLOW", 9: "MIMO_ECUDA",
-    10: "MIMO_ERANGE",
+    10: "MIMO_ERANGE", 11: "MIMO_ELIMIT",
 }
 EXPORTED = ("mimo_params_default", "mimo_smart_resize", "mimo_num_patches", "mimo_plan_batch",
-            "mimo_preprocess_batch", "mimo_preprocess_batch_host", "mimo_status_string", "mimo_version")
+            "mimo_preprocess_batch", "mimo_preprocess_batch_host", "mimo_preprocess_batch_host_noalloc",
+            "mimo_status_string", "mimo_version")
+NOALLOC_STAGING_BYTES = 64 << 20
 
 
 class MimoLibraryMissing(RuntimeError):
@@ -95,6 +97,9 @@ def lib() -> ctypes.CDLL:
             L.mimo_preprocess_batch_host.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p,
                                                      _i32, _p, _i64, _p, _p, _sz, _p, _i64, _p, _p]
             L.mimo_preprocess_batch_host.restype = ctypes.c_int
+            L.mimo_preprocess_batch_host_noalloc.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p,
+                                                             _p, _i32, _p, _i64, _p, _p]
+            L.mimo_preprocess_batch_host_noalloc.restype = ctypes.c_int
             L.mimo_status_string.argtypes = [ctypes.c_int]
             L.mimo_status_string.restype = ctypes.c_char_p
             L.mimo_version.argtypes = []
@@ -301,3 +306,19 @@ def preprocess_batch_host(params: MimoParams, packed_host: PackedBatch, out_host
         out_stage.shape[0], ctypes.c_void_p(perm_stage.data_ptr() if perm_stage is not None else 0),
         _stream_handle(stream, src_stage.device))
     _check(st, "preprocess_batch_host")
+
+
+def preprocess_batch_host_noalloc(params: MimoParams, packed_host: PackedBatch, out_host, perm_host=None,
+                                  stream=None) -> None:
+    """Host images in, host rows out, staged through the library's fixed device area: for callers that
+    cannot allocate device memory. Runs on the current CUDA device; returns when ``out_host`` is filled."""
+    import torch
+
+    buf = packed_host.buffer
+    st = lib().mimo_preprocess_batch_host_noalloc(
+        ctypes.byref(params), packed_host.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
+        packed_host.offsets.ctypes.data, packed_host.heights.ctypes.data, packed_host.widths.ctypes.data,
+        packed_host.channels.ctypes.data, _dtype_code(out_host.dtype), ctypes.c_void_p(out_host.data_ptr()),
+        out_host.shape[0], ctypes.c_void_p(perm_host.data_ptr() if perm_host is not None else 0),
+        _stream_handle(stream, torch.device("cuda", torch.cuda.current_device())))
+    _check(st, "preprocess_batch_host_noalloc")
