@@ -45,37 +45,19 @@ __device__ __forceinline__ float byte_f(uint32_t w) {
     return byte_bits<k>(w) - kTwo23;
 }
 
-__device__ __forceinline__ uint64_t pack2(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ float2 unpack2(uint64_t v) {
-    float2 f;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
-    return f;
-}
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
+// Packed fp32 pairs: sm_100 executes one FMA/ADD on both halves of a float2.
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 // Composite channel pairs onto white: nearest integer of (c*a + 255*(255-a))
 // / 255 per lane of the pair. c*a + white is an exact integer below 2^24;
 // t/255 is never within 1/510 of a half-integer (255 is odd) while the
 // product with fl(1/255) is within 1e-5 of it, so one FMA with the 1.5*2^23
 // constant rounds it exactly.
-__device__ __forceinline__ uint64_t on_white2(uint64_t c2, uint64_t a2, uint64_t white2) {
-    const uint64_t t = fma2(c2, a2, white2);
-    const uint64_t inv = pack2(1.0f / 255.0f, 1.0f / 255.0f);
-    const uint64_t rnd = pack2(kRound, kRound);
-    return sub2(fma2(t, inv, rnd), rnd);
+__device__ __forceinline__ float2 on_white2(float2 c2, float2 a2, float2 white2) {
+    const float2 t = fma2(c2, a2, white2);
+    return add2(fma2(t, f2(1.0f / 255.0f, 1.0f / 255.0f), f2(kRound, kRound)), f2(-kRound, -kRound));
 }
 
 // last i with block_start[i] <= blk
@@ -103,6 +85,8 @@ struct TapSet {
     int32_t x_first, ncols;  // first source column / staged columns
     int32_t flags, W, C, CQ; // image flags, width, channels, 16-byte chunks per staged row
     int32_t gw2, gh2, bh, bw;
+    int32_t Q, pad_q;          // staging jobs (4 pixels) per tile row
+    uint32_t qmagic, cmagic;  // x / Q and x / CQ as (x * magic) >> 16 for the job counts here
     int64_t src_off;         // image offset in the source buffer
     int64_t limit;           // bytes readable from src_off (caller's buffer end)
     int64_t row_base;        // first output row of the block
@@ -113,23 +97,48 @@ struct TapSet {
 // output index d in the last block seen along the warp's axis, and the
 // change of both from one block to the next.
 struct AxisCursor {
+    int blk = -2, ii = 0, bh = 0, bw = 0;  // position of the last block handled
     int img = -1, b = -2;
     int64_t q = 0, r = 0;
     int64_t den = 1, step_q = 0, step_r = 0;
     double inv_den = 1.0;
+    float inv_den_f = 1.0f;
 };
 
 // Warps 0 (rows) and 1 (columns): taps of block blk into T. `prev` holds the
 // taps of the block before blk in this CTA's order.
-__device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, const TapSet &prev, int blk, int &ii,
+__device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, const TapSet &prev, int blk,
                                              AxisCursor &cur, int warp, int lane) {
-    while (ii + 1 < P.n && P.block_start[ii + 1] <= blk) ++ii;
+    // block position: consecutive blocks advance one column (or start the
+    // next block row / image); only the CTA's first block needs a division
+    int ii = cur.ii, bh, bw;
+    if (blk == cur.blk + 1) {
+        if (ii + 1 < P.n && P.block_start[ii + 1] <= blk) {
+            ++ii;
+            bh = 0;
+            bw = 0;
+        } else {
+            bh = cur.bh;
+            bw = cur.bw + 1;
+            if (bw == P.img[ii].Wr / kBlock) {
+                bw = 0;
+                ++bh;
+            }
+        }
+    } else {
+        ii = find_image(P, blk);
+        const int local = blk - P.block_start[ii];
+        const int g = P.img[ii].Wr / kBlock;
+        bh = local / g;
+        bw = local - bh * g;
+    }
+    cur.blk = blk;
+    cur.ii = ii;
+    cur.bh = bh;
+    cur.bw = bw;
     const ImageDesc &D = P.img[ii];
     const int32_t H = D.H, W = D.W, Hr = D.Hr, Wr = D.Wr, flags = D.flags, C = D.C;
-    const int local = blk - P.block_start[ii];
     const int gw2 = Wr / kBlock;
-    const int bh = local / gw2;
-    const int bw = local - bh * gw2;
     const bool is_col = warp == 1;
     const int64_t in = is_col ? W : H;
     const int64_t out = is_col ? Wr : Hr;
@@ -152,6 +161,7 @@ __device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, c
             cur.b = -2;
             cur.den = 2 * out;
             cur.inv_den = 1.0 / static_cast<double>(cur.den);
+            cur.inv_den_f = static_cast<float>(cur.inv_den);
             const int64_t step = 2 * kBlock * in;  // numerator change between blocks
             cur.step_q = step / cur.den;
             cur.step_r = step - cur.step_q * cur.den;
@@ -186,7 +196,11 @@ __device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, c
         const bool clamp = cur.q < 0;
         const int32_t i0 = clamp ? 0 : static_cast<int32_t>(cur.q);
         const int32_t i1 = (static_cast<int64_t>(i0) + 1 < in) ? i0 + 1 : static_cast<int32_t>(in - 1);
-        const float lam = clamp ? 0.0f : __fdiv_rn(static_cast<float>(cur.r), static_cast<float>(cur.den));
+        // r < den; below 2^23 the float conversion is exact with the 2^23 bit trick
+        const float rf = (cur.r < (int64_t(1) << 23))
+                             ? __uint_as_float(0x4B000000u | static_cast<uint32_t>(cur.r)) - kTwo23
+                             : static_cast<float>(cur.r);
+        const float lam = clamp ? 0.0f : rf * cur.inv_den_f;
         const bool gather = (flags & (is_col ? kGatherCols : kGatherRows)) != 0;
         const bool ident = (flags & (is_col ? kIdentityCols : kIdentityRows)) != 0;
         const int32_t first = __shfl_sync(0xffffffffu, i0, 0);
@@ -217,7 +231,12 @@ __device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, c
             if (is_col) {
                 T.x_first = gather ? 0 : first;
                 T.ncols = count;
-                T.CQ = (30 + C * count) >> 4;  // chunks covering a row segment at any 16-byte offset
+                const int CQ = (30 + C * count) >> 4;  // chunks covering a row segment at any 16-byte offset
+                const int Q = (count + 3) >> 2;
+                T.CQ = CQ;
+                T.Q = Q;
+                T.cmagic = (65536u + CQ - 1) / CQ;  // exact for x < 64 * 18
+                T.qmagic = (65536u + Q - 1) / Q;    // exact for x < 64 * 16
             } else {
                 T.y_first = gather ? 0 : first;
                 T.nrows = count;
@@ -257,7 +276,7 @@ __device__ __forceinline__ void issue_stage(const LaunchParams &P, const TapSet 
         const int L = C * T.ncols;
         const bool grow = (flags & kGatherRows) != 0;
         const int jobs = T.nrows * CQ;
-        const uint32_t cmagic = (65536u + CQ - 1) / CQ;  // job / CQ for job < 64 * 18
+        const uint32_t cmagic = T.cmagic;
         for (int job = tid; job < jobs; job += kThreads) {
             const int j = static_cast<int>((static_cast<uint32_t>(job) * cmagic) >> 16);
             const int c = job - j * CQ;
@@ -280,16 +299,21 @@ __device__ __forceinline__ void issue_stage(const LaunchParams &P, const TapSet 
 __device__ __forceinline__ void finish_stage(const LaunchParams &P, const TapSet &T, const uint8_t *raw, float *tile,
                                              int TS, int plane, int tid) {
     const int flags = T.flags;
-    const int nrows = T.nrows, ncols = T.ncols;
+    const int nrows = T.nrows;
     const int C = T.C;
-    const uint64_t two23 = pack2(kTwo23, kTwo23);
+    const float2 m23 = f2(-kTwo23, -kTwo23);
     if ((flags & kGatherCols) == 0) {
         const int W = T.W, y_first = T.y_first, x_first = T.x_first;
         const bool grow = (flags & kGatherRows) != 0;
-        const int Q = (ncols + 3) >> 2;
+        const int Q = T.Q;
+        const uint32_t qmagic = T.qmagic;
         const int jobs = nrows * Q;
-        const uint32_t qmagic = (65536u + Q - 1) / Q;  // job / Q for job < 1024
-        for (int job = tid; job < jobs; job += kThreads) {
+        // warps 0-1 compute the next block's taps in this phase: leave them
+        // out of the conversion unless the block has many jobs
+        const int t0 = (jobs <= 2 * (kThreads - 64)) ? 64 : 0;
+        const int step = kThreads - t0;
+        for (int job = tid - t0; job < jobs; job += step) {
+            if (job < 0) break;
             const int j = static_cast<int>((static_cast<uint32_t>(job) * qmagic) >> 16);
             const int px0 = (job - j * Q) * 4;
             const int sy = grow ? T.srow[j] : y_first + j;
@@ -299,23 +323,19 @@ __device__ __forceinline__ void finish_stage(const LaunchParams &P, const TapSet
             const uint32_t o = mis + static_cast<uint32_t>(C * px0);
             const uint32_t *rw = reinterpret_cast<const uint32_t *>(raw + j * P.raw_stride) + (o >> 2);
             const uint32_t w0 = rw[0], w1 = rw[1], w2 = rw[2], w3 = rw[3];
-            float4 c0, c1, c2;
+            float2 R0, R1, G0, G1, B0, B1;
             if (C == 4) {
-                // o is a multiple of 4: 4 whole RGBA pixels
-                const uint64_t A01 = sub2(pack2(byte_bits<3>(w0), byte_bits<3>(w1)), two23);
-                const uint64_t A23 = sub2(pack2(byte_bits<3>(w2), byte_bits<3>(w3)), two23);
-                // white = 255 * (255 - a) = 65025 - 255 a
-                const uint64_t m255 = pack2(-255.0f, -255.0f), k65025 = pack2(65025.0f, 65025.0f);
-                const uint64_t wh01 = fma2(A01, m255, k65025), wh23 = fma2(A23, m255, k65025);
-                const float2 R0 = unpack2(on_white2(sub2(pack2(byte_bits<0>(w0), byte_bits<0>(w1)), two23), A01, wh01));
-                const float2 R1 = unpack2(on_white2(sub2(pack2(byte_bits<0>(w2), byte_bits<0>(w3)), two23), A23, wh23));
-                const float2 G0 = unpack2(on_white2(sub2(pack2(byte_bits<1>(w0), byte_bits<1>(w1)), two23), A01, wh01));
-                const float2 G1 = unpack2(on_white2(sub2(pack2(byte_bits<1>(w2), byte_bits<1>(w3)), two23), A23, wh23));
-                const float2 B0 = unpack2(on_white2(sub2(pack2(byte_bits<2>(w0), byte_bits<2>(w1)), two23), A01, wh01));
-                const float2 B1 = unpack2(on_white2(sub2(pack2(byte_bits<2>(w2), byte_bits<2>(w3)), two23), A23, wh23));
-                c0 = make_float4(R0.x, R0.y, R1.x, R1.y);
-                c1 = make_float4(G0.x, G0.y, G1.x, G1.y);
-                c2 = make_float4(B0.x, B0.y, B1.x, B1.y);
+                // o is a multiple of 4: 4 whole RGBA pixels; white = 65025 - 255 a
+                const float2 A01 = add2(f2(byte_bits<3>(w0), byte_bits<3>(w1)), m23);
+                const float2 A23 = add2(f2(byte_bits<3>(w2), byte_bits<3>(w3)), m23);
+                const float2 wh01 = fma2(A01, f2(-255.0f, -255.0f), f2(65025.0f, 65025.0f));
+                const float2 wh23 = fma2(A23, f2(-255.0f, -255.0f), f2(65025.0f, 65025.0f));
+                R0 = on_white2(add2(f2(byte_bits<0>(w0), byte_bits<0>(w1)), m23), A01, wh01);
+                R1 = on_white2(add2(f2(byte_bits<0>(w2), byte_bits<0>(w3)), m23), A23, wh23);
+                G0 = on_white2(add2(f2(byte_bits<1>(w0), byte_bits<1>(w1)), m23), A01, wh01);
+                G1 = on_white2(add2(f2(byte_bits<1>(w2), byte_bits<1>(w3)), m23), A23, wh23);
+                B0 = on_white2(add2(f2(byte_bits<2>(w0), byte_bits<2>(w1)), m23), A01, wh01);
+                B1 = on_white2(add2(f2(byte_bits<2>(w2), byte_bits<2>(w3)), m23), A23, wh23);
             } else {
                 // 12 bytes from o, realigned by the byte offset within the word
                 const int sh = static_cast<int>(o & 3u) * 8;
@@ -323,20 +343,17 @@ __device__ __forceinline__ void finish_stage(const LaunchParams &P, const TapSet
                 const uint32_t r1 = __funnelshift_r(w1, w2, sh);
                 const uint32_t r2 = __funnelshift_r(w2, w3, sh);
                 // bytes: r0 = R0 G0 B0 R1 | r1 = G1 B1 R2 G2 | r2 = B2 R3 G3 B3
-                const float2 R0 = unpack2(sub2(pack2(byte_bits<0>(r0), byte_bits<3>(r0)), two23));
-                const float2 R1 = unpack2(sub2(pack2(byte_bits<2>(r1), byte_bits<1>(r2)), two23));
-                const float2 G0 = unpack2(sub2(pack2(byte_bits<1>(r0), byte_bits<0>(r1)), two23));
-                const float2 G1 = unpack2(sub2(pack2(byte_bits<3>(r1), byte_bits<2>(r2)), two23));
-                const float2 B0 = unpack2(sub2(pack2(byte_bits<2>(r0), byte_bits<1>(r1)), two23));
-                const float2 B1 = unpack2(sub2(pack2(byte_bits<0>(r2), byte_bits<3>(r2)), two23));
-                c0 = make_float4(R0.x, R0.y, R1.x, R1.y);
-                c1 = make_float4(G0.x, G0.y, G1.x, G1.y);
-                c2 = make_float4(B0.x, B0.y, B1.x, B1.y);
+                R0 = add2(f2(byte_bits<0>(r0), byte_bits<3>(r0)), m23);
+                R1 = add2(f2(byte_bits<2>(r1), byte_bits<1>(r2)), m23);
+                G0 = add2(f2(byte_bits<1>(r0), byte_bits<0>(r1)), m23);
+                G1 = add2(f2(byte_bits<3>(r1), byte_bits<2>(r2)), m23);
+                B0 = add2(f2(byte_bits<2>(r0), byte_bits<1>(r1)), m23);
+                B1 = add2(f2(byte_bits<0>(r2), byte_bits<3>(r2)), m23);
             }
             float *t = tile + j * TS + px0;
-            *reinterpret_cast<float4 *>(t) = c0;
-            *reinterpret_cast<float4 *>(t + plane) = c1;
-            *reinterpret_cast<float4 *>(t + 2 * plane) = c2;
+            *reinterpret_cast<float4 *>(t) = make_float4(R0.x, R0.y, R1.x, R1.y);
+            *reinterpret_cast<float4 *>(t + plane) = make_float4(G0.x, G0.y, G1.x, G1.y);
+            *reinterpret_cast<float4 *>(t + 2 * plane) = make_float4(B0.x, B0.y, B1.x, B1.y);
         }
     } else {
         const uint8_t *img = P.src + T.src_off;
@@ -353,9 +370,8 @@ __device__ __forceinline__ void finish_stage(const LaunchParams &P, const TapSet
                 const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(img) + pix);
                 const float a = byte_f<3>(v);
                 const float wh = fmaf(a, -255.0f, 65025.0f);
-                const uint64_t a2 = pack2(a, a), wh2 = pack2(wh, wh);
-                const float2 rg = unpack2(on_white2(sub2(pack2(byte_bits<0>(v), byte_bits<1>(v)), two23), a2, wh2));
-                const float2 bx = unpack2(on_white2(sub2(pack2(byte_bits<2>(v), byte_bits<2>(v)), two23), a2, wh2));
+                const float2 rg = on_white2(add2(f2(byte_bits<0>(v), byte_bits<1>(v)), m23), f2(a, a), f2(wh, wh));
+                const float2 bx = on_white2(add2(f2(byte_bits<2>(v), byte_bits<2>(v)), m23), f2(a, a), f2(wh, wh));
                 r = rg.x;
                 g = rg.y;
                 b = bx.x;
@@ -413,24 +429,25 @@ __device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &
     const int stride = hpass ? kBlock : TS;
     const int vplane = hpass ? P.tile_rows * kBlock : plane;
     const bool yident = (flags & kIdentityRows) != 0;
-    const int r0 = T.ty[0][dy] * stride + dx0;
-    const int r1 = T.ty[1][dy] * stride + dx0;
+    const float *a_row = buf + T.ty[0][dy] * stride + dx0;
+    const float *b_row = buf + T.ty[1][dy] * stride + dx0;
+    // (1 - ly) a + ly b as two FMAs: a - ly a, then + ly b
     const float ly = T.ly[dy];
-    const uint64_t ly2 = pack2(ly, ly);
+    const float2 ly2 = f2(ly, ly), nly2 = f2(-ly, -ly);
     const int64_t row = T.row_base + (mh * 2 + mw);
     const int col = py * 16 + q * 4;
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
-        const float4 A = *reinterpret_cast<const float4 *>(buf + c * vplane + r0);
-        uint64_t v01 = pack2(A.x, A.y), v23 = pack2(A.z, A.w);
+        const float4 A = *reinterpret_cast<const float4 *>(a_row + c * vplane);
+        float2 v01 = f2(A.x, A.y), v23 = f2(A.z, A.w);
         if (!yident) {
-            const float4 B = *reinterpret_cast<const float4 *>(buf + c * vplane + r1);
-            v01 = fma2(ly2, sub2(pack2(B.x, B.y), v01), v01);
-            v23 = fma2(ly2, sub2(pack2(B.z, B.w), v23), v23);
+            const float4 B = *reinterpret_cast<const float4 *>(b_row + c * vplane);
+            v01 = fma2(ly2, f2(B.x, B.y), fma2(nly2, v01, v01));
+            v23 = fma2(ly2, f2(B.z, B.w), fma2(nly2, v23, v23));
         }
-        const uint64_t k2 = pack2(P.k[c], P.k[c]), b2 = pack2(P.b[c], P.b[c]);
-        const float2 n01 = unpack2(fma2(v01, k2, b2));
-        const float2 n23 = unpack2(fma2(v23, k2, b2));
+        const float2 k2 = f2(P.k[c], P.k[c]), b2 = f2(P.b[c], P.b[c]);
+        const float2 n01 = fma2(v01, k2, b2);
+        const float2 n23 = fma2(v23, k2, b2);
         if constexpr (!kBF16) {
             float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col;
             const float4 f4 = make_float4(n01.x, n01.y, n23.x, n23.y);
@@ -479,15 +496,13 @@ __global__ void __launch_bounds__(kThreads, 6) preprocess_kernel(const __grid_co
     const int end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * B / gridDim.x);
     if (begin >= end) return;
 
-    int ii = 0;  // image cursor of warps 0-1
-    AxisCursor &cur = s_cur[tid & 63];
+    AxisCursor &cur = s_cur[tid & 63];  // meaningful for warps 0-1 only
     if (warp < 2) {
         cur = AxisCursor();
-        ii = find_image(P, begin);
-        compute_taps(P, S[0], S[1], begin, ii, cur, warp, lane);
+        compute_taps(P, S[0], S[1], begin, cur, warp, lane);
     }
     __syncthreads();
-    if (warp < 2 && begin + 1 < end) compute_taps(P, S[1], S[0], begin + 1, ii, cur, warp, lane);
+    if (warp < 2 && begin + 1 < end) compute_taps(P, S[1], S[0], begin + 1, cur, warp, lane);
     issue_stage(P, S[0], raw, tid);
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
@@ -501,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 6) preprocess_kernel(const __grid_co
         asm volatile("cp.async.wait_all;" ::: "memory");
         __syncthreads();  // tile, hbuf and S[slot] free; raw holds block blk+1
         if (blk + 1 < end) finish_stage(P, S[slot ^ 1], raw, tile, TS, plane, tid);
-        if (warp < 2 && blk + 2 < end) compute_taps(P, S[slot], S[slot ^ 1], blk + 2, ii, cur, warp, lane);
+        if (warp < 2 && blk + 2 < end) compute_taps(P, S[slot], S[slot ^ 1], blk + 2, cur, warp, lane);
         __syncthreads();  // tile holds block blk+1, S[slot] the taps of blk+2, raw is free
         if (blk + 2 < end) issue_stage(P, S[slot], raw, tid);
         slot ^= 1;
