@@ -526,11 +526,10 @@ __global__ void __launch_bounds__(kThreads, 6) preprocess_kernel(const __grid_co
 template <bool kBF16>
 int launch_typed(const LaunchParams &lp, int64_t blocks, size_t smem_bytes, cudaStream_t stream) {
     auto kern = preprocess_kernel<kBF16>;
-    if (smem_bytes > 48 * 1024) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes)) !=
-            cudaSuccess)
-            return MIMO_ECUDA;
-    }
+    // the opt-in covers dynamic + static shared memory above the 48 KB default
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes)) !=
+        cudaSuccess)
+        return MIMO_ECUDA;
     // persistent grid: as many CTAs as can be resident at once
     int dev = 0, sms = 0, per_sm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
