@@ -231,7 +231,6 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
         fold_normalisation(p, &lp);
         int64_t blocks = 0;
         int32_t tr = 1, tc = 1, k = 0;
-        bool hpass = false;
         while (i < last && k < mimo::kMaxImagesPerLaunch &&
                blocks + v.plan.img[i].blocks <= static_cast<int64_t>(INT32_MAX)) {
             const ImagePlan &ip = v.plan.img[i];
@@ -247,7 +246,6 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
             // staging copies are 16-byte chunks that may run up to 15 bytes past
             // the image; they read nothing past the end of the caller's buffer
             d.limit = static_cast<int64_t>(src_bytes) - src_offsets[i];
-            hpass = hpass || (ip.flags & mimo::kIdentityCols) == 0;
             lp.block_start[k] = static_cast<int32_t>(blocks);
             blocks += ip.blocks;
             tr = std::max(tr, ip.tile_rows);
@@ -258,16 +256,16 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
         lp.block_start[k] = static_cast<int32_t>(blocks);
         lp.n = k;
         lp.tile_rows = tr;
-        lp.tile_stride = (tc + 3) & ~3;  // 16-byte rows: whole-float4 staging stores and loads
+        // 16-byte rows (whole-float4 staging stores and loads), at least the 32
+        // columns the in-place horizontal pass writes
+        lp.tile_stride = (std::max(tc, mimo::kBlock) + 3) & ~3;
         const size_t tile_floats = 3u * static_cast<size_t>(tr) * static_cast<size_t>(lp.tile_stride);
-        lp.hbuf = hpass ? static_cast<int32_t>(tile_floats) : 0;
-        const size_t hbuf_floats = hpass ? 3u * static_cast<size_t>(tr) * mimo::kBlock : 0u;
         // raw staging rows: a row segment of up to 4*tc bytes at any 16-byte
         // misalignment, plus the word a 12-byte RGB read may touch past it
         lp.raw_stride = ((32 + 4 * tc) + 15) & ~15;
         const size_t raw_floats = static_cast<size_t>(tr) * static_cast<size_t>(lp.raw_stride) / 4u;
-        lp.raw = static_cast<int32_t>(tile_floats + hbuf_floats);
-        const size_t smem = sizeof(float) * (tile_floats + hbuf_floats + raw_floats);
+        lp.raw = static_cast<int32_t>(tile_floats);  // tile | raw staging rows
+        const size_t smem = sizeof(float) * (tile_floats + raw_floats);
         const int st = mimo::launch_preprocess(lp, blocks, out_dtype, smem, stream);
         if (st != MIMO_OK) return st;
     }

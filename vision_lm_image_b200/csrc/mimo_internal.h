@@ -52,7 +52,6 @@ struct LaunchParams {
     int32_t n;           // images in this launch
     int32_t tile_rows;   // rows of the shared-memory tile (max over images)
     int32_t tile_stride; // row stride (floats, multiple of 4) of the tile
-    int32_t hbuf;        // float offset of the horizontal-pass buffer, 0 if unused
     int32_t raw;         // float offset of the raw staging rows
     int32_t raw_stride;  // bytes per raw staging row (multiple of 16)
     int32_t block_start[kMaxImagesPerLaunch + 1];  // prefix sum of merge blocks

@@ -9,8 +9,8 @@
 //   - copies the source row segments those taps touch into shared memory
 //     with 16-byte cp.async, then converts them to planar fp32 on the 0..255
 //     scale, compositing RGBA onto white on the way (function _to_rgb);
-//   - interpolates along W for every staged row (skipped when the width is
-//     not resized), then along H with packed f32x2 arithmetic, applies
+//   - interpolates along W for every staged row, in place (skipped when the
+//     width is not resized), then along H with packed f32x2 arithmetic, applies
 //     (x - 255*mean)/(255*std) folded to x*k + b (module docstring), and
 //     writes each 16-pixel row segment twice, once per temporal frame, laid
 //     out (c, tt, py, px) in merge-block row order (cortiq page, conventions);
@@ -396,21 +396,25 @@ __device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &
     const int flags = T.flags;
     const int nrows = T.nrows;
 
-    // horizontal pass (resized widths only): hbuf[c][j][dx]
+    // horizontal pass (resized widths only), in place: the warp owning tile
+    // row j reads every lane's two taps, then writes the 32 interpolated
+    // values over columns 0..31 of the same row
     const bool hpass = (flags & kIdentityCols) == 0;
     if (hpass) {
-        float *hb = tile + P.hbuf;
-        const int hplane = P.tile_rows * kBlock;
         const int x0 = T.tx[0][lane], x1 = T.tx[1][lane];
         const float lx = T.lx[lane];
         for (int j = warp; j < nrows; j += kThreads / 32) {
-            const float *t = tile + j * TS;
+            float *t = tile + j * TS;
+            float h[3];
 #pragma unroll
             for (int c = 0; c < 3; ++c) {
                 const float a = t[c * plane + x0];
                 const float b = t[c * plane + x1];
-                hb[c * hplane + j * kBlock + lane] = fmaf(lx, b - a, a);
+                h[c] = fmaf(lx, b - a, a);
             }
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 3; ++c) t[c * plane + lane] = h[c];
         }
         __syncthreads();
     }
@@ -425,12 +429,9 @@ __device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &
     const int q = lane & 3;
     const int dy = (mh << 4) | py;
     const int dx0 = (mw << 4) | (q << 2);
-    const float *buf = hpass ? tile + P.hbuf : tile;
-    const int stride = hpass ? kBlock : TS;
-    const int vplane = hpass ? P.tile_rows * kBlock : plane;
     const bool yident = (flags & kIdentityRows) != 0;
-    const float *a_row = buf + T.ty[0][dy] * stride + dx0;
-    const float *b_row = buf + T.ty[1][dy] * stride + dx0;
+    const float *a_row = tile + T.ty[0][dy] * TS + dx0;
+    const float *b_row = tile + T.ty[1][dy] * TS + dx0;
     // (1 - ly) a + ly b as two FMAs: a - ly a, then + ly b
     const float ly = T.ly[dy];
     const float2 ly2 = f2(ly, ly), nly2 = f2(-ly, -ly);
@@ -438,10 +439,10 @@ __device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &
     const int col = py * 16 + q * 4;
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
-        const float4 A = *reinterpret_cast<const float4 *>(a_row + c * vplane);
+        const float4 A = *reinterpret_cast<const float4 *>(a_row + c * plane);
         float2 v01 = f2(A.x, A.y), v23 = f2(A.z, A.w);
         if (!yident) {
-            const float4 B = *reinterpret_cast<const float4 *>(b_row + c * vplane);
+            const float4 B = *reinterpret_cast<const float4 *>(b_row + c * plane);
             v01 = fma2(ly2, f2(B.x, B.y), fma2(nly2, v01, v01));
             v23 = fma2(ly2, f2(B.z, B.w), fma2(nly2, v23, v23));
         }
@@ -482,7 +483,7 @@ __device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &
 template <bool kBF16>
 __global__ void __launch_bounds__(kThreads, 6) preprocess_kernel(const __grid_constant__ LaunchParams P) {
     extern __shared__ float4 smem4[];
-    float *const tile = reinterpret_cast<float *>(smem4);  // [3][rows][stride] | hbuf | raw bytes
+    float *const tile = reinterpret_cast<float *>(smem4);  // [3][rows][stride] | raw bytes
     uint8_t *const raw = reinterpret_cast<uint8_t *>(tile + P.raw);
     __shared__ TapSet S[2];
     __shared__ AxisCursor s_cur[64];  // one per lane of the two tap warps
@@ -514,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 6) preprocess_kernel(const __grid_co
     for (int blk = begin; blk < end; ++blk) {
         emit_block<kBF16>(P, S[slot], tile, TS, plane, tid, warp, lane);
         asm volatile("cp.async.wait_all;" ::: "memory");
-        __syncthreads();  // tile, hbuf and S[slot] free; raw holds block blk+1
+        __syncthreads();  // tile and S[slot] free; raw holds block blk+1
         if (blk + 1 < end) finish_stage(P, S[slot ^ 1], raw, tile, TS, plane, tid);
         if (warp < 2 && blk + 2 < end) compute_taps(P, S[slot], S[slot ^ 1], blk + 2, cur, warp, lane);
         __syncthreads();  // tile holds block blk+1, S[slot] the taps of blk+2, raw is free
