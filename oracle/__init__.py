@@ -74,6 +74,12 @@ def lib():
             L.oracle_patch_value.restype = ctypes.c_int
             L.oracle_column_permutation.argtypes = [_i64, _i64, _i64, _i32, _i64, _p]
             L.oracle_column_permutation.restype = None
+            L.oracle_patchify_column.argtypes = [_p, _i64, _i64, _i32, _i32, _i32, _p]
+            L.oracle_patchify_column.restype = None
+            L.oracle_rotary_positions.argtypes = [_i64, _i64, _i64, _i32, _i32, _p]
+            L.oracle_rotary_positions.restype = None
+            L.oracle_window_index.argtypes = [_i64, _i64, _i64, _i32, _i64, _p]
+            L.oracle_window_index.restype = None
             _lib = L
     return _lib
 
@@ -163,6 +169,30 @@ def patchify(planes: np.ndarray, patch=16, temporal=2, merge=2) -> np.ndarray:
     return out
 
 
+def patchify_column(planes: np.ndarray, patch=16, temporal=2, merge=2) -> np.ndarray:
+    planes = np.ascontiguousarray(planes, dtype=np.float64)
+    _, Hr, Wr = planes.shape
+    rows = (Hr // patch) * (Wr // patch)
+    out = np.empty((rows, 3 * temporal * patch * patch), np.float32)
+    lib().oracle_patchify_column(_ptr(planes), Hr, Wr, patch, temporal, merge, _ptr(out))
+    return out
+
+
+def rotary_positions(grid_h: int, grid_w: int, merge: int = 2, column_order: bool = False,
+                     grid_t: int = 1) -> np.ndarray:
+    """[rows, 2] int32 (patch row, patch column) of every emitted row."""
+    out = np.empty((grid_t * grid_h * grid_w, 2), np.int32)
+    lib().oracle_rotary_positions(grid_t, grid_h, grid_w, merge, int(column_order), _ptr(out))
+    return out
+
+
+def window_index(grid_h: int, grid_w: int, merge: int = 2, unit0: int = 0, grid_t: int = 1) -> np.ndarray:
+    """[units] int32: merge-order unit index of each unit in column-major order."""
+    out = np.empty(grid_t * (grid_h // merge) * (grid_w // merge), np.int32)
+    lib().oracle_window_index(grid_t, grid_h, grid_w, merge, unit0, _ptr(out))
+    return out
+
+
 def column_permutation(grid_h: int, grid_w: int, merge: int = 2, row0: int = 0, grid_t: int = 1) -> np.ndarray:
     out = np.empty(grid_t * grid_h * grid_w, np.int32)
     lib().oracle_column_permutation(grid_t, grid_h, grid_w, merge, row0, _ptr(out))
@@ -204,6 +234,18 @@ def patch_value(img: np.ndarray, resized_hw, row: int, col: int, mean, std,
     return float(v.value)
 
 
+def preprocess_image_column(img: np.ndarray, mean, std, min_pixels=8192, max_pixels=8388608,
+                            patch=16, temporal=2, merge=2):
+    """One image through the path with rows emitted in column order (units by block column)."""
+    img = np.ascontiguousarray(img, dtype=np.uint8)
+    H, W, _ = img.shape
+    Hr, Wr = smart_resize(H, W, patch * merge, min_pixels, max_pixels)
+    planes = load_planes(to_rgb(img))
+    resized = np.stack([resize_plane(planes[c], Hr, Wr) for c in range(3)])
+    rows = patchify_column(normalize_planes(resized, mean, std), patch, temporal, merge)
+    return rows, (1, Hr // patch, Wr // patch)
+
+
 def _flatten_one_level(images):
     flat = []
     for item in images:
@@ -215,19 +257,20 @@ def _flatten_one_level(images):
 
 
 def preprocess(images, mean, std, min_pixels=8192, max_pixels=8388608, column_perm=False,
-               patch=16, temporal=2, merge=2, threads: int = 1):
+               patch=16, temporal=2, merge=2, threads: int = 1, order: str = "merge",
+               positions: bool = False, window: bool = False):
     """The batch call: returns (pixel_values fp32 [sum rows, 1536], image_grid_thw int64 [n, 3], perm|None).
 
     ``threads`` > 1 runs independent images on a thread pool (ctypes drops the
     GIL inside the C code); the arithmetic is unchanged.
     """
     imgs = _flatten_one_level(images)
+    one = preprocess_image if order == "merge" else preprocess_image_column
     if threads > 1 and len(imgs) > 1:
         with ThreadPoolExecutor(max_workers=threads) as ex:
-            res = list(ex.map(lambda im: preprocess_image(im, mean, std, min_pixels, max_pixels,
-                                                          patch, temporal, merge), imgs))
+            res = list(ex.map(lambda im: one(im, mean, std, min_pixels, max_pixels, patch, temporal, merge), imgs))
     else:
-        res = [preprocess_image(im, mean, std, min_pixels, max_pixels, patch, temporal, merge) for im in imgs]
+        res = [one(im, mean, std, min_pixels, max_pixels, patch, temporal, merge) for im in imgs]
     cols = 3 * temporal * patch * patch
     pv = np.concatenate([r[0] for r in res], axis=0) if res else np.zeros((0, cols), np.float32)
     grid = np.array([r[1] for r in res], dtype=np.int64).reshape(-1, 3)
@@ -238,7 +281,16 @@ def preprocess(images, mean, std, min_pixels=8192, max_pixels=8388608, column_pe
             parts.append(column_permutation(gh, gw, merge, row0))
             row0 += gh * gw
         perm = np.concatenate(parts) if parts else np.zeros(0, np.int32)
-    return pv, grid, perm
+    if not (positions or window):
+        return pv, grid, perm
+    pos_parts, win_parts, unit0 = [], [], 0
+    for (_, gh, gw) in grid.tolist():
+        pos_parts.append(rotary_positions(gh, gw, merge, column_order=(order == "column")))
+        win_parts.append(window_index(gh, gw, merge, unit0))
+        unit0 += (gh // merge) * (gw // merge)
+    pos = np.concatenate(pos_parts) if pos_parts else np.zeros((0, 2), np.int32)
+    win = np.concatenate(win_parts) if win_parts else np.zeros(0, np.int32)
+    return pv, grid, perm, pos, win
 
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:

@@ -17,6 +17,11 @@
  *        conventions (T = 2, (c, tt, py, px) rows, merge-block row order,
  *        column order), functions resize_bilinear, smart_resize and
  *        column_permutation.
+ *   [V]  NeMo Automodel, "mimo_v2_flash.vision": MiMoVisionTransformer
+ *        _rotary_positions and _get_window_index, MiMoVisionRotaryEmbedding.
+ *        The pages give their signatures only; the tables here are the
+ *        reading stated above each function (positions of the emitted rows;
+ *        merge units in column-major order), pinned to hand-worked grids.
  *
  * Arithmetic: geometry in IEEE fp64 (as the Python original does), pixels in
  * fp64 from the uint8 values; every patch value is rounded to fp32 once, at
@@ -346,4 +351,77 @@ void oracle_column_permutation(int64_t grid_t, int64_t grid_h, int64_t grid_w,
             for (int64_t a = 0; a < gh2; ++a)   /* block row    */
                 for (int64_t k = 0; k < m * m; ++k)
                     perm[dst++] = (int32_t)(row0 + ((t * gh2 + a) * gw2 + b) * m * m + k);
+}
+
+/*
+ * [C] conventions: "whole merge units are listed by (t, block col, block
+ * row)" -- the same rows as oracle_patchify, emitted in column order: units
+ * by (t, block col, block row), the m*m rows of a unit kept together in
+ * (mh, mw) order. Equals the merge-order rows gathered with
+ * oracle_column_permutation.
+ */
+void oracle_patchify_column(const double *planes, int64_t Hr, int64_t Wr,
+                            int32_t patch, int32_t temporal, int32_t merge, float *out)
+{
+    const int64_t p = patch, T = temporal, m = merge;
+    const int64_t gh = Hr / p, gw = Wr / p;
+    const int64_t cols = 3 * T * p * p;
+    int64_t row = 0;
+    for (int64_t bw = 0; bw < gw / m; ++bw)
+        for (int64_t bh = 0; bh < gh / m; ++bh)
+            for (int64_t mh = 0; mh < m; ++mh)
+                for (int64_t mw = 0; mw < m; ++mw, ++row) {
+                    int64_t col = 0;
+                    for (int64_t c = 0; c < 3; ++c)
+                        for (int64_t tt = 0; tt < T; ++tt)
+                            for (int64_t py = 0; py < p; ++py)
+                                for (int64_t px = 0; px < p; ++px, ++col) {
+                                    int64_t y = (bh * m + mh) * p + py;
+                                    int64_t x = (bw * m + mw) * p + px;
+                                    out[row * cols + col] = (float)planes[c * Hr * Wr + y * Wr + x];
+                                }
+                }
+}
+
+/*
+ * Two-dimensional rotary positions of the vision tower (NeMo Automodel
+ * "mimo_v2_flash.vision", MiMoVisionTransformer._rotary_positions and
+ * MiMoVisionRotaryEmbedding: two-dimensional frequencies): for every patch
+ * row, its patch row index and patch column index in the grid, in the order
+ * the rows are emitted (merge-block order, or column order when
+ * column_order != 0, [C] conventions: "the RoPE tables are permuted the same
+ * way"). pos has 2 entries per row: (h, w).
+ */
+void oracle_rotary_positions(int64_t grid_t, int64_t grid_h, int64_t grid_w, int32_t merge,
+                             int32_t column_order, int32_t *pos)
+{
+    const int64_t m = merge, gh2 = grid_h / m, gw2 = grid_w / m;
+    int64_t row = 0;
+    for (int64_t t = 0; t < grid_t; ++t)
+        for (int64_t a = 0; a < (column_order ? gw2 : gh2); ++a)
+            for (int64_t b = 0; b < (column_order ? gh2 : gw2); ++b)
+                for (int64_t mh = 0; mh < m; ++mh)
+                    for (int64_t mw = 0; mw < m; ++mw, ++row) {
+                        int64_t bh = column_order ? b : a;
+                        int64_t bw = column_order ? a : b;
+                        pos[2 * row + 0] = (int32_t)(bh * m + mh);
+                        pos[2 * row + 1] = (int32_t)(bw * m + mw);
+                    }
+}
+
+/*
+ * Window index over merge units (MiMoVisionTransformer._get_window_index with
+ * column_major; [C] conventions: column-order windows list whole merge units
+ * by (t, block col, block row)): win[j] = merge-order index of the j-th unit
+ * in column-major order, offset by unit0 (the image's first unit in a batch).
+ */
+void oracle_window_index(int64_t grid_t, int64_t grid_h, int64_t grid_w, int32_t merge,
+                         int64_t unit0, int32_t *win)
+{
+    const int64_t m = merge, gh2 = grid_h / m, gw2 = grid_w / m;
+    int64_t j = 0;
+    for (int64_t t = 0; t < grid_t; ++t)
+        for (int64_t b = 0; b < gw2; ++b)
+            for (int64_t a = 0; a < gh2; ++a)
+                win[j++] = (int32_t)(unit0 + (t * gh2 + a) * gw2 + b);
 }

@@ -1,0 +1,73 @@
+"""Pins for the oracle's column-order emission and the vision-tower index tables.
+
+Reading (docs.rs 'cortiq_engine::mimo_vision', conventions; NeMo Automodel 'mimo_v2_flash.vision',
+MiMoVisionTransformer._rotary_positions / _get_window_index): column order lists whole merge units
+by (t, block col, block row); the rotary positions are each emitted row's (patch row, patch column)
+and are permuted with the rows; the window index lists merge units in column-major order.
+"""
+import numpy as np
+import torch
+
+import oracle
+import workloads
+
+
+def test_positions_hand_worked_4x6():
+    pos = oracle.rotary_positions(4, 6)
+    want = []
+    for bh in range(2):
+        for bw in range(3):
+            for mh in range(2):
+                for mw in range(2):
+                    want.append((2 * bh + mh, 2 * bw + mw))
+    assert pos.tolist() == [list(w) for w in want]
+    assert pos[:8].tolist() == [[0, 0], [0, 1], [1, 0], [1, 1], [0, 2], [0, 3], [1, 2], [1, 3]]
+
+
+def test_positions_match_reshape_formulation():
+    # hpos/wpos of a (gh, gw) grid re-ordered into merge blocks with reshape/permute
+    for gh, gw in [(2, 2), (4, 6), (8, 6), (68, 120), (2, 24)]:
+        h = torch.arange(gh)[:, None].expand(gh, gw)
+        w = torch.arange(gw)[None, :].expand(gh, gw)
+        def merge(t):
+            return t.reshape(gh // 2, 2, gw // 2, 2).permute(0, 2, 1, 3).reshape(-1)
+        ref = torch.stack([merge(h), merge(w)], dim=1).numpy()
+        assert np.array_equal(oracle.rotary_positions(gh, gw), ref)
+
+
+def test_column_order_tables_follow_the_permutation():
+    for gh, gw in [(2, 2), (4, 6), (6, 4), (68, 120)]:
+        perm = oracle.column_permutation(gh, gw)
+        pos = oracle.rotary_positions(gh, gw)
+        assert np.array_equal(oracle.rotary_positions(gh, gw, column_order=True), pos[perm])
+        win = oracle.window_index(gh, gw)
+        assert np.array_equal(win, perm[::4] // 4)
+        assert np.array_equal(np.sort(win), np.arange(gh * gw // 4))
+
+
+def test_window_index_hand_worked_and_offset():
+    assert oracle.window_index(4, 6).tolist() == [0, 3, 1, 4, 2, 5]
+    assert oracle.window_index(4, 6, unit0=10).tolist() == [10, 13, 11, 14, 12, 15]
+    assert oracle.window_index(2, 2).tolist() == [0]
+
+
+def test_column_rows_are_merge_rows_permuted():
+    img = workloads.random_small_batch(81, 1, max_side=200)[0]
+    rows, g = oracle.preprocess_image(img, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    col, gc = oracle.preprocess_image_column(img, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    assert g == gc
+    perm = oracle.column_permutation(g[1], g[2])
+    assert np.array_equal(col, rows[perm])
+
+
+def test_batch_tables_are_batch_global():
+    imgs = workloads.random_small_batch(82, 4, max_side=150)
+    pv, grid, perm, pos, win = oracle.preprocess(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD,
+                                                 column_perm=True, positions=True, window=True)
+    pvc, _, _, posc, winc = oracle.preprocess(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD,
+                                              column_perm=True, positions=True, window=True, order="column")
+    assert np.array_equal(pvc, pv[perm])
+    assert np.array_equal(posc, pos[perm])
+    assert np.array_equal(win, winc)
+    assert np.array_equal(win, perm[::4] // 4)
+    assert pos.shape == (pv.shape[0], 2) and win.shape == (pv.shape[0] // 4,)
