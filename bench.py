@@ -55,6 +55,7 @@ def parse():
     ap.add_argument("--workload", default="c5", choices=["c2", "c3", "c4", "c5"])
     ap.add_argument("--dtype", default=None, choices=["f32", "bf16"])
     ap.add_argument("--images", type=int, default=None, help="override the workload's image count")
+    ap.add_argument("--order", default="merge", choices=["merge", "column"], help="row order of the output")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -246,7 +247,7 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        mimo.preprocess_batch(params, packed, out, perm, stream)
+        mimo.preprocess_batch_ex(params, packed, out, perm, order=args.order, stream=stream)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -321,6 +322,7 @@ def run_ours(args, rank, world, local_rank):
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": args.workload, "description": w["description"], "images_per_gpu": n_img,
                        "out_dtype": out_dtype, "column_perm": perm is not None, "rows_per_gpu": total,
+                       "row_order": args.order,
                        "l2": "inputs and outputs larger than L2 (no flush)", "parallelism": f"dp{world}"},
             "output_gbs": out_gbs,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

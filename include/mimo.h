@@ -64,6 +64,14 @@ typedef enum {
     MIMO_BF16 = 1   /* bfloat16, rounded to nearest-even from the float32 value */
 } mimo_dtype;
 
+typedef enum {
+    MIMO_ORDER_MERGE = 0,  /* rows by (t, block row, block col, mh, mw): the processor's order */
+    MIMO_ORDER_COLUMN = 1  /* merge units by (t, block col, block row), a unit's 4 rows kept
+                              together (cortiq page, conventions: column-order windows);
+                              the same rows as MIMO_ORDER_MERGE gathered with the column
+                              permutation */
+} mimo_row_order;
+
 /*
  * Processor knobs (class MimoV2ImageProcessor constructor; per-call
  * min_pixels / max_pixels overrides of __call__ are expressed by passing a
@@ -145,6 +153,45 @@ int mimo_preprocess_batch(const mimo_params *p, int32_t n,
                           const int32_t *heights, const int32_t *widths, const int32_t *channels,
                           int32_t out_dtype, void *d_out, int64_t out_rows_capacity,
                           int32_t *d_column_perm, void *stream);
+
+/*
+ * Outputs of mimo_preprocess_batch_ex. Every pointer is a device pointer,
+ * 16-byte aligned; the tables are optional (NULL = not written) and index the
+ * whole batch, so they need total_rows to fit int32 (MIMO_EOVERFLOW).
+ *   out_dtype, d_out, out_rows_capacity: as in mimo_preprocess_batch.
+ *   row_order:      MIMO_ORDER_MERGE or MIMO_ORDER_COLUMN; only the position
+ *                   of whole rows changes, never their contents.
+ *   d_column_perm:  int32 [total_rows], perm[j] = merge-order row of the j-th
+ *                   row in column order (column_permutation), whatever
+ *                   row_order is.
+ *   d_positions:    int32 [total_rows][2], (patch row, patch column) of every
+ *                   emitted row in the image's patch grid: the 2-D rotary
+ *                   positions of the vision tower (vision page,
+ *                   MiMoVisionTransformer._rotary_positions), in the emitted
+ *                   order.
+ *   d_window_index: int32 [total_rows / 4], j-th entry = merge-order index of
+ *                   the j-th merge unit in column-major order, batch-global
+ *                   (vision page, MiMoVisionTransformer._get_window_index with
+ *                   column_major; cortiq page, conventions).
+ */
+typedef struct {
+    int32_t out_dtype;
+    int32_t row_order;
+    void *d_out;
+    int64_t out_rows_capacity;
+    int32_t *d_column_perm;
+    int32_t *d_positions;
+    int32_t *d_window_index;
+} mimo_outputs;
+
+/* The fused pixel path with the row order and the vision-tower index tables
+ * chosen by `out`; all other arguments and guarantees as in
+ * mimo_preprocess_batch (which is this call with merge order, no positions
+ * and no window index). */
+int mimo_preprocess_batch_ex(const mimo_params *p, int32_t n,
+                             const uint8_t *d_src, size_t src_bytes, const int64_t *src_offsets,
+                             const int32_t *heights, const int32_t *widths, const int32_t *channels,
+                             const mimo_outputs *out, void *stream);
 
 /*
  * The same path from host memory to host memory (inputs copied in, rows and

@@ -252,3 +252,32 @@ def test_device_validation_errors():
     with pytest.raises(mimo.MimoError) as e:
         mimo.preprocess_batch(params, packed, shifted)
     assert e.value.status == 6
+
+
+# ---------------------------------------------------------------- row order and index tables
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_column_order_and_tables_match_oracle(dtype):
+    imgs = workloads.random_small_batch(301, 12, max_side=280, min_side=1)
+    mean, std = workloads.CLIP_MEAN, workloads.CLIP_STD
+    for order in ("merge", "column"):
+        pv, grid, perm, pos, win = mimo.preprocess(imgs, mean, std, dtype=dtype, column_perm=True, order=order,
+                                                   positions=True, window_index=True)
+        torch.cuda.synchronize()
+        ref, rgrid, rperm, rpos, rwin = oracle.preprocess(imgs, mean, std, column_perm=True, order=order,
+                                                          positions=True, window=True, threads=8)
+        assert np.array_equal(grid.numpy(), rgrid)
+        assert np.array_equal(perm.cpu().numpy(), rperm)
+        assert np.array_equal(pos.cpu().numpy(), rpos)
+        assert np.array_equal(win.cpu().numpy(), rwin)
+        if dtype == torch.float32:
+            assert_fp32_close(pv.cpu().numpy(), ref, order)
+        else:
+            assert_bf16_close(pv, ref, order)
+
+
+def test_column_order_is_a_row_gather_full_c5():
+    w = workloads.workload("c5", n_images=8)
+    a, _, perm = gpu_run(w["images"], w["mean"], w["std"], column_perm=True)
+    b, _, _ = mimo.preprocess(w["images"], w["mean"], w["std"], order="column")
+    torch.cuda.synchronize()
+    assert torch.equal(b, a[perm.long()])

@@ -218,9 +218,16 @@ void fold_normalisation(const mimo_params *p, mimo::LaunchParams *lp) {
 // Launches images [first, last) of a validated batch, cut into launches of at
 // most kMaxImagesPerLaunch images and INT32_MAX blocks. Output rows and
 // source offsets stay batch-global.
+struct Tables {
+    int32_t order = MIMO_ORDER_MERGE;
+    int32_t *pos = nullptr;
+    int32_t *win = nullptr;
+};
+
 int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_t last, const uint8_t *d_src,
                  size_t src_bytes, const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
-                 const int32_t *channels, int32_t out_dtype, void *d_out, int32_t *d_perm, void *stream) {
+                 const int32_t *channels, int32_t out_dtype, void *d_out, int32_t *d_perm, void *stream,
+                 const Tables &tables = Tables()) {
     static thread_local mimo::LaunchParams lp;  // 23 KB: kept off the stack
     int32_t i = first;
     while (i < last) {
@@ -228,6 +235,9 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
         lp.src = d_src;
         lp.out = d_out;
         lp.perm = d_perm;
+        lp.pos = tables.pos;
+        lp.win = tables.win;
+        lp.order = tables.order;
         fold_normalisation(p, &lp);
         int64_t blocks = 0;
         int32_t tr = 1, tc = 1, k = 0;
@@ -328,16 +338,40 @@ int mimo_plan_batch(int32_t n, const int32_t *heights, const int32_t *widths, co
     return MIMO_OK;
 }
 
+int mimo_preprocess_batch_ex(const mimo_params *p, int32_t n, const uint8_t *d_src, size_t src_bytes,
+                             const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
+                             const int32_t *channels, const mimo_outputs *out, void *stream) {
+    if (!out) return MIMO_EINVAL;
+    if (out->row_order != MIMO_ORDER_MERGE && out->row_order != MIMO_ORDER_COLUMN) return MIMO_EINVAL;
+    Validated v;
+    int st = validate_batch(p, n, d_src, src_bytes, src_offsets, heights, widths, channels, out->out_dtype,
+                            out->d_out, out->out_rows_capacity, out->d_column_perm, &v);
+    if (st != MIMO_OK || n == 0) return st;
+    // the tables are optional; like the permutation they hold batch-global int32 indices
+    for (const void *t : {static_cast<const void *>(out->d_positions), static_cast<const void *>(out->d_window_index)}) {
+        if (!t) continue;
+        if (!aligned16(t)) return MIMO_EALIGN;
+        if (v.total_rows > INT32_MAX) return MIMO_EOVERFLOW;
+    }
+    Tables tables;
+    tables.order = out->row_order;
+    tables.pos = out->d_positions;
+    tables.win = out->d_window_index;
+    return launch_range(p, v, 0, n, d_src, src_bytes, src_offsets, heights, widths, channels, out->out_dtype,
+                        out->d_out, out->d_column_perm, stream, tables);
+}
+
 int mimo_preprocess_batch(const mimo_params *p, int32_t n, const uint8_t *d_src, size_t src_bytes,
                           const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
                           const int32_t *channels, int32_t out_dtype, void *d_out, int64_t out_rows_capacity,
                           int32_t *d_column_perm, void *stream) {
-    Validated v;
-    const int st = validate_batch(p, n, d_src, src_bytes, src_offsets, heights, widths, channels, out_dtype, d_out,
-                                  out_rows_capacity, d_column_perm, &v);
-    if (st != MIMO_OK || n == 0) return st;
-    return launch_range(p, v, 0, n, d_src, src_bytes, src_offsets, heights, widths, channels, out_dtype, d_out,
-                        d_column_perm, stream);
+    mimo_outputs out{};
+    out.out_dtype = out_dtype;
+    out.row_order = MIMO_ORDER_MERGE;
+    out.d_out = d_out;
+    out.out_rows_capacity = out_rows_capacity;
+    out.d_column_perm = d_column_perm;
+    return mimo_preprocess_batch_ex(p, n, d_src, src_bytes, src_offsets, heights, widths, channels, &out, stream);
 }
 
 int mimo_preprocess_batch_host(const mimo_params *p, int32_t n, const uint8_t *h_src, size_t src_bytes,

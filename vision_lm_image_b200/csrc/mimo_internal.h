@@ -48,6 +48,10 @@ struct LaunchParams {
     const uint8_t *src;
     void *out;
     int32_t *perm;       // may be null
+    int32_t *pos;        // may be null: (patch row, patch column) per emitted row
+    int32_t *win;        // may be null: merge-order unit of each column-major unit
+    int32_t order;       // 0: merge-block order, 1: column order
+    int32_t pad0;
     float k[3], b[3];    // normalisation folded: v = x*k[c] + b[c]
     int32_t n;           // images in this launch
     int32_t tile_rows;   // rows of the shared-memory tile (max over images)

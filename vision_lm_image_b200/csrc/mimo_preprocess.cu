@@ -89,7 +89,8 @@ struct TapSet {
     uint32_t qmagic, cmagic;  // x / Q and x / CQ as (x * magic) >> 16 for the job counts here
     int64_t src_off;         // image offset in the source buffer
     int64_t limit;           // bytes readable from src_off (caller's buffer end)
-    int64_t row_base;        // first output row of the block
+    int64_t row0;            // first output row of the image
+    int64_t row_base;        // first output row of the block, in the emitted order
 };
 
 // Per-lane state of a tap warp across the blocks of a CTA: the exact floor
@@ -253,7 +254,11 @@ __device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, c
         T.bw = bw;
         T.src_off = D.src_off;
         T.limit = D.limit;
-        T.row_base = D.row0 + 4LL * (static_cast<int64_t>(bh) * gw2 + bw);
+        T.row0 = D.row0;
+        // merge order lists units by (block row, block col), column order by (block col, block row)
+        const int64_t unit = P.order ? static_cast<int64_t>(bw) * (Hr / kBlock) + bh
+                                     : static_cast<int64_t>(bh) * gw2 + bw;
+        T.row_base = D.row0 + 4 * unit;
     }
 }
 
@@ -466,12 +471,24 @@ __device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &
         }
     }
 
-    // column-order permutation: unit (bh, bw) is listed at (bw, bh)
-    if (P.perm != nullptr && tid == 0) {
-        const int64_t unit_row0 = T.row_base - 4LL * (static_cast<int64_t>(T.bh) * T.gw2 + T.bw);
-        const int64_t dst = unit_row0 + 4LL * (static_cast<int64_t>(T.bw) * T.gh2 + T.bh);
-        const int32_t s0 = static_cast<int32_t>(T.row_base);
-        __stcs(reinterpret_cast<int4 *>(P.perm + dst), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
+    // the merge unit's table entries: permutation (thread 0), rotary
+    // positions of its 4 emitted rows (thread 1), window index (thread 2)
+    if (tid < 3) {
+        const int64_t src_unit = static_cast<int64_t>(T.bh) * T.gw2 + T.bw;  // merge order
+        const int64_t dst_unit = static_cast<int64_t>(T.bw) * T.gh2 + T.bh;  // column order
+        if (tid == 0 && P.perm != nullptr) {
+            const int32_t s0 = static_cast<int32_t>(T.row0 + 4 * src_unit);
+            __stcs(reinterpret_cast<int4 *>(P.perm + T.row0 + 4 * dst_unit), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
+        } else if (tid == 1 && P.pos != nullptr) {
+            // rows (mh, mw) = (0,0), (0,1), (1,0), (1,1) of the unit
+            const int32_t h = 2 * T.bh, w = 2 * T.bw;
+            int4 *d = reinterpret_cast<int4 *>(P.pos + 2 * T.row_base);
+            __stcs(d, make_int4(h, w, h, w + 1));
+            __stcs(d + 1, make_int4(h + 1, w, h + 1, w + 1));
+        } else if (tid == 2 && P.win != nullptr) {
+            const int64_t u0 = T.row0 / 4;
+            P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
+        }
     }
 }
 

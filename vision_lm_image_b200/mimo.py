@@ -25,6 +25,7 @@ from . import build as _build
 
 OK = 0
 F32, BF16 = 0, 1
+ORDER_MERGE, ORDER_COLUMN = 0, 1
 ROW_WIDTH = 1536
 ALIGN = 16
 
@@ -34,7 +35,8 @@ STATUS_NAMES = {
     10: "MIMO_ERANGE", 11: "MIMO_ELIMIT",
 }
 EXPORTED = ("mimo_params_default", "mimo_smart_resize", "mimo_num_patches", "mimo_plan_batch",
-            "mimo_preprocess_batch", "mimo_preprocess_batch_host", "mimo_preprocess_batch_host_noalloc",
+            "mimo_preprocess_batch", "mimo_preprocess_batch_ex", "mimo_preprocess_batch_host",
+            "mimo_preprocess_batch_host_noalloc",
             "mimo_status_string", "mimo_version")
 NOALLOC_STAGING_BYTES = 64 << 20
 
@@ -60,6 +62,18 @@ class MimoParams(ctypes.Structure):
         ("max_pixels", ctypes.c_int64),
         ("image_mean", ctypes.c_float * 3),
         ("image_std", ctypes.c_float * 3),
+    ]
+
+
+class MimoOutputs(ctypes.Structure):
+    _fields_ = [
+        ("out_dtype", ctypes.c_int32),
+        ("row_order", ctypes.c_int32),
+        ("d_out", ctypes.c_void_p),
+        ("out_rows_capacity", ctypes.c_int64),
+        ("d_column_perm", ctypes.c_void_p),
+        ("d_positions", ctypes.c_void_p),
+        ("d_window_index", ctypes.c_void_p),
     ]
 
 
@@ -94,6 +108,9 @@ def lib() -> ctypes.CDLL:
             L.mimo_preprocess_batch.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p, _i32,
                                                 _p, _i64, _p, _p]
             L.mimo_preprocess_batch.restype = ctypes.c_int
+            L.mimo_preprocess_batch_ex.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p,
+                                                   ctypes.POINTER(MimoOutputs), _p]
+            L.mimo_preprocess_batch_ex.restype = ctypes.c_int
             L.mimo_preprocess_batch_host.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p,
                                                      _i32, _p, _i64, _p, _p, _sz, _p, _i64, _p, _p]
             L.mimo_preprocess_batch_host.restype = ctypes.c_int
@@ -266,14 +283,37 @@ def _dtype_code(dtype) -> int:
     raise ValueError(f"unsupported output dtype {dtype}")
 
 
+def preprocess_batch_ex(params: MimoParams, packed: PackedBatch, out, perm=None, positions=None, window=None,
+                        order: str = "merge", stream=None) -> None:
+    """Raw ABI call of mimo_preprocess_batch_ex: row order and the optional index tables (device tensors)."""
+    buf = packed.buffer
+    o = MimoOutputs()
+    o.out_dtype = _dtype_code(out.dtype)
+    o.row_order = {"merge": ORDER_MERGE, "column": ORDER_COLUMN}[order]
+    o.d_out = out.data_ptr()
+    o.out_rows_capacity = out.shape[0] if out.ndim == 2 else 0
+    o.d_column_perm = perm.data_ptr() if perm is not None else None
+    o.d_positions = positions.data_ptr() if positions is not None else None
+    o.d_window_index = window.data_ptr() if window is not None else None
+    st = lib().mimo_preprocess_batch_ex(
+        ctypes.byref(params), packed.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
+        packed.offsets.ctypes.data, packed.heights.ctypes.data, packed.widths.ctypes.data,
+        packed.channels.ctypes.data, ctypes.byref(o), _stream_handle(stream, buf.device))
+    _check(st, "preprocess_batch_ex")
+
+
 def preprocess(images, mean=None, std=None, min_pixels: int | None = None, max_pixels: int | None = None,
-               dtype=None, column_perm: bool = False, device="cuda", stream=None):
+               dtype=None, column_perm: bool = False, device="cuda", stream=None, order: str = "merge",
+               positions: bool = False, window_index: bool = False):
     """The processor call on the GPU: returns (pixel_values, image_grid_thw, perm | None).
 
     ``images``: HWC uint8 numpy arrays or torch tensors (CPU or CUDA), RGB or
     RGBA, or a list of such lists (flattened one level). ``pixel_values`` is a
     CUDA tensor [total_patches, 1536] (float32 by default, bfloat16 on
-    request); ``image_grid_thw`` a CPU int64 tensor [n, 3].
+    request); ``image_grid_thw`` a CPU int64 tensor [n, 3]. ``order="column"``
+    emits the rows in column order. With ``positions`` or ``window_index`` the
+    result gains two more entries: the int32 [rows, 2] rotary positions of the
+    emitted rows and the int32 [rows / 4] window index (None when not asked).
     """
     import torch
 
@@ -287,7 +327,11 @@ def preprocess(images, mean=None, std=None, min_pixels: int | None = None, max_p
     total = int(offs[-1])
     out = torch.empty((total, ROW_WIDTH), dtype=dtype, device=dev)
     perm = torch.empty(total, dtype=torch.int32, device=dev) if column_perm else None
-    preprocess_batch(params, packed, out, perm, stream)
+    pos = torch.empty((total, 2), dtype=torch.int32, device=dev) if positions else None
+    win = torch.empty(total // 4, dtype=torch.int32, device=dev) if window_index else None
+    preprocess_batch_ex(params, packed, out, perm, pos, win, order, stream)
+    if positions or window_index:
+        return out, torch.from_numpy(grid), perm, pos, win
     return out, torch.from_numpy(grid), perm
 
 
