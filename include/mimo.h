@@ -246,6 +246,22 @@ int mimo_preprocess_batch_host_noalloc(const mimo_params *p, int32_t n,
                                        int32_t out_dtype, void *h_out, int64_t out_rows_capacity,
                                        int32_t *h_column_perm, void *stream);
 
+/*
+ * Prompt placeholder expansion (cortiq page, expand_prompt_ids): copies `ids`
+ * to `out`, replacing the k-th occurrence of `pad_id` by counts[k] copies of
+ * it. counts[k] is the number of vision tokens of the k-th media item:
+ * mimo_num_patches / merge_size^2 for an image (get_number_of_image_patches
+ * before the merge reduction, processing page). Host only.
+ *   ids: host [n_ids]; counts: host [n_items], each >= 0; out: host
+ *   [out_capacity]; *out_len receives the expanded length.
+ * Errors: MIMO_EINVAL when the prompt holds a different number of
+ * placeholders than n_items or a count is negative; MIMO_ECAPACITY when the
+ * expansion does not fit out_capacity (nothing useful is left in out).
+ */
+int mimo_expand_prompt_ids(const int32_t *ids, int64_t n_ids, int32_t pad_id,
+                           const int64_t *counts, int64_t n_items,
+                           int32_t *out, int64_t out_capacity, int64_t *out_len);
+
 /* Static description of a status code. */
 const char *mimo_status_string(int status);
 

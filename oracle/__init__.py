@@ -80,6 +80,8 @@ def lib():
             L.oracle_rotary_positions.restype = None
             L.oracle_window_index.argtypes = [_i64, _i64, _i64, _i32, _i64, _p]
             L.oracle_window_index.restype = None
+            L.oracle_expand_prompt_ids.argtypes = [_p, _i64, _i32, _p, _i64, _p, _i64]
+            L.oracle_expand_prompt_ids.restype = _i64
             _lib = L
     return _lib
 
@@ -244,6 +246,18 @@ def preprocess_image_column(img: np.ndarray, mean, std, min_pixels=8192, max_pix
     resized = np.stack([resize_plane(planes[c], Hr, Wr) for c in range(3)])
     rows = patchify_column(normalize_planes(resized, mean, std), patch, temporal, merge)
     return rows, (1, Hr // patch, Wr // patch)
+
+
+def expand_prompt_ids(ids, pad_id: int, counts) -> np.ndarray:
+    """Expands the k-th ``pad_id`` of ``ids`` into ``counts[k]`` copies."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    counts = np.ascontiguousarray(counts, dtype=np.int64)
+    cap = int(ids.size + max(int(counts.sum()), 0))
+    out = np.empty(max(cap, 1), np.int32)
+    n = lib().oracle_expand_prompt_ids(_ptr(ids), ids.size, pad_id, _ptr(counts), counts.size, _ptr(out), cap)
+    if n < 0:
+        raise OracleError(EINVAL, "placeholder count does not match the items")
+    return out[:n]
 
 
 def _flatten_one_level(images):

@@ -425,3 +425,35 @@ void oracle_window_index(int64_t grid_t, int64_t grid_h, int64_t grid_w, int32_t
             for (int64_t a = 0; a < gh2; ++a)
                 win[j++] = (int32_t)(unit0 + (t * gh2 + a) * gw2 + b);
 }
+
+/*
+ * [C] expand_prompt_ids: each media placeholder token of the rendered prompt
+ * is expanded into as many copies as the media item has vision tokens (for an
+ * image: grid_h * grid_w / merge^2, [P] get_number_of_image_patches divided
+ * by the merge reduction). Placeholders are matched to items in order.
+ * Returns the expanded length, or -1 if the prompt holds a different number
+ * of placeholders than items, or -2 if out_capacity is too small.
+ */
+int64_t oracle_expand_prompt_ids(const int32_t *ids, int64_t n_ids, int32_t pad_id,
+                                 const int64_t *counts, int64_t n_items,
+                                 int32_t *out, int64_t out_capacity)
+{
+    int64_t used = 0, len = 0;
+    for (int64_t i = 0; i < n_ids; ++i) {
+        if (ids[i] == pad_id) {
+            if (used >= n_items)
+                return -1;
+            for (int64_t k = 0; k < counts[used]; ++k) {
+                if (len >= out_capacity)
+                    return -2;
+                out[len++] = pad_id;
+            }
+            ++used;
+        } else {
+            if (len >= out_capacity)
+                return -2;
+            out[len++] = ids[i];
+        }
+    }
+    return used == n_items ? len : -1;
+}

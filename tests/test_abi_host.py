@@ -150,3 +150,35 @@ def test_validation_statuses():
     assert _call(p=p) == 5                                  # std must be > 0
     p = mimo.make_params(merge_size=1)
     assert _call(p=p) == 5
+
+
+def test_expand_prompt_ids_matches_oracle():
+    rng = np.random.Generator(np.random.PCG64(41))
+    PAD = 99
+    for _ in range(200):
+        n_items = int(rng.integers(0, 6))
+        sizes = [(int(rng.integers(1, 3000)), int(rng.integers(1, 3000))) for _ in range(n_items)]
+        sizes = [(h, w) for h, w in sizes if oracle.smart_resize_status(h, w) == oracle.OK]
+        counts = [mimo.media_tokens(h, w) for h, w in sizes]
+        assert counts == [oracle.get_number_of_image_patches(h, w) // 4 for h, w in sizes]
+        text = rng.integers(0, 50, size=int(rng.integers(0, 20))).tolist()
+        ids = text[:]
+        for _ in counts:
+            ids.insert(int(rng.integers(0, len(ids) + 1)), PAD)
+        assert np.array_equal(mimo.expand_prompt_ids(ids, PAD, counts), oracle.expand_prompt_ids(ids, PAD, counts))
+
+
+def test_expand_prompt_ids_errors():
+    with pytest.raises(mimo.MimoError) as e:
+        mimo.expand_prompt_ids([1, 7, 7], 7, [3])
+    assert e.value.status == 1
+    with pytest.raises(mimo.MimoError) as e:
+        mimo.expand_prompt_ids([7], 7, [-1])
+    assert e.value.status == 1
+    ids = np.array([7], np.int32)
+    counts = np.array([5], np.int64)
+    out = np.empty(3, np.int32)
+    n = ctypes.c_int64()
+    st = mimo.lib().mimo_expand_prompt_ids(ids.ctypes.data, 1, 7, counts.ctypes.data, 1, out.ctypes.data, 3,
+                                           ctypes.byref(n))
+    assert st == 7

@@ -71,3 +71,23 @@ def test_batch_tables_are_batch_global():
     assert np.array_equal(win, winc)
     assert np.array_equal(win, perm[::4] // 4)
     assert pos.shape == (pv.shape[0], 2) and win.shape == (pv.shape[0] // 4,)
+
+
+def test_expand_prompt_ids_hand_worked():
+    PAD = 151655
+    # two images: 16x192 -> grid (1, 2, 24) -> 12 tokens; 64x48 -> grid (1, 8, 6) -> 12 tokens
+    counts = [oracle.get_number_of_image_patches(16, 192) // 4, oracle.get_number_of_image_patches(64, 48) // 4]
+    assert counts == [12, 12]
+    ids = [1, 2, PAD, 3, PAD, 4]
+    out = oracle.expand_prompt_ids(ids, PAD, counts)
+    assert out.tolist() == [1, 2] + [PAD] * 12 + [3] + [PAD] * 12 + [4]
+    assert oracle.expand_prompt_ids([5, 6], PAD, []).tolist() == [5, 6]
+    assert oracle.expand_prompt_ids([PAD], PAD, [0]).tolist() == []
+
+
+def test_expand_prompt_ids_rejects_a_count_mismatch():
+    import pytest
+    with pytest.raises(oracle.OracleError):
+        oracle.expand_prompt_ids([1, 7, 7], 7, [3])
+    with pytest.raises(oracle.OracleError):
+        oracle.expand_prompt_ids([1, 7], 7, [3, 4])

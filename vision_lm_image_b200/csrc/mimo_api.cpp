@@ -530,6 +530,33 @@ int mimo_preprocess_batch_host_noalloc(const mimo_params *p, int32_t n, const ui
     return cudaStreamSynchronize(s) == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
 }
 
+int mimo_expand_prompt_ids(const int32_t *ids, int64_t n_ids, int32_t pad_id, const int64_t *counts,
+                           int64_t n_items, int32_t *out, int64_t out_capacity, int64_t *out_len) {
+    if (n_ids < 0 || n_items < 0 || out_capacity < 0 || !out_len) return MIMO_EINVAL;
+    if ((n_ids > 0 && !ids) || (n_items > 0 && !counts) || (out_capacity > 0 && !out)) return MIMO_EINVAL;
+    // sizes first: placeholders must match the items one to one
+    int64_t pads = 0, total = 0;
+    for (int64_t i = 0; i < n_ids; ++i) pads += ids[i] == pad_id;
+    if (pads != n_items) return MIMO_EINVAL;
+    for (int64_t k = 0; k < n_items; ++k) {
+        if (counts[k] < 0 || counts[k] > std::numeric_limits<int64_t>::max() / 2 - total) return MIMO_EINVAL;
+        total += counts[k];
+    }
+    const int64_t len = n_ids - n_items + total;
+    if (len > out_capacity) return MIMO_ECAPACITY;
+    int64_t k = 0, o = 0;
+    for (int64_t i = 0; i < n_ids; ++i) {
+        if (ids[i] == pad_id) {
+            std::fill(out + o, out + o + counts[k], pad_id);
+            o += counts[k++];
+        } else {
+            out[o++] = ids[i];
+        }
+    }
+    *out_len = len;
+    return MIMO_OK;
+}
+
 const char *mimo_status_string(int status) {
     switch (status) {
         case MIMO_OK: return "ok";

@@ -36,7 +36,7 @@ STATUS_NAMES = {
 }
 EXPORTED = ("mimo_params_default", "mimo_smart_resize", "mimo_num_patches", "mimo_plan_batch",
             "mimo_preprocess_batch", "mimo_preprocess_batch_ex", "mimo_preprocess_batch_host",
-            "mimo_preprocess_batch_host_noalloc",
+            "mimo_preprocess_batch_host_noalloc", "mimo_expand_prompt_ids",
             "mimo_status_string", "mimo_version")
 NOALLOC_STAGING_BYTES = 64 << 20
 
@@ -117,6 +117,8 @@ def lib() -> ctypes.CDLL:
             L.mimo_preprocess_batch_host_noalloc.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p,
                                                              _p, _i32, _p, _i64, _p, _p]
             L.mimo_preprocess_batch_host_noalloc.restype = ctypes.c_int
+            L.mimo_expand_prompt_ids.argtypes = [_p, _i64, _i32, _p, _i64, _p, _i64, ctypes.POINTER(_i64)]
+            L.mimo_expand_prompt_ids.restype = ctypes.c_int
             L.mimo_status_string.argtypes = [ctypes.c_int]
             L.mimo_status_string.restype = ctypes.c_char_p
             L.mimo_version.argtypes = []
@@ -189,6 +191,24 @@ def plan_batch(heights: Sequence[int], widths: Sequence[int], params: MimoParams
     _check(lib().mimo_plan_batch(n, h.ctypes.data, w.ctypes.data, ctypes.byref(p), grid.ctypes.data,
                                  offs.ctypes.data), "plan_batch")
     return grid, offs
+
+
+def media_tokens(height: int, width: int, params: MimoParams | None = None) -> int:
+    """Vision tokens of one image: patches after smart_resize over the merge_size**2 reduction."""
+    p = params if params is not None else make_params()
+    return get_number_of_image_patches(height, width, p) // (p.merge_size * p.merge_size)
+
+
+def expand_prompt_ids(ids, pad_id: int, counts) -> np.ndarray:
+    """Replaces the k-th ``pad_id`` in ``ids`` by ``counts[k]`` copies (int32 result)."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    counts = np.ascontiguousarray(counts, dtype=np.int64)
+    cap = int(ids.size + max(int(counts.sum()) if counts.size else 0, 0))
+    out = np.empty(max(cap, 1), np.int32)
+    n = _i64()
+    _check(lib().mimo_expand_prompt_ids(ids.ctypes.data, ids.size, pad_id, counts.ctypes.data, counts.size,
+                                        out.ctypes.data, cap, ctypes.byref(n)), "expand_prompt_ids")
+    return out[:n.value]
 
 
 # ----------------------------------------------------------------- packing
