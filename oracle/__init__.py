@@ -82,6 +82,15 @@ def lib():
             L.oracle_window_index.restype = None
             L.oracle_expand_prompt_ids.argtypes = [_p, _i64, _i32, _p, _i64, _p, _i64]
             L.oracle_expand_prompt_ids.restype = _i64
+            L.oracle_video_max_pixels.argtypes = [_i64, _i64, _i32, _i64, _i64]
+            L.oracle_video_max_pixels.restype = _i64
+            L.oracle_smart_nframes.argtypes = [_i64, ctypes.c_double, ctypes.c_double, _i64, _i64, ctypes.POINTER(_i64)]
+            L.oracle_smart_nframes.restype = ctypes.c_int
+            L.oracle_sample_frames.argtypes = [_i64, _i64, ctypes.c_double, _p, _p]
+            L.oracle_sample_frames.restype = _i64
+            L.oracle_preprocess_video.argtypes = [_p, _i64, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i64, _i64,
+                                                  _i64, _p, _p, _p, _i64, _p]
+            L.oracle_preprocess_video.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -258,6 +267,50 @@ def expand_prompt_ids(ids, pad_id: int, counts) -> np.ndarray:
     if n < 0:
         raise OracleError(EINVAL, "placeholder count does not match the items")
     return out[:n]
+
+
+# ---------------------------------------------------------------- video
+def video_max_pixels(n_sampled: int, total_max: int, temporal: int = 2, min_pixels: int = 8192,
+                     max_pixels: int = 8388608) -> int:
+    return int(lib().oracle_video_max_pixels(n_sampled, total_max, temporal, min_pixels, max_pixels))
+
+
+def smart_nframes(total: int, fps_src: float, fps: float, min_frames: int, max_frames: int) -> int:
+    out = _i64()
+    st = lib().oracle_smart_nframes(total, fps_src, fps, min_frames, max_frames, ctypes.byref(out))
+    if st != OK:
+        raise OracleError(st, "smart_nframes")
+    return out.value
+
+
+def sample_frames(total: int, n: int, fps_src: float):
+    idx = np.empty(max(n, 1), np.int64)
+    ts = np.empty(max(n, 1), np.float32)
+    k = lib().oracle_sample_frames(total, n, fps_src, _ptr(idx), _ptr(ts))
+    if k < 0:
+        raise OracleError(EINVAL, "sample_frames")
+    return idx[:k], ts[:k]
+
+
+def preprocess_video(frames, mean, std, min_pixels=8192, max_pixels=8388608, total_max_pixels=0,
+                     patch=16, temporal=2, merge=2):
+    """Frames [n, H, W, C] uint8 -> (rows fp32, grid_thw (t, h, w))."""
+    frames = np.ascontiguousarray(frames, dtype=np.uint8)
+    n, H, W, C = frames.shape
+    budget = video_max_pixels(n, total_max_pixels, temporal, min_pixels, max_pixels) if total_max_pixels > 0 \
+        else max_pixels
+    Hr, Wr = smart_resize(H, W, patch * merge, min_pixels, budget)
+    gt = (n + 1) // 2
+    rows = gt * (Hr // patch) * (Wr // patch)
+    out = np.empty((rows, 3 * temporal * patch * patch), np.float32)
+    m = np.ascontiguousarray(mean, dtype=np.float64)
+    s = np.ascontiguousarray(std, dtype=np.float64)
+    g = np.zeros(3, np.int64)
+    st = lib().oracle_preprocess_video(_ptr(frames), n, H * W * C, H, W, C, patch, temporal, merge, min_pixels,
+                                       max_pixels, total_max_pixels, _ptr(m), _ptr(s), _ptr(out), rows, _ptr(g))
+    if st != OK:
+        raise OracleError(st, "preprocess_video")
+    return out, tuple(int(v) for v in g)
 
 
 def _flatten_one_level(images):

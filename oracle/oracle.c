@@ -457,3 +457,142 @@ int64_t oracle_expand_prompt_ids(const int32_t *ids, int64_t n_ids, int32_t pad_
     }
     return used == n_items ? len : -1;
 }
+
+/* ------------------------------------------------------------------ video */
+
+/*
+ * [C] video_max_pixels: per-frame pixel ceiling for n sampled frames,
+ * max(min_pixels, min(total_max * T // n, max_pixels)).
+ */
+int64_t oracle_video_max_pixels(int64_t n_sampled, int64_t total_max, int32_t temporal,
+                                int64_t min_pixels, int64_t max_pixels)
+{
+    int64_t share = (total_max * temporal) / n_sampled; /* floor division, all >= 0 */
+    int64_t cap = share < max_pixels ? share : max_pixels;
+    return cap > min_pixels ? cap : min_pixels;
+}
+
+/*
+ * [C] smart_nframes: total / fps_src * fps, clamped to [min_frames,
+ * max_frames] and to total, floored to even. A result of 0 frames is an
+ * error (OR_EINVAL), as is a non-positive count or rate.
+ */
+int oracle_smart_nframes(int64_t total, double fps_src, double fps, int64_t min_frames, int64_t max_frames,
+                         int64_t *out)
+{
+    if (total <= 0 || !(fps_src > 0.0) || !(fps > 0.0) || min_frames < 0 || max_frames < min_frames)
+        return OR_EINVAL;
+    double n = (double)total / fps_src * fps;
+    if (n < (double)min_frames)
+        n = (double)min_frames;
+    if (n > (double)max_frames)
+        n = (double)max_frames;
+    if (n > (double)total)
+        n = (double)total;
+    int64_t even = (int64_t)floor(n / 2.0) * 2;
+    if (even <= 0)
+        return OR_EINVAL;
+    *out = even;
+    return OR_OK;
+}
+
+/*
+ * [C] sample_frames: indices unique(int64(linspace(0, total - 1, n))) and
+ * timestamps float32(idx) / fps_src. linspace: start + k * (stop - start) /
+ * (n - 1) in fp64 with the last sample exactly stop (n = 1 gives [0]); int64
+ * truncates; unique keeps one of each value in increasing order. Returns the
+ * number of indices written (<= n), or -1 on bad arguments.
+ */
+int64_t oracle_sample_frames(int64_t total, int64_t n, double fps_src, int64_t *idx, float *ts)
+{
+    if (total <= 0 || n <= 0 || !(fps_src > 0.0))
+        return -1;
+    double stop = (double)(total - 1);
+    double step = n > 1 ? stop / (double)(n - 1) : 0.0;
+    int64_t count = 0;
+    for (int64_t k = 0; k < n; ++k) {
+        double v = (k == n - 1 && n > 1) ? stop : (double)k * step;
+        int64_t i = (int64_t)v;
+        if (count > 0 && idx[count - 1] == i)
+            continue; /* linspace is non-decreasing: duplicates are adjacent */
+        idx[count] = i;
+        ts[count] = (float)i / (float)fps_src;
+        ++count;
+    }
+    return count;
+}
+
+/*
+ * [C] prepare_video_frames, pixel part: frames (HWC uint8, all H x W x C, at
+ * stride `frame_stride` bytes) -> per-frame budget video_max_pixels(n, ...),
+ * one smart_resize for all frames, an odd count padded by repeating the last
+ * frame, each frame through _to_rgb, _load, resize and standardisation, and
+ * consecutive frames paired as temporal patches: row (t, block row, block
+ * col, mh, mw), column (c, tt, py, px) taking frame 2t + tt.
+ * total_max <= 0 means no budget (max_pixels applies as it is).
+ */
+int oracle_preprocess_video(const uint8_t *frames, int64_t n, int64_t frame_stride, int64_t H, int64_t W,
+                            int32_t C, int32_t patch, int32_t temporal, int32_t merge,
+                            int64_t min_px, int64_t max_px, int64_t total_max,
+                            const double mean[3], const double stdv[3],
+                            float *out, int64_t out_rows_capacity, int64_t grid_thw[3])
+{
+    if (n <= 0 || H <= 0 || W <= 0 || (C != 3 && C != 4) || temporal != 2)
+        return OR_EINVAL;
+    const int64_t budget = total_max > 0 ? oracle_video_max_pixels(n, total_max, temporal, min_px, max_px) : max_px;
+    int64_t Hr, Wr;
+    int st = oracle_smart_resize(H, W, (int64_t)patch * merge, min_px, budget, &Hr, &Wr);
+    if (st != OR_OK)
+        return st;
+    const int64_t n_pad = n + (n & 1);
+    const int64_t gt = n_pad / 2, gh = Hr / patch, gw = Wr / patch;
+    if (gt * gh * gw > out_rows_capacity)
+        return OR_ECAPACITY;
+
+    uint8_t *rgb = (uint8_t *)malloc((size_t)(H * W * 3));
+    double *planes = (double *)malloc(sizeof(double) * (size_t)(3 * H * W));
+    double *resized = (double *)malloc(sizeof(double) * (size_t)(n * 3 * Hr * Wr));
+    if (!rgb || !planes || !resized) {
+        free(rgb);
+        free(planes);
+        free(resized);
+        return OR_ENOMEM;
+    }
+    for (int64_t f = 0; f < n; ++f) {
+        double *r = resized + f * 3 * Hr * Wr;
+        oracle_to_rgb(frames + f * frame_stride, H, W, C, rgb);
+        oracle_load_planes(rgb, H, W, planes);
+        for (int k = 0; k < 3; ++k)
+            oracle_resize_plane(planes + k * H * W, H, W, r + k * Hr * Wr, Hr, Wr);
+        oracle_normalize_planes(r, Hr * Wr, mean, stdv);
+    }
+    const int64_t p = patch, T = temporal, m = merge, cols = 3 * T * p * p;
+    int64_t row = 0;
+    for (int64_t t = 0; t < gt; ++t)
+        for (int64_t bh = 0; bh < gh / m; ++bh)
+            for (int64_t bw = 0; bw < gw / m; ++bw)
+                for (int64_t mh = 0; mh < m; ++mh)
+                    for (int64_t mw = 0; mw < m; ++mw, ++row) {
+                        int64_t col = 0;
+                        for (int64_t c = 0; c < 3; ++c)
+                            for (int64_t tt = 0; tt < T; ++tt) {
+                                int64_t f = t * T + tt;
+                                if (f > n - 1)
+                                    f = n - 1; /* even padding: repeat the last frame */
+                                const double *pl = resized + f * 3 * Hr * Wr + c * Hr * Wr;
+                                for (int64_t py = 0; py < p; ++py)
+                                    for (int64_t px = 0; px < p; ++px, ++col) {
+                                        int64_t y = (bh * m + mh) * p + py;
+                                        int64_t x = (bw * m + mw) * p + px;
+                                        out[row * cols + col] = (float)pl[y * Wr + x];
+                                    }
+                            }
+                    }
+    grid_thw[0] = gt;
+    grid_thw[1] = gh;
+    grid_thw[2] = gw;
+    free(rgb);
+    free(planes);
+    free(resized);
+    return OR_OK;
+}
