@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c5", choices=["c2", "c3", "c4", "c5"])
+    ap.add_argument("--workload", default="c5", choices=["c2", "c3", "c4", "c5", "v1"])
     ap.add_argument("--dtype", default=None, choices=["f32", "bf16"])
     ap.add_argument("--images", type=int, default=None, help="override the workload's image count")
     ap.add_argument("--order", default="merge", choices=["merge", "column"], help="row order of the output")
@@ -209,6 +209,64 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_video(args, rank, world, local_rank):
+    """Frames/s of the video path (one clip per rank, frames resident in HBM)."""
+    import numpy as np
+    import torch
+
+    import workloads
+    from vision_lm_image_b200 import mimo
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.video_workload(args.workload, seed_offset=7919 * rank, n_frames=args.images)
+    frames = w["frames"]
+    n, H, W, C = frames.shape
+    out_dtype = args.dtype or w["dtype"]
+    tdtype = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+    params = mimo.make_params(w["mean"], w["std"])
+    stride = (H * W * C + 15) // 16 * 16
+    d_frames = torch.zeros(n * stride, dtype=torch.uint8, device=dev)
+    d_frames.view(n, stride)[:, :H * W * C].copy_(torch.from_numpy(frames.reshape(n, -1)))
+    grid, rows = mimo.plan_video(n, H, W, w["total_max_pixels"], params)
+    out = torch.empty((rows, 1536), dtype=tdtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mimo.preprocess_video_raw(params, d_frames, n, stride, H, W, C, out, w["total_max_pixels"],
+                                  order=args.order, stream=stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        e0.record(stream)
+        for _ in range(K):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    read = n * H * W * C
+    written = rows * 1536 * (2 if out_dtype == "bf16" else 4)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = (read + written) / (ms / K * 1e-3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC + " (video frames)", "value": world * n * K / (ms * 1e-3), "unit": "frames/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "description": w["description"], "frames": int(n),
+                       "grid_thw": [int(v) for v in grid], "out_dtype": out_dtype, "row_order": args.order,
+                       "l2": "inputs and outputs larger than L2 (no flush)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": peak_kind, "traffic": None, "algorithmic_bytes_per_launch": read + written,
+                         "kernel": "preprocess_kernel", "avg_launch_ms": ms / K},
+            "gpu_launches": K, "clocks": clocks.summary(), "e2e": None, "cpu_baseline": None,
+        }), flush=True)
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -347,6 +405,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.workload.startswith("v"):
+        run_video(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

@@ -262,6 +262,49 @@ int mimo_expand_prompt_ids(const int32_t *ids, int64_t n_ids, int32_t pad_id,
                            const int64_t *counts, int64_t n_items,
                            int32_t *out, int64_t out_capacity, int64_t *out_len);
 
+/*
+ * Video frames (cortiq page: prepare_video_frames, video_max_pixels,
+ * smart_nframes, sample_frames). Decoding and frame selection from a file
+ * stay with the caller; these take frames already decoded to HWC uint8.
+ *
+ * mimo_video_max_pixels: per-frame pixel ceiling for n sampled frames,
+ *   max(min_pixels, min(total_max_pixels * temporal_patch_size // n,
+ *   max_pixels)); total_max_pixels = 0 means no overall budget (max_pixels).
+ * mimo_smart_nframes: total / fps_src * fps, clamped to [min_frames,
+ *   max_frames] and to total, floored to even; MIMO_EINVAL if that is 0.
+ * mimo_sample_frames: idx = unique(int64(linspace(0, total - 1, n))) and
+ *   ts = float32(idx) / fps_src; idx and ts hold n entries, *count gets the
+ *   number of distinct indices written.
+ * All three are host only.
+ */
+int mimo_video_max_pixels(int64_t n_sampled, int64_t total_max_pixels, const mimo_params *p, int64_t *out);
+int mimo_smart_nframes(int64_t total, double fps_src, double fps, int64_t min_frames, int64_t max_frames,
+                       int64_t *out);
+int mimo_sample_frames(int64_t total, int64_t n, double fps_src, int64_t *idx, float *ts, int64_t *count);
+
+/*
+ * Plan of one video of n_frames frames of height x width: one smart_resize
+ * under the per-frame budget for all frames, an odd count padded with its
+ * last frame, grid_thw = (ceil(n/2), H'/16, W'/16), *rows = the product.
+ * Host only.
+ */
+int mimo_plan_video(int32_t n_frames, int32_t height, int32_t width, int64_t total_max_pixels,
+                    const mimo_params *p, int64_t *grid_thw, int64_t *rows);
+
+/*
+ * The pixel path for one video on the GPU. Frame f is at d_frames + f *
+ * frame_stride (device, HWC uint8, all frames height x width x channels;
+ * frame_stride a multiple of 16 and >= one frame's bytes; src_bytes covers
+ * all frames, else MIMO_ERANGE). Consecutive frames pair up as temporal
+ * patches: row (t, block row, block col, mh, mw), column (c, tt, py, px) takes
+ * frame 2t + tt, the last frame standing in for a missing one. `out` as in
+ * mimo_preprocess_batch_ex (the tables use the temporal patch t too: merge
+ * units are listed per t). Asynchronous on `stream`.
+ */
+int mimo_preprocess_video(const mimo_params *p, int32_t n_frames, const uint8_t *d_frames, size_t src_bytes,
+                          int64_t frame_stride, int32_t height, int32_t width, int32_t channels,
+                          int64_t total_max_pixels, const mimo_outputs *out, void *stream);
+
 /* Static description of a status code. */
 const char *mimo_status_string(int status);
 

@@ -182,3 +182,45 @@ def test_expand_prompt_ids_errors():
     st = mimo.lib().mimo_expand_prompt_ids(ids.ctypes.data, 1, 7, counts.ctypes.data, 1, out.ctypes.data, 3,
                                            ctypes.byref(n))
     assert st == 7
+
+
+def test_video_host_formulas_match_oracle():
+    rng = np.random.Generator(np.random.PCG64(43))
+    p = mimo.make_params()
+    for _ in range(300):
+        n = int(rng.integers(1, 2000))
+        total_max = int(rng.integers(1, 10**9))
+        assert mimo.video_max_pixels(n, total_max, p) == oracle.video_max_pixels(n, total_max, 2, 8192, 8388608)
+        total = int(rng.integers(1, 50000))
+        fps_src = float(rng.uniform(1, 120))
+        fps = float(rng.uniform(0.1, 8))
+        mn = int(rng.integers(0, 8))
+        mx = mn + int(rng.integers(0, 1000))
+        try:
+            want = oracle.smart_nframes(total, fps_src, fps, mn, mx)
+        except oracle.OracleError:
+            with pytest.raises(mimo.MimoError):
+                mimo.smart_nframes(total, fps_src, fps, mn, mx)
+            continue
+        assert mimo.smart_nframes(total, fps_src, fps, mn, mx) == want
+        k = int(rng.integers(1, 800))
+        i1, t1 = mimo.sample_frames(total, k, fps_src)
+        i2, t2 = oracle.sample_frames(total, k, fps_src)
+        assert np.array_equal(i1, i2) and np.array_equal(t1, t2)
+    assert mimo.video_max_pixels(7, 0, p) == 8388608  # no overall budget
+
+
+def test_plan_video_matches_oracle_geometry():
+    rng = np.random.Generator(np.random.PCG64(44))
+    for _ in range(300):
+        n = int(rng.integers(1, 64))
+        h, w = (int(v) for v in rng.integers(1, 3000, size=2))
+        total_max = int(rng.choice([0, int(rng.integers(100_000, 10**8))]))
+        budget = oracle.video_max_pixels(n, total_max, 2, 8192, 8388608) if total_max else 8388608
+        if oracle.smart_resize_status(h, w, 32, 8192, budget) != oracle.OK:
+            with pytest.raises(mimo.MimoError):
+                mimo.plan_video(n, h, w, total_max)
+            continue
+        hr, wr = oracle.smart_resize(h, w, 32, 8192, budget)
+        g, rows = mimo.plan_video(n, h, w, total_max)
+        assert tuple(g) == ((n + 1) // 2, hr // 16, wr // 16) and rows == g[0] * g[1] * g[2]

@@ -281,3 +281,48 @@ def test_column_order_is_a_row_gather_full_c5():
     b, _, _ = mimo.preprocess(w["images"], w["mean"], w["std"], order="column")
     torch.cuda.synchronize()
     assert torch.equal(b, a[perm.long()])
+
+
+# ---------------------------------------------------------------- video frames
+@pytest.mark.parametrize("n,shape,c", [(2, (48, 80), 3), (5, (31, 200), 4), (8, (120, 90), 3), (1, (64, 64), 4)])
+def test_video_matches_oracle(n, shape, c):
+    rng = workloads.rng_for(500 + n)
+    frames = np.stack([workloads.uniform_image(rng, shape[0], shape[1], 3) if c == 3
+                       else workloads.rgba_image(rng, shape[0], shape[1]) for _ in range(n)])
+    mean, std = workloads.IMAGENET_MEAN, workloads.IMAGENET_STD
+    ref, g = oracle.preprocess_video(frames, mean, std)
+    for order in ("merge", "column"):
+        pv, grid, perm, pos, win = mimo.preprocess_video(frames, mean, std, column_perm=True, order=order,
+                                                         positions=True, window_index=True)
+        torch.cuda.synchronize()
+        assert tuple(grid[0].tolist()) == g
+        gt, gh, gw = g
+        rperm = np.concatenate([oracle.column_permutation(gh, gw, 2, 0, gt)])
+        assert np.array_equal(perm.cpu().numpy(), rperm)
+        assert np.array_equal(win.cpu().numpy(), oracle.window_index(gh, gw, 2, 0, gt))
+        assert np.array_equal(pos.cpu().numpy(), oracle.rotary_positions(gh, gw, 2, order == "column", gt))
+        want = ref if order == "merge" else ref[rperm]
+        assert_fp32_close(pv.cpu().numpy(), want, f"video {order}")
+
+
+def test_video_budget_and_bf16_full_hd():
+    rng = workloads.rng_for(600)
+    frames = np.stack([workloads.uniform_image(rng, 1080, 1920, 3) for _ in range(6)])
+    mean, std = workloads.IMAGENET_MEAN, workloads.IMAGENET_STD
+    total_max = 6 * 600_000
+    ref, g = oracle.preprocess_video(frames, mean, std, total_max_pixels=total_max)
+    pv, grid, _ = mimo.preprocess_video(frames, mean, std, total_max_pixels=total_max)
+    torch.cuda.synchronize()
+    assert tuple(grid[0].tolist()) == g
+    assert_fp32_close(pv.cpu().numpy(), ref, "video fp32")
+    pvb, _, _ = mimo.preprocess_video(frames, mean, std, total_max_pixels=total_max, dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert_bf16_close(pvb, ref, "video bf16")
+
+
+def test_video_of_equal_frames_equals_the_image_path():
+    img = workloads.random_small_batch(601, 1, max_side=300)[0]
+    a, _, _ = gpu_run([img], workloads.CLIP_MEAN, workloads.CLIP_STD)
+    b, g, _ = mimo.preprocess_video(np.stack([img, img]), workloads.CLIP_MEAN, workloads.CLIP_STD)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)

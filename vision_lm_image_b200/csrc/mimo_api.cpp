@@ -251,8 +251,9 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
             d.W = widths[i];
             d.Hr = static_cast<int32_t>(ip.Hr);
             d.Wr = static_cast<int32_t>(ip.Wr);
-            d.C = channels[i];
-            d.flags = ip.flags;
+            d.flags = ip.flags | (channels[i] << mimo::kChannelShift);
+            d.frame_stride = 0;
+            d.frames = 1;
             // staging copies are 16-byte chunks that may run up to 15 bytes past
             // the image; they read nothing past the end of the caller's buffer
             d.limit = static_cast<int64_t>(src_bytes) - src_offsets[i];
@@ -576,5 +577,150 @@ const char *mimo_status_string(int status) {
 }
 
 int mimo_version(void) { return 10000; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- video
+namespace {
+
+int64_t video_budget(int64_t n, int64_t total_max, const mimo_params *p) {
+    if (total_max <= 0) return p->max_pixels;
+    const int64_t share = (total_max * p->temporal_patch_size) / n;
+    return std::max<int64_t>(p->min_pixels, std::min<int64_t>(share, p->max_pixels));
+}
+
+struct VideoPlan {
+    ImagePlan ip;
+    int64_t gt = 0, rows = 0;
+};
+
+int plan_video(int32_t n_frames, int32_t height, int32_t width, int64_t total_max, const mimo_params *p,
+               VideoPlan *vp) {
+    int st = check_params(p);
+    if (st != MIMO_OK) return st;
+    if (n_frames <= 0 || height <= 0 || width <= 0) return MIMO_EINVAL;
+    if (total_max > std::numeric_limits<int64_t>::max() / 4) return MIMO_EOVERFLOW;
+    mimo_params q = *p;
+    q.max_pixels = video_budget(n_frames, total_max, p);
+    st = plan_image(height, width, &q, &vp->ip);
+    if (st != MIMO_OK) return st;
+    vp->gt = (static_cast<int64_t>(n_frames) + 1) / 2;  // an odd count repeats its last frame
+    if (vp->ip.blocks * vp->gt * 2 > INT32_MAX) return MIMO_EOVERFLOW;
+    vp->rows = vp->gt * vp->ip.rows;
+    return MIMO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mimo_video_max_pixels(int64_t n_sampled, int64_t total_max_pixels, const mimo_params *p, int64_t *out) {
+    if (!p || !out || n_sampled <= 0 || total_max_pixels < 0) return MIMO_EINVAL;
+    if (total_max_pixels > std::numeric_limits<int64_t>::max() / 4) return MIMO_EOVERFLOW;
+    *out = video_budget(n_sampled, total_max_pixels, p);
+    return MIMO_OK;
+}
+
+int mimo_smart_nframes(int64_t total, double fps_src, double fps, int64_t min_frames, int64_t max_frames,
+                       int64_t *out) {
+    if (!out || total <= 0 || !(fps_src > 0.0) || !(fps > 0.0) || min_frames < 0 || max_frames < min_frames)
+        return MIMO_EINVAL;
+    const double n = std::min(std::min(std::max(static_cast<double>(total) / fps_src * fps,
+                                                static_cast<double>(min_frames)),
+                                       static_cast<double>(max_frames)),
+                              static_cast<double>(total));
+    const int64_t even = 2 * static_cast<int64_t>(std::floor(n * 0.5));
+    if (even <= 0) return MIMO_EINVAL;
+    *out = even;
+    return MIMO_OK;
+}
+
+int mimo_sample_frames(int64_t total, int64_t n, double fps_src, int64_t *idx, float *ts, int64_t *count) {
+    if (total <= 0 || n <= 0 || !(fps_src > 0.0) || !idx || !ts || !count) return MIMO_EINVAL;
+    const double last = static_cast<double>(total - 1);
+    const double step = n > 1 ? last / static_cast<double>(n - 1) : 0.0;
+    const float rate = static_cast<float>(fps_src);
+    int64_t k = 0;
+    for (int64_t j = 0; j < n; ++j) {
+        const int64_t i = (n > 1 && j == n - 1) ? total - 1 : static_cast<int64_t>(static_cast<double>(j) * step);
+        if (k == 0 || idx[k - 1] != i) {
+            idx[k] = i;
+            ts[k] = static_cast<float>(i) / rate;
+            ++k;
+        }
+    }
+    *count = k;
+    return MIMO_OK;
+}
+
+int mimo_plan_video(int32_t n_frames, int32_t height, int32_t width, int64_t total_max_pixels,
+                    const mimo_params *p, int64_t *grid_thw, int64_t *rows) {
+    if (!grid_thw || !rows) return MIMO_EINVAL;
+    VideoPlan vp;
+    const int st = plan_video(n_frames, height, width, total_max_pixels, p, &vp);
+    if (st != MIMO_OK) return st;
+    grid_thw[0] = vp.gt;
+    grid_thw[1] = vp.ip.Hr / 16;
+    grid_thw[2] = vp.ip.Wr / 16;
+    *rows = vp.rows;
+    return MIMO_OK;
+}
+
+int mimo_preprocess_video(const mimo_params *p, int32_t n_frames, const uint8_t *d_frames, size_t src_bytes,
+                          int64_t frame_stride, int32_t height, int32_t width, int32_t channels,
+                          int64_t total_max_pixels, const mimo_outputs *out, void *stream) {
+    if (!out || !d_frames) return MIMO_EINVAL;
+    if (out->row_order != MIMO_ORDER_MERGE && out->row_order != MIMO_ORDER_COLUMN) return MIMO_EINVAL;
+    if (out->out_dtype != MIMO_F32 && out->out_dtype != MIMO_BF16) return MIMO_EINVAL;
+    if (channels != 3 && channels != 4) return MIMO_ECHANNELS;
+    VideoPlan vp;
+    int st = plan_video(n_frames, height, width, total_max_pixels, p, &vp);
+    if (st != MIMO_OK) return st;
+    const uint64_t frame_bytes = static_cast<uint64_t>(height) * static_cast<uint64_t>(width) * channels;
+    if (frame_stride < 0 || static_cast<uint64_t>(frame_stride) < frame_bytes) return MIMO_EINVAL;
+    if ((frame_stride & 15) != 0 || !aligned16(d_frames) || !aligned16(out->d_out)) return MIMO_EALIGN;
+    const uint64_t need = static_cast<uint64_t>(n_frames - 1) * static_cast<uint64_t>(frame_stride) + frame_bytes;
+    if (need > src_bytes) return MIMO_ERANGE;
+    if (vp.rows > out->out_rows_capacity) return MIMO_ECAPACITY;
+    if (!out->d_out) return MIMO_EINVAL;
+    for (const void *t : {static_cast<const void *>(out->d_column_perm), static_cast<const void *>(out->d_positions),
+                          static_cast<const void *>(out->d_window_index)}) {
+        if (!t) continue;
+        if (!aligned16(t)) return MIMO_EALIGN;
+        if (vp.rows > INT32_MAX) return MIMO_EOVERFLOW;
+    }
+
+    static thread_local mimo::LaunchParams lp;
+    std::memset(&lp, 0, sizeof(lp));
+    lp.src = d_frames;
+    lp.out = out->d_out;
+    lp.perm = out->d_column_perm;
+    lp.pos = out->d_positions;
+    lp.win = out->d_window_index;
+    lp.order = out->row_order;
+    fold_normalisation(p, &lp);
+    mimo::ImageDesc &d = lp.img[0];
+    d.src_off = 0;
+    d.row0 = 0;
+    d.limit = static_cast<int64_t>(src_bytes);
+    d.frame_stride = frame_stride;
+    d.H = height;
+    d.W = width;
+    d.Hr = static_cast<int32_t>(vp.ip.Hr);
+    d.Wr = static_cast<int32_t>(vp.ip.Wr);
+    d.flags = vp.ip.flags | mimo::kVideo | (channels << mimo::kChannelShift);
+    d.frames = n_frames;
+    const int64_t blocks = vp.ip.blocks * vp.gt * 2;  // (t, block, tt) halves
+    lp.block_start[0] = 0;
+    lp.block_start[1] = static_cast<int32_t>(blocks);
+    lp.n = 1;
+    lp.tile_rows = vp.ip.tile_rows;
+    lp.tile_stride = (std::max(vp.ip.tile_cols, mimo::kBlock) + 3) & ~3;
+    const size_t tile_floats = 3u * static_cast<size_t>(lp.tile_rows) * static_cast<size_t>(lp.tile_stride);
+    lp.raw_stride = ((32 + 4 * vp.ip.tile_cols) + 15) & ~15;
+    const size_t raw_floats = static_cast<size_t>(lp.tile_rows) * static_cast<size_t>(lp.raw_stride) / 4u;
+    lp.raw = static_cast<int32_t>(tile_floats);
+    return mimo::launch_preprocess(lp, blocks, out->out_dtype, sizeof(float) * (tile_floats + raw_floats), stream);
+}
 
 }  // extern "C"

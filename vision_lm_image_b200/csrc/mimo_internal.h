@@ -28,18 +28,24 @@ constexpr int kMaxImagesPerLaunch = 512;
 //  - identity: the axis is not resized (in == out), every weight is 0 and
 //    only the first tap of each output is staged (32 entries);
 //  - otherwise the span from the first to the last tap is staged whole.
-enum : int32_t { kGatherRows = 1, kGatherCols = 2, kIdentityRows = 4, kIdentityCols = 8 };
+enum : int32_t { kGatherRows = 1, kGatherCols = 2, kIdentityRows = 4, kIdentityCols = 8, kVideo = 16 };
+constexpr int kChannelShift = 8;  // channels (3 or 4) live in bits 8..15 of the flags
 
+// One image, or one video whose consecutive frames pair up as temporal
+// patches. A video's blocks are (t, block row, block col, tt) halves, tt
+// innermost: each half stages frame min(2t + tt, frames - 1) and writes the
+// temporal slot tt of its merge unit's rows.
 struct ImageDesc {
-    int64_t src_off;   // byte offset of the image in the packed source buffer
-    int64_t row0;      // first output row of the image in the batch
-    int64_t limit;     // bytes of the caller's source buffer from src_off on
-    int32_t H, W;      // source size
-    int32_t Hr, Wr;    // resized size, multiples of 32
-    int32_t C;         // 3 or 4
-    int32_t flags;     // kGather* | kIdentity*
+    int64_t src_off;       // byte offset of the (first) frame in the source buffer
+    int64_t row0;          // first output row of the item in the batch
+    int64_t limit;         // bytes of the caller's source buffer from src_off on
+    int64_t frame_stride;  // bytes from one frame to the next (videos)
+    int32_t H, W;          // source size
+    int32_t Hr, Wr;        // resized size, multiples of 32
+    int32_t flags;         // kGather* | kIdentity* | kVideo | channels << kChannelShift
+    int32_t frames;        // source frames (1 for an image)
 };
-static_assert(sizeof(ImageDesc) == 48, "descriptor layout");
+static_assert(sizeof(ImageDesc) == 56, "descriptor layout");
 
 // Everything one launch needs travels by value as the kernel's parameter
 // block (__grid_constant__), so a launch needs no device-side table and no
@@ -58,7 +64,7 @@ struct LaunchParams {
     int32_t tile_stride; // row stride (floats, multiple of 4) of the tile
     int32_t raw;         // float offset of the raw staging rows
     int32_t raw_stride;  // bytes per raw staging row (multiple of 16)
-    int32_t block_start[kMaxImagesPerLaunch + 1];  // prefix sum of merge blocks
+    int32_t block_start[kMaxImagesPerLaunch + 1];  // prefix sum of blocks (video blocks are halves)
     ImageDesc img[kMaxImagesPerLaunch];
 };
 static_assert(sizeof(LaunchParams) <= 32764 - 64, "kernel parameter limit");

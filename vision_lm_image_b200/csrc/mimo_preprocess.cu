@@ -85,6 +85,7 @@ struct TapSet {
     int32_t x_first, ncols;  // first source column / staged columns
     int32_t flags, W, C, CQ; // image flags, width, channels, 16-byte chunks per staged row
     int32_t gw2, gh2, bh, bw;
+    int32_t t, tt;            // temporal patch and slot (videos; 0 for images)
     int32_t Q, pad_q;          // staging jobs (4 pixels) per tile row
     uint32_t qmagic, cmagic;  // x / Q and x / CQ as (x * magic) >> 16 for the job counts here
     int64_t src_off;         // image offset in the source buffer
@@ -98,7 +99,7 @@ struct TapSet {
 // output index d in the last block seen along the warp's axis, and the
 // change of both from one block to the next.
 struct AxisCursor {
-    int blk = -2, ii = 0, bh = 0, bw = 0;  // position of the last block handled
+    int blk = -2, ii = 0, t = 0, bh = 0, bw = 0, tt = 0;  // position of the last block handled
     int img = -1, b = -2;
     int64_t q = 0, r = 0;
     int64_t den = 1, step_q = 0, step_r = 0;
@@ -111,50 +112,87 @@ struct AxisCursor {
 __device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, const TapSet &prev, int blk,
                                              AxisCursor &cur, int warp, int lane) {
     // block position: consecutive blocks advance one column (or start the
-    // next block row / image); only the CTA's first block needs a division
-    int ii = cur.ii, bh, bw;
+    // next block row / temporal patch / item), a video first through its
+    // two temporal halves; only the CTA's first block needs divisions
+    int ii = cur.ii, t, bh, bw, tt;
     if (blk == cur.blk + 1) {
         if (ii + 1 < P.n && P.block_start[ii + 1] <= blk) {
             ++ii;
-            bh = 0;
-            bw = 0;
+            t = bh = bw = tt = 0;
         } else {
+            const ImageDesc &Dc = P.img[ii];
+            t = cur.t;
             bh = cur.bh;
-            bw = cur.bw + 1;
-            if (bw == P.img[ii].Wr / kBlock) {
-                bw = 0;
-                ++bh;
+            bw = cur.bw;
+            tt = cur.tt;
+            if ((Dc.flags & kVideo) != 0 && tt == 0) {
+                tt = 1;
+            } else {
+                tt = 0;
+                if (++bw == Dc.Wr / kBlock) {
+                    bw = 0;
+                    if (++bh == Dc.Hr / kBlock) {
+                        bh = 0;
+                        ++t;
+                    }
+                }
             }
         }
     } else {
         ii = find_image(P, blk);
-        const int local = blk - P.block_start[ii];
-        const int g = P.img[ii].Wr / kBlock;
+        const ImageDesc &Dc = P.img[ii];
+        int local = blk - P.block_start[ii];
+        const bool vid = (Dc.flags & kVideo) != 0;
+        tt = vid ? (local & 1) : 0;
+        if (vid) local >>= 1;
+        const int g = Dc.Wr / kBlock;
+        const int units = (Dc.Hr / kBlock) * g;
+        t = local / units;
+        local -= t * units;
         bh = local / g;
         bw = local - bh * g;
     }
     cur.blk = blk;
     cur.ii = ii;
+    cur.t = t;
     cur.bh = bh;
     cur.bw = bw;
+    cur.tt = tt;
     const ImageDesc &D = P.img[ii];
-    const int32_t H = D.H, W = D.W, Hr = D.Hr, Wr = D.Wr, flags = D.flags, C = D.C;
+    const int32_t H = D.H, W = D.W, Hr = D.Hr, Wr = D.Wr, flags = D.flags;
+    const int32_t C = (flags >> kChannelShift) & 0xFF;
     const int gw2 = Wr / kBlock;
     const bool is_col = warp == 1;
     const int64_t in = is_col ? W : H;
     const int64_t out = is_col ? Wr : Hr;
     const int b = is_col ? bw : bh;
 
-    if (!is_col && ii == cur.img && b == cur.b) {
-        // same block row as the previous block: row taps unchanged
-        T.ty[0][lane] = prev.ty[0][lane];
-        T.ty[1][lane] = prev.ty[1][lane];
-        T.ly[lane] = prev.ly[lane];
-        T.srow[lane] = prev.srow[lane];
-        T.srow[lane + 32] = prev.srow[lane + 32];
-        if (lane == 0) {
-            T.y_first = prev.y_first;
-            T.nrows = prev.nrows;
+    if (ii == cur.img && b == cur.b) {
+        // same block row (column) as the previous block: its taps are unchanged
+        if (!is_col) {
+            T.ty[0][lane] = prev.ty[0][lane];
+            T.ty[1][lane] = prev.ty[1][lane];
+            T.ly[lane] = prev.ly[lane];
+            T.srow[lane] = prev.srow[lane];
+            T.srow[lane + 32] = prev.srow[lane + 32];
+            if (lane == 0) {
+                T.y_first = prev.y_first;
+                T.nrows = prev.nrows;
+            }
+        } else {
+            T.tx[0][lane] = prev.tx[0][lane];
+            T.tx[1][lane] = prev.tx[1][lane];
+            T.lx[lane] = prev.lx[lane];
+            T.scol[lane] = prev.scol[lane];
+            T.scol[lane + 32] = prev.scol[lane + 32];
+            if (lane == 0) {
+                T.x_first = prev.x_first;
+                T.ncols = prev.ncols;
+                T.CQ = prev.CQ;
+                T.Q = prev.Q;
+                T.cmagic = prev.cmagic;
+                T.qmagic = prev.qmagic;
+            }
         }
     } else {
         if (ii != cur.img) {
@@ -252,12 +290,17 @@ __device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, c
         T.gh2 = Hr / kBlock;
         T.bh = bh;
         T.bw = bw;
-        T.src_off = D.src_off;
-        T.limit = D.limit;
+        T.t = t;
+        T.tt = tt;
+        // a video half stages frame 2t + tt, the last frame standing in past the end
+        const int64_t f = (flags & kVideo) ? min(2 * t + tt, D.frames - 1) : 0;
+        T.src_off = D.src_off + f * D.frame_stride;
+        T.limit = D.limit - f * D.frame_stride;
         T.row0 = D.row0;
-        // merge order lists units by (block row, block col), column order by (block col, block row)
-        const int64_t unit = P.order ? static_cast<int64_t>(bw) * (Hr / kBlock) + bh
-                                     : static_cast<int64_t>(bh) * gw2 + bw;
+        // merge order lists units by (t, block row, block col), column order by (t, block col, block row)
+        const int gh2 = Hr / kBlock;
+        const int64_t unit = static_cast<int64_t>(t) * gh2 * gw2 +
+                             (P.order ? static_cast<int64_t>(bw) * gh2 + bh : static_cast<int64_t>(bh) * gw2 + bw);
         T.row_base = D.row0 + 4 * unit;
     }
 }
@@ -442,6 +485,9 @@ __device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &
     const float2 ly2 = f2(ly, ly), nly2 = f2(-ly, -ly);
     const int64_t row = T.row_base + (mh * 2 + mw);
     const int col = py * 16 + q * 4;
+    const bool video = (flags & kVideo) != 0;
+    const bool both = !video;
+    const int slot0 = video ? 256 * T.tt : 0;
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
         const float4 A = *reinterpret_cast<const float4 *>(a_row + c * plane);
@@ -454,28 +500,30 @@ __device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &
         const float2 k2 = f2(P.k[c], P.k[c]), b2 = f2(P.b[c], P.b[c]);
         const float2 n01 = fma2(v01, k2, b2);
         const float2 n23 = fma2(v23, k2, b2);
+        // an image fills both temporal slots with its one frame; a video half fills slot tt
         if constexpr (!kBF16) {
-            float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col;
+            float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
             const float4 f4 = make_float4(n01.x, n01.y, n23.x, n23.y);
-            __stcs(reinterpret_cast<float4 *>(o), f4);        // tt = 0
-            __stcs(reinterpret_cast<float4 *>(o + 256), f4);  // tt = 1
+            __stcs(reinterpret_cast<float4 *>(o), f4);
+            if (both) __stcs(reinterpret_cast<float4 *>(o + 256), f4);
         } else {
-            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col;
+            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
             const __nv_bfloat162 lo2 = __floats2bfloat162_rn(n01.x, n01.y);
             const __nv_bfloat162 hi2 = __floats2bfloat162_rn(n23.x, n23.y);
             uint2 u;
             u.x = *reinterpret_cast<const uint32_t *>(&lo2);
             u.y = *reinterpret_cast<const uint32_t *>(&hi2);
             __stcs(reinterpret_cast<uint2 *>(o), u);
-            __stcs(reinterpret_cast<uint2 *>(o + 256), u);
+            if (both) __stcs(reinterpret_cast<uint2 *>(o + 256), u);
         }
     }
 
     // the merge unit's table entries: permutation (thread 0), rotary
     // positions of its 4 emitted rows (thread 1), window index (thread 2)
-    if (tid < 3) {
-        const int64_t src_unit = static_cast<int64_t>(T.bh) * T.gw2 + T.bw;  // merge order
-        const int64_t dst_unit = static_cast<int64_t>(T.bw) * T.gh2 + T.bh;  // column order
+    if (tid < 3 && (!video || T.tt == 0)) {
+        const int64_t t_units = static_cast<int64_t>(T.t) * T.gh2 * T.gw2;
+        const int64_t src_unit = t_units + static_cast<int64_t>(T.bh) * T.gw2 + T.bw;  // merge order
+        const int64_t dst_unit = t_units + static_cast<int64_t>(T.bw) * T.gh2 + T.bh;  // column order
         if (tid == 0 && P.perm != nullptr) {
             const int32_t s0 = static_cast<int32_t>(T.row0 + 4 * src_unit);
             __stcs(reinterpret_cast<int4 *>(P.perm + T.row0 + 4 * dst_unit), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));

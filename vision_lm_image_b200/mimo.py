@@ -36,7 +36,8 @@ STATUS_NAMES = {
 }
 EXPORTED = ("mimo_params_default", "mimo_smart_resize", "mimo_num_patches", "mimo_plan_batch",
             "mimo_preprocess_batch", "mimo_preprocess_batch_ex", "mimo_preprocess_batch_host",
-            "mimo_preprocess_batch_host_noalloc", "mimo_expand_prompt_ids",
+            "mimo_preprocess_batch_host_noalloc", "mimo_expand_prompt_ids", "mimo_video_max_pixels",
+            "mimo_smart_nframes", "mimo_sample_frames", "mimo_plan_video", "mimo_preprocess_video",
             "mimo_status_string", "mimo_version")
 NOALLOC_STAGING_BYTES = 64 << 20
 
@@ -119,6 +120,19 @@ def lib() -> ctypes.CDLL:
             L.mimo_preprocess_batch_host_noalloc.restype = ctypes.c_int
             L.mimo_expand_prompt_ids.argtypes = [_p, _i64, _i32, _p, _i64, _p, _i64, ctypes.POINTER(_i64)]
             L.mimo_expand_prompt_ids.restype = ctypes.c_int
+            L.mimo_video_max_pixels.argtypes = [_i64, _i64, ctypes.POINTER(MimoParams), ctypes.POINTER(_i64)]
+            L.mimo_video_max_pixels.restype = ctypes.c_int
+            L.mimo_smart_nframes.argtypes = [_i64, ctypes.c_double, ctypes.c_double, _i64, _i64,
+                                             ctypes.POINTER(_i64)]
+            L.mimo_smart_nframes.restype = ctypes.c_int
+            L.mimo_sample_frames.argtypes = [_i64, _i64, ctypes.c_double, _p, _p, ctypes.POINTER(_i64)]
+            L.mimo_sample_frames.restype = ctypes.c_int
+            L.mimo_plan_video.argtypes = [_i32, _i32, _i32, _i64, ctypes.POINTER(MimoParams), _p,
+                                          ctypes.POINTER(_i64)]
+            L.mimo_plan_video.restype = ctypes.c_int
+            L.mimo_preprocess_video.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _i64, _i32, _i32, _i32,
+                                                _i64, ctypes.POINTER(MimoOutputs), _p]
+            L.mimo_preprocess_video.restype = ctypes.c_int
             L.mimo_status_string.argtypes = [ctypes.c_int]
             L.mimo_status_string.restype = ctypes.c_char_p
             L.mimo_version.argtypes = []
@@ -353,6 +367,102 @@ def preprocess(images, mean=None, std=None, min_pixels: int | None = None, max_p
     if positions or window_index:
         return out, torch.from_numpy(grid), perm, pos, win
     return out, torch.from_numpy(grid), perm
+
+
+# ----------------------------------------------------------------- video
+def video_max_pixels(n_sampled: int, total_max_pixels: int, params: MimoParams | None = None) -> int:
+    p = params if params is not None else make_params()
+    out = _i64()
+    _check(lib().mimo_video_max_pixels(n_sampled, total_max_pixels, ctypes.byref(p), ctypes.byref(out)))
+    return out.value
+
+
+def smart_nframes(total: int, fps_src: float, fps: float, min_frames: int, max_frames: int) -> int:
+    out = _i64()
+    _check(lib().mimo_smart_nframes(total, fps_src, fps, min_frames, max_frames, ctypes.byref(out)), "smart_nframes")
+    return out.value
+
+
+def sample_frames(total: int, n: int, fps_src: float):
+    """(frame indices int64, timestamps float32 seconds)."""
+    idx = np.empty(max(n, 1), np.int64)
+    ts = np.empty(max(n, 1), np.float32)
+    k = _i64()
+    _check(lib().mimo_sample_frames(total, n, fps_src, idx.ctypes.data, ts.ctypes.data, ctypes.byref(k)),
+           "sample_frames")
+    return idx[:k.value], ts[:k.value]
+
+
+def plan_video(n_frames: int, height: int, width: int, total_max_pixels: int = 0, params: MimoParams | None = None):
+    """(grid_thw int64 [3], rows)."""
+    p = params if params is not None else make_params()
+    g = np.zeros(3, np.int64)
+    rows = _i64()
+    _check(lib().mimo_plan_video(n_frames, height, width, total_max_pixels, ctypes.byref(p), g.ctypes.data,
+                                 ctypes.byref(rows)), "plan_video")
+    return g, rows.value
+
+
+def preprocess_video_raw(params: MimoParams, d_frames, n_frames: int, frame_stride: int, height: int, width: int,
+                         channels: int, out, total_max_pixels: int = 0, perm=None, positions=None, window=None,
+                         order: str = "merge", stream=None) -> None:
+    """Raw ABI call of mimo_preprocess_video on frames already in device memory (uint8 tensor)."""
+    o = MimoOutputs()
+    o.out_dtype = _dtype_code(out.dtype)
+    o.row_order = {"merge": ORDER_MERGE, "column": ORDER_COLUMN}[order]
+    o.d_out = out.data_ptr()
+    o.out_rows_capacity = out.shape[0]
+    o.d_column_perm = perm.data_ptr() if perm is not None else None
+    o.d_positions = positions.data_ptr() if positions is not None else None
+    o.d_window_index = window.data_ptr() if window is not None else None
+    _check(lib().mimo_preprocess_video(ctypes.byref(params), n_frames, ctypes.c_void_p(d_frames.data_ptr()),
+                                       d_frames.numel(), frame_stride, height, width, channels, total_max_pixels,
+                                       ctypes.byref(o), _stream_handle(stream, d_frames.device)), "preprocess_video")
+
+
+def preprocess_video(frames, mean=None, std=None, min_pixels: int | None = None, max_pixels: int | None = None,
+                     total_max_pixels: int = 0, dtype=None, column_perm: bool = False, device="cuda", stream=None,
+                     order: str = "merge", positions: bool = False, window_index: bool = False):
+    """One video (frames [n, H, W, C] uint8, numpy or torch) through the GPU path.
+
+    Returns (pixel_values, video_grid_thw [1, 3], perm | None) and, with
+    ``positions`` / ``window_index``, the two tables as well.
+    """
+    import torch
+
+    dtype = torch.float32 if dtype is None else dtype
+    dev = torch.device(device)
+    if dev.type != "cuda":
+        raise ValueError("the MiMo preprocessing library runs on CUDA devices only")
+    params = make_params(mean, std, min_pixels, max_pixels)
+    t = frames if isinstance(frames, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(frames, dtype=np.uint8))
+    if t.ndim != 4 or t.dtype != torch.uint8:
+        raise ValueError("frames must be a uint8 array [n, H, W, C]")
+    n, H, W, C = (int(v) for v in t.shape)
+    frame_bytes = H * W * C
+    stride = (frame_bytes + ALIGN - 1) // ALIGN * ALIGN
+    buf = torch.zeros(n * stride, dtype=torch.uint8, device=dev)
+    buf.view(n, stride)[:, :frame_bytes].copy_(t.reshape(n, frame_bytes), non_blocking=True)
+    grid, rows = plan_video(n, H, W, total_max_pixels, params)
+    out = torch.empty((rows, ROW_WIDTH), dtype=dtype, device=dev)
+    perm = torch.empty(rows, dtype=torch.int32, device=dev) if column_perm else None
+    pos = torch.empty((rows, 2), dtype=torch.int32, device=dev) if positions else None
+    win = torch.empty(rows // 4, dtype=torch.int32, device=dev) if window_index else None
+    o = MimoOutputs()
+    o.out_dtype = _dtype_code(dtype)
+    o.row_order = {"merge": ORDER_MERGE, "column": ORDER_COLUMN}[order]
+    o.d_out = out.data_ptr()
+    o.out_rows_capacity = rows
+    o.d_column_perm = perm.data_ptr() if perm is not None else None
+    o.d_positions = pos.data_ptr() if pos is not None else None
+    o.d_window_index = win.data_ptr() if win is not None else None
+    _check(lib().mimo_preprocess_video(ctypes.byref(params), n, ctypes.c_void_p(buf.data_ptr()), buf.numel(), stride,
+                                       H, W, C, total_max_pixels, ctypes.byref(o), _stream_handle(stream, dev)),
+           "preprocess_video")
+    g = torch.from_numpy(grid.reshape(1, 3))
+    if positions or window_index:
+        return out, g, perm, pos, win
+    return out, g, perm
 
 
 # ----------------------------------------------------------------- host-to-host path

@@ -19,6 +19,9 @@ Workloads (all drawn with numpy ``Generator(PCG64(seed))``):
         clipped to 0..255; ImageNet statistics.
 ``c5``  256 images 1080x1920, even indices RGB and odd indices RGBA (alpha as in
         c2), uniform 0..255; ImageNet statistics.
+``v1``  one video clip: 64 RGB frames 1080x1920, uniform 0..255, no overall
+        pixel budget (each frame pair becomes one temporal patch); ImageNet
+        statistics.
 """
 from __future__ import annotations
 
@@ -72,6 +75,17 @@ def random_sizes(rng: np.random.Generator, n: int, lo: int = 224, hi: int = 2048
             continue
         sizes.append((h, w))
     return sizes
+
+
+def video_workload(name: str, seed_offset: int = 0, n_frames: int | None = None):
+    """Returns dict(frames=[n, H, W, C] uint8, mean, std, total_max_pixels, description)."""
+    if name != "v1":
+        raise KeyError(name)
+    rng = rng_for(SEED_BASE + 10 + seed_offset)
+    n = 64 if n_frames is None else n_frames
+    frames = rng.integers(0, 256, size=(n, 1080, 1920, 3), dtype=np.uint8)
+    return dict(frames=frames, mean=IMAGENET_MEAN, std=IMAGENET_STD, total_max_pixels=0, dtype="f32",
+                description=f"{n} x RGB 1080x1920 video frames -> {(n + 1) // 2} temporal patches of 1088x1920")
 
 
 def workload(name: str, seed_offset: int = 0, n_images: int | None = None):
