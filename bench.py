@@ -52,7 +52,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c5", choices=["c2", "c3", "c4", "c5", "v1"])
+    ap.add_argument("--workload", default="c5", choices=["c2", "c3", "c4", "c5", "v1", "pe"],
+                    help="pe: the patch embedding GEMM on the bf16 rows of c5 (--images sets the image count)")
+    ap.add_argument("--embed-dim", type=int, default=1280, help="pe: output width of the patch embedding")
     ap.add_argument("--dtype", default=None, choices=["f32", "bf16"])
     ap.add_argument("--images", type=int, default=None, help="override the workload's image count")
     ap.add_argument("--order", default="merge", choices=["merge", "column"], help="row order of the output")
@@ -267,6 +269,89 @@ def run_video(args, rank, world, local_rank):
         }), flush=True)
 
 
+def run_patch_embed(args, rank, world, local_rank):
+    """Tokens/s of the tensor-core patch embedding on the bf16 rows of the c5 batch (rows resident in HBM)."""
+    import numpy as np
+    import torch
+
+    import workloads
+    from vision_lm_image_b200 import mimo
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.workload("c5", seed_offset=7919 * rank, n_images=args.images)
+    rows, _, _ = mimo.preprocess(w["images"], w["mean"], w["std"], dtype=torch.bfloat16, device=dev)
+    M, K, N = rows.shape[0], rows.shape[1], args.embed_dim
+    g = torch.Generator(device="cpu").manual_seed(17 + rank)
+    weight = (torch.randn((N, K), generator=g) * 0.02).to(torch.bfloat16).to(dev)
+    bias = torch.randn(N, generator=g).to(dev)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for _ in range(steps):
+            fn()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        return ev[0].elapsed_time(ev[1]) / steps
+
+    step = lambda: mimo.patch_embed(rows, weight, bias, out=out, error=err, stream=stream, check=False)
+    for _ in range(max(args.warmup, 0)):
+        step()
+    with ClockSampler(local_rank) as clocks:
+        ms = timed(step, args.steps)
+    code = int(err.item())
+    if code:
+        raise SystemExit(f"patch_embed reported pipeline error {code}")
+    # library GEMM on the same operands (cuBLAS through torch), for context
+    out_ref = torch.empty_like(out)
+    lib_step = lambda: torch.addmm(bias.to(torch.bfloat16), rows, weight.t(), out=out_ref)
+    for _ in range(max(args.warmup, 0)):
+        lib_step()
+    lib_ms = timed(lib_step, args.steps)
+    flops = 2.0 * M * N * K
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        peak, peak_sus, kind = float(pk["bf16_tflops"]), float(pk["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        peak, peak_sus, kind = 1590.0, 1400.0, "fallback"
+    achieved = flops / (ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        oracle.build()
+        sample = 256
+        a = rows[:sample].float().cpu().numpy()
+        wt = weight.float().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.patch_embed(a, wt, bias.cpu().numpy())
+        dt = time.perf_counter() - t0
+        cpu = {"value": sample / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"first {sample} of {M} rows, one pass, {dt:.1f} s, single thread"}
+    if rank == 0:
+        print(json.dumps({
+            "metric": "patch-embedding tokens/s (Conv3d 3x2x16x16 -> embed_dim as a bf16 GEMM)",
+            "value": world * M / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "pe", "description": f"bf16 rows of c5 ({M} x {K}) x weight [{N}, {K}] + bias "
+                       f"-> bf16 [{M}, {N}]", "rows": M, "embed_dim": N, "K": K,
+                       "l2": "rows (%.1f GB) and output larger than L2 (no flush)" % (M * K * 2 / 1e9)},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "frac_of_sustained": achieved / peak_sus, "peak_kind": kind,
+                         "traffic": None, "algorithmic_flops_per_launch": flops, "kernel": "patch_embed_kernel",
+                         "avg_launch_ms": ms},
+            "library_gemm": {"impl": "torch.addmm (cuBLAS)", "ms": lib_ms, "tflops": flops / (lib_ms * 1e-3) / 1e12},
+            "gpu_launches": args.steps, "clocks": clocks.summary(), "e2e": None, "cpu_baseline": cpu,
+        }), flush=True)
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -405,6 +490,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.workload == "pe":
+        run_patch_embed(args, rank, world, local_rank)
     elif args.workload.startswith("v"):
         run_video(args, rank, world, local_rank)
     else:

@@ -305,6 +305,27 @@ int mimo_preprocess_video(const mimo_params *p, int32_t n_frames, const uint8_t 
                           int64_t frame_stride, int32_t height, int32_t width, int32_t channels,
                           int64_t total_max_pixels, const mimo_outputs *out, void *stream);
 
+/*
+ * Patch embedding of the vision tower (vision page, MiMoVisionPatchEmbed: the
+ * Conv3d with kernel = stride = (temporal 2, 16, 16) applied to the patch
+ * rows) on the tensor cores:
+ *   out[m, n] = sum_k rows[m, k] * weight[n, k] (+ bias[n]),  k < 1536,
+ * with the weight laid out like the rows, (c, tt, py, px), i.e. the Conv3d
+ * weight [embed_dim, 3, 2, 16, 16] flattened. bf16 inputs, fp32 accumulation.
+ *   d_rows:   device bf16 [rows, 1536] (for example mimo_preprocess_batch with
+ *             MIMO_BF16 output); rows >= 0.
+ *   d_weight: device bf16 [embed_dim, 1536]; embed_dim a positive multiple
+ *             of 256 (1280 for the MiMo-V2 tower).
+ *   d_bias:   device fp32 [embed_dim] or NULL.
+ *   d_out:    device [rows, embed_dim] of out_dtype (MIMO_F32 / MIMO_BF16).
+ *   d_error:  device int32, read after the stream synchronises: 0, or a
+ *             nonzero code if the kernel gave up waiting on its own pipeline
+ *             (its output is then incomplete). The call does not clear it.
+ * All pointers 16-byte aligned (MIMO_EALIGN). Asynchronous on `stream`.
+ */
+int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int32_t embed_dim,
+                     const float *d_bias, int32_t out_dtype, void *d_out, int32_t *d_error, void *stream);
+
 /* Static description of a status code. */
 const char *mimo_status_string(int status);
 

@@ -91,6 +91,8 @@ def lib():
             L.oracle_preprocess_video.argtypes = [_p, _i64, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i64, _i64,
                                                   _i64, _p, _p, _p, _i64, _p]
             L.oracle_preprocess_video.restype = ctypes.c_int
+            L.oracle_patch_embed.argtypes = [_p, _i64, _i64, _p, _i64, _p, _p]
+            L.oracle_patch_embed.restype = None
             _lib = L
     return _lib
 
@@ -311,6 +313,18 @@ def preprocess_video(frames, mean, std, min_pixels=8192, max_pixels=8388608, tot
     if st != OK:
         raise OracleError(st, "preprocess_video")
     return out, tuple(int(v) for v in g)
+
+
+def patch_embed(rows: np.ndarray, weight: np.ndarray, bias=None) -> np.ndarray:
+    """fp64 [M, N] = rows [M, K] @ weight[N, K]^T (+ bias), inputs taken as given (float32 values)."""
+    rows = np.ascontiguousarray(rows, dtype=np.float32)
+    weight = np.ascontiguousarray(weight, dtype=np.float32)
+    M, K = rows.shape
+    N = weight.shape[0]
+    out = np.empty((M, N), np.float64)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64)
+    lib().oracle_patch_embed(_ptr(rows), M, K, _ptr(weight), N, _ptr(b) if b is not None else None, _ptr(out))
+    return out
 
 
 def _flatten_one_level(images):

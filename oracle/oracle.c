@@ -596,3 +596,21 @@ int oracle_preprocess_video(const uint8_t *frames, int64_t n, int64_t frame_stri
     free(resized);
     return OR_OK;
 }
+
+/*
+ * [V] MiMoVisionPatchEmbed: the Conv3d with kernel = stride = (T, p, p) over
+ * the frames is, for each patch row, the dot product of the row's 3*T*p*p
+ * values (c, tt, py, px) with each output channel's weight of the same layout:
+ * out[m][n] = sum_k rows[m][k] * w[n][k] (+ bias[n]), in fp64.
+ */
+void oracle_patch_embed(const float *rows, int64_t M, int64_t K, const float *w, int64_t N,
+                        const double *bias, double *out)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = bias ? bias[n] : 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += (double)rows[m * K + k] * (double)w[n * K + k];
+            out[m * N + n] = acc;
+        }
+}

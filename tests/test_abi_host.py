@@ -224,3 +224,20 @@ def test_plan_video_matches_oracle_geometry():
         hr, wr = oracle.smart_resize(h, w, 32, 8192, budget)
         g, rows = mimo.plan_video(n, h, w, total_max)
         assert tuple(g) == ((n + 1) // 2, hr // 16, wr // 16) and rows == g[0] * g[1] * g[2]
+
+
+@no_gpu_only
+def test_patch_embed_validation_statuses():
+    L = mimo.lib()
+    P = ctypes.c_void_p
+
+    def call(rows=128, w=FAKE, n=256, bias=0, dt=0, out=FAKE, err=FAKE, a=FAKE):
+        return L.mimo_patch_embed(P(a), rows, P(w), n, P(bias), dt, P(out), P(err), None)
+
+    assert call(rows=0) == 0
+    assert call(rows=-1) == 1
+    assert call(n=100) == 1 and call(n=0) == 1
+    assert call(dt=7) == 1
+    assert call(a=0) == 1 and call(err=0) == 1
+    assert call(a=FAKE + 8) == 6 and call(out=FAKE + 2) == 6 and call(bias=FAKE + 4) == 6 and call(err=FAKE + 2) == 6
+    assert call(rows=1 << 31) == 8

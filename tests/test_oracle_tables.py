@@ -91,3 +91,31 @@ def test_expand_prompt_ids_rejects_a_count_mismatch():
         oracle.expand_prompt_ids([1, 7, 7], 7, [3])
     with pytest.raises(oracle.OracleError):
         oracle.expand_prompt_ids([1, 7], 7, [3, 4])
+
+
+
+def test_patch_embed_is_the_conv3d_of_the_pages():
+    # MiMoVisionPatchEmbed is a Conv3d with kernel = stride = (2, 16, 16): the oracle's row GEMM with the
+    # weight flattened (c, tt, py, px) must equal torch's conv3d over the two duplicated frames
+    import torch.nn.functional as F
+    rng = np.random.Generator(np.random.PCG64(5))
+    img = workloads.random_small_batch(83, 1, max_side=120)[0]
+    rows, g = oracle.preprocess_image(img, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    N = 48
+    w = rng.standard_normal((N, 3, 2, 16, 16)).astype(np.float32)
+    b = rng.standard_normal(N)
+    out = oracle.patch_embed(rows, w.reshape(N, -1), b)
+    gh, gw = g[1], g[2]
+    # rebuild the normalised frames from the rows (merge order -> planes), then convolve
+    x = torch.from_numpy(rows.astype(np.float64)).reshape(gh // 2, gw // 2, 2, 2, 3, 2, 16, 16)
+    x = x.permute(4, 5, 0, 2, 6, 1, 3, 7).reshape(1, 3, 2, gh * 16, gw * 16)  # (c, tt, y, x)
+    conv = F.conv3d(x, torch.from_numpy(w.astype(np.float64)), torch.from_numpy(b), stride=(2, 16, 16))
+    ref = conv[0, :, 0].reshape(N, gh // 2, 2, gw // 2, 2).permute(1, 3, 2, 4, 0).reshape(-1, N).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-9)
+
+
+def test_patch_embed_hand_worked():
+    rows = np.array([[1.0, 2.0, 3.0], [0.5, -1.0, 4.0]], np.float32)
+    w = np.array([[1.0, 0.0, -1.0], [2.0, 1.0, 0.5]], np.float32)
+    out = oracle.patch_embed(rows, w, [10.0, -1.0])
+    assert out.tolist() == [[1 - 3 + 10, 2 + 2 + 1.5 - 1], [0.5 - 4 + 10, 1 - 1 + 2 - 1]]

@@ -326,3 +326,50 @@ def test_video_of_equal_frames_equals_the_image_path():
     b, g, _ = mimo.preprocess_video(np.stack([img, img]), workloads.CLIP_MEAN, workloads.CLIP_STD)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- patch embedding on the tensor cores
+def _embed_ref(rows_bf16: torch.Tensor, w_bf16: torch.Tensor, bias):
+    a = rows_bf16.float().cpu().numpy()
+    w = w_bf16.float().cpu().numpy()
+    ref = oracle.patch_embed(a, w, None if bias is None else bias.cpu().numpy())
+    scale = np.abs(a.astype(np.float64)) @ np.abs(w.astype(np.float64)).T  # sum_k |a_k w_k|
+    return ref, scale
+
+
+def _assert_embed_close(got: torch.Tensor, ref, scale, what):
+    g = got.float().cpu().numpy().astype(np.float64)
+    tol = 1e-5 * scale + 1e-6 + (2.0 ** -8 * np.abs(ref) if got.dtype == torch.bfloat16 else 0.0)
+    bad = np.abs(g - ref) > tol
+    assert not bad.any(), f"{what}: {int(bad.sum())} of {bad.size} beyond tolerance, worst {np.abs(g - ref).max():.3e}"
+
+
+@pytest.mark.parametrize("M,N", [(1, 256), (128, 256), (129, 1280), (1000, 1280), (4113, 512)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_patch_embed_matches_oracle(M, N, out_dtype):
+    g = torch.Generator(device="cpu").manual_seed(M * 7 + N)
+    rows = torch.randn((M, 1536), generator=g).to(torch.bfloat16).cuda()
+    w = (torch.randn((N, 1536), generator=g) * 0.02).to(torch.bfloat16).cuda()
+    bias = torch.randn(N, generator=g).cuda() if M % 2 else None
+    out = mimo.patch_embed(rows, w, bias, out_dtype=out_dtype)
+    ref, scale = _embed_ref(rows, w, bias)
+    _assert_embed_close(out, ref, scale, f"M={M} N={N}")
+
+
+def test_preprocess_then_patch_embed_chain():
+    imgs = workloads.random_small_batch(700, 10, max_side=300, min_side=1)
+    mean, std = workloads.CLIP_MEAN, workloads.CLIP_STD
+    pv, grid, _ = mimo.preprocess(imgs, mean, std, dtype=torch.bfloat16)
+    g = torch.Generator(device="cpu").manual_seed(1)
+    w = (torch.randn((1280, 1536), generator=g) * 0.02).to(torch.bfloat16).cuda()
+    out = mimo.patch_embed(pv, w)
+    # oracle chain: fp64 rows rounded to bf16 (the tower consumes bf16 rows), then the fp64 contraction
+    ref_rows, _, _ = oracle.preprocess(imgs, mean, std, threads=8)
+    a = oracle.bf16_bits_to_f32(oracle.round_to_bf16(ref_rows))
+    ref = oracle.patch_embed(a, w.float().cpu().numpy())
+    scale = np.abs(a.astype(np.float64)) @ np.abs(w.float().cpu().numpy().astype(np.float64)).T
+    # the GPU's bf16 rows may differ from the oracle's by one bf16 ulp: allow that through the weights
+    tol_rows = 2.0 ** -8 * scale
+    g_out = out.float().cpu().numpy().astype(np.float64)
+    tol = tol_rows + 1e-5 * scale + 2.0 ** -8 * np.abs(ref) + 1e-6
+    assert (np.abs(g_out - ref) <= tol).all(), np.abs(g_out - ref).max()

@@ -558,6 +558,20 @@ int mimo_expand_prompt_ids(const int32_t *ids, int64_t n_ids, int32_t pad_id, co
     return MIMO_OK;
 }
 
+int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int32_t embed_dim, const float *d_bias,
+                     int32_t out_dtype, void *d_out, int32_t *d_error, void *stream) {
+    if (rows < 0 || embed_dim <= 0 || (embed_dim % 256) != 0) return MIMO_EINVAL;
+    if (out_dtype != MIMO_F32 && out_dtype != MIMO_BF16) return MIMO_EINVAL;
+    if (rows == 0) return MIMO_OK;
+    if (!d_rows || !d_weight || !d_out || !d_error) return MIMO_EINVAL;
+    if (!aligned16(d_rows) || !aligned16(d_weight) || !aligned16(d_out) || (d_bias && !aligned16(d_bias)) ||
+        (reinterpret_cast<uintptr_t>(d_error) & 3u) != 0)
+        return MIMO_EALIGN;
+    if (rows > (int64_t(1) << 31) - 1) return MIMO_EOVERFLOW;  // TMA coordinates are int32
+    return mimo::launch_patch_embed(d_rows, rows, mimo::kRowWidth, d_weight, embed_dim, d_bias, out_dtype, d_out,
+                                    d_error, stream);
+}
+
 const char *mimo_status_string(int status) {
     switch (status) {
         case MIMO_OK: return "ok";

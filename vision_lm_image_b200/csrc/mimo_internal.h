@@ -102,6 +102,10 @@ MIMO_HD int64_t block_span(int64_t b, int64_t in, int64_t out) {
 
 int launch_preprocess(const LaunchParams &lp, int64_t blocks, int out_dtype, size_t smem_bytes, void *stream);
 
+// Patch embedding GEMM on the tensor cores (mimo_patch_embed.cu).
+int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_weight, int32_t N, const float *d_bias,
+                       int32_t out_dtype, void *d_out, int32_t *d_err, void *stream);
+
 // Device address and size of the library's fixed staging area on the
 // current device (mimo_noalloc.cu).
 int noalloc_staging(void **dev_ptr, size_t *bytes);

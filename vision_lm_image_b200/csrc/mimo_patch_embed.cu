@@ -1,0 +1,320 @@
+// mimo_patch_embed.cu -- the vision tower's patch embedding on the 5th-gen
+// tensor cores (NeMo Automodel "mimo_v2_flash.vision", MiMoVisionPatchEmbed:
+// flattened spatiotemporal patches to vision tokens). The Conv3d with kernel =
+// stride = (2, 16, 16) is a dense contraction of each 1536-value patch row
+// with a [embed_dim, 1536] weight laid out (c, tt, py, px), the same order as
+// the rows:
+//
+//   C[m, n] = sum_k A[m, k] * B[n, k] (+ bias[n]),  A = patch rows (bf16),
+//   B = weight (bf16), accumulated in fp32, C in bf16 or fp32.
+//
+// One CTA per 128 x 256 tile of C. Warp 0 streams 64-wide K blocks of A and B
+// into a 4-stage shared-memory ring with TMA (128-byte swizzle); one lane of
+// warp 1 issues tcgen05.mma (M128 N256 K16, fp32 accumulator in TMEM) as the
+// stages land and frees each stage with tcgen05.commit; warps 2-5 read the
+// finished accumulator with tcgen05.ld, add the bias, convert and store.
+// Every wait on an mbarrier is bounded: on expiry the kernel records an error
+// code in *err, stops issuing work, waits (bounded) for copies it started,
+// frees its TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "mimo.h"
+#include "mimo_internal.h"
+
+namespace mimo {
+namespace {
+
+constexpr int kBM = 128, kBN = 256, kBK = 64;  // tile; kBK * 2 B = one 128-byte swizzle row
+constexpr int kStages = 4;
+constexpr int kUmmaK = 16;
+constexpr int kATileBytes = kBM * kBK * 2;  // 16 KB
+constexpr int kBTileBytes = kBN * kBK * 2;  // 32 KB
+constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kGemmThreads = 192;           // 6 warps
+constexpr int kTmemCols = 256;              // fp32 accumulator: 128 lanes x 256 columns
+constexpr uint32_t kWaitLimit = 1u << 20;   // try_wait rounds (about a second) before a wait is declared stuck
+
+enum : int { kErrNone = 0, kErrFullWait = 1, kErrEmptyWait = 2, kErrAccumWait = 3 };
+
+struct GemmSmem {
+    uint64_t full[kStages];   // TMA -> MMA: stage loaded
+    uint64_t empty[kStages];  // MMA -> TMA: stage consumed
+    uint64_t accum;           // MMA -> epilogue: accumulator complete
+    uint32_t tmem_base;
+    int32_t failed;           // a role gave up waiting: the others stop too
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Bounded wait for the phase with the given parity to complete; false if the
+// limit ran out (the caller records the error and stops).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+        "[%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile stored as 128-byte rows
+// with the 128-byte swizzle (what TMA writes with CU_TENSOR_MAP_SWIZZLE_128B):
+// start address >> 4, leading offset 16 B (unused by this layout), stride
+// 1024 B between groups of 8 rows, descriptor version 1, layout 128B swizzle.
+__device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+           (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+           (static_cast<uint64_t>(2) << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24);
+
+template <bool kOutBF16>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    patch_embed_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                       const float *__restrict__ bias, void *__restrict__ out, int64_t M, int32_t N, int32_t K,
+                       int32_t *__restrict__ err) {
+    extern __shared__ __align__(1024) uint8_t gemm_smem_raw[];
+    // 1024-byte aligned tiles (the swizzle pattern repeats every 1024 bytes)
+    uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ GemmSmem S;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = N / kBN;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.x / n_tiles) * kBM;
+    const int n0 = static_cast<int>(blockIdx.x % n_tiles) * kBN;
+    const int kblocks = K / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&S.full[s], 1);
+            mbar_init(&S.empty[s], 1);
+        }
+        mbar_init(&S.accum, 1);
+        S.failed = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == 0) {
+        // ---- producer: TMA into the stage ring
+        int issued = 0;
+        if (lane == 0) {
+            for (int kb = 0; kb < kblocks; ++kb) {
+                const int s = kb % kStages;
+                const uint32_t use = kb / kStages;
+                if (kb >= kStages && !mbar_wait(&S.empty[s], (use - 1) & 1)) {
+                    atomicCAS(err, kErrNone, kErrEmptyWait);
+                    S.failed = 1;
+                    break;
+                }
+                if (*reinterpret_cast<volatile int32_t *>(&S.failed)) break;
+                uint8_t *a = tiles + s * kStageBytes;
+                uint8_t *b = a + kATileBytes;
+                mbar_expect_tx(&S.full[s], kStageBytes);
+                tma_load_2d(a, &map_a, &S.full[s], kb * kBK, static_cast<int>(m0));
+                tma_load_2d(b, &map_b, &S.full[s], kb * kBK, n0);
+                ++issued;
+            }
+            // copies still in flight land before the CTA can leave (bounded)
+            for (int kb = (issued > kStages ? issued - kStages : 0); kb < issued; ++kb)
+                mbar_wait(&S.full[kb % kStages], (kb / kStages) & 1);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer: one lane drives the tensor core
+        if (lane == 0) {
+            bool ok = true;
+            for (int kb = 0; kb < kblocks && ok; ++kb) {
+                const int s = kb % kStages;
+                if (!mbar_wait(&S.full[s], (kb / kStages) & 1)) {
+                    atomicCAS(err, kErrNone, kErrFullWait);
+                    S.failed = 1;
+                    ok = false;
+                    break;
+                }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t a = smem_u32(tiles + s * kStageBytes);
+                const uint32_t b = a + kATileBytes;
+#pragma unroll
+                for (int k = 0; k < kBK / kUmmaK; ++k) {
+                    // advancing 16 bf16 (32 bytes) inside the swizzled 128-byte row
+                    const uint64_t da = kmajor_sw128_desc(a + k * kUmmaK * 2);
+                    const uint64_t db = kmajor_sw128_desc(b + k * kUmmaK * 2);
+                    const uint32_t accumulate = (kb > 0 || k > 0) ? 1u : 0u;
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\t"
+                        "setp.ne.b32 p, %4, 0;\n\t"
+                        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                        "l"(da), "l"(db), "r"(kInstrDesc), "r"(accumulate)
+                        : "memory");
+                }
+                // the stage is free once these MMAs have read it
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 smem_u32(&S.empty[s]))
+                             : "memory");
+            }
+            if (ok)
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 smem_u32(&S.accum))
+                             : "memory");
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31 (its accessible quarter)
+        const int quarter = warp & 3;
+        // uniform across the warp: tcgen05.ld below is a warp-wide instruction
+        const bool ready = __all_sync(0xffffffffu, mbar_wait(&S.accum, 0));
+        if (!ready) {
+            if (lane == 0) atomicCAS(err, kErrNone, kErrAccumWait);
+        } else {
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const int64_t row = m0 + quarter * 32 + lane;
+            for (int c0 = 0; c0 < kBN; c0 += 32) {
+                uint32_t v[32];
+                const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(c0);
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                    "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                      "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+                      "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
+                      "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
+                      "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                    : "r"(taddr));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                if (row < M) {
+                    float f[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]) + (bias ? bias[n0 + c0 + j] : 0.0f);
+                    if constexpr (kOutBF16) {
+                        uint4 *o = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + row * N + n0 + c0);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint4 u;
+                            __nv_bfloat162 p0 = __floats2bfloat162_rn(f[8 * j + 0], f[8 * j + 1]);
+                            __nv_bfloat162 p1 = __floats2bfloat162_rn(f[8 * j + 2], f[8 * j + 3]);
+                            __nv_bfloat162 p2 = __floats2bfloat162_rn(f[8 * j + 4], f[8 * j + 5]);
+                            __nv_bfloat162 p3 = __floats2bfloat162_rn(f[8 * j + 6], f[8 * j + 7]);
+                            u.x = *reinterpret_cast<uint32_t *>(&p0);
+                            u.y = *reinterpret_cast<uint32_t *>(&p1);
+                            u.z = *reinterpret_cast<uint32_t *>(&p2);
+                            u.w = *reinterpret_cast<uint32_t *>(&p3);
+                            __stcs(o + j, u);
+                        }
+                    } else {
+                        float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + row * N + n0 + c0);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            __stcs(o + j, make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]));
+                    }
+                }
+            }
+        }
+    }
+
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 1) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 row-major [rows, cols] map with a box of box_rows x 64 columns,
+// 128-byte swizzle; rows past the end read as zero.
+bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_weight, int32_t N, const float *d_bias,
+                       int32_t out_dtype, void *d_out, int32_t *d_err, void *stream) {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, d_rows, M, K, kBM) || !make_map(&mb, d_weight, N, K, kBN)) return MIMO_ECUDA;
+    const int64_t tiles = ((M + kBM - 1) / kBM) * (N / kBN);
+    if (tiles > INT32_MAX) return MIMO_EOVERFLOW;
+    const size_t smem = static_cast<size_t>(kStages) * kStageBytes + 1024;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (out_dtype == MIMO_BF16) {
+        if (cudaFuncSetAttribute(patch_embed_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess)
+            return MIMO_ECUDA;
+        patch_embed_kernel<true><<<static_cast<unsigned>(tiles), kGemmThreads, smem, s>>>(ma, mb, d_bias, d_out, M, N,
+                                                                                            K, d_err);
+    } else {
+        if (cudaFuncSetAttribute(patch_embed_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess)
+            return MIMO_ECUDA;
+        patch_embed_kernel<false><<<static_cast<unsigned>(tiles), kGemmThreads, smem, s>>>(ma, mb, d_bias, d_out, M,
+                                                                                             N, K, d_err);
+    }
+    return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
+}
+
+}  // namespace mimo

@@ -38,6 +38,7 @@ EXPORTED = ("mimo_params_default", "mimo_smart_resize", "mimo_num_patches", "mim
             "mimo_preprocess_batch", "mimo_preprocess_batch_ex", "mimo_preprocess_batch_host",
             "mimo_preprocess_batch_host_noalloc", "mimo_expand_prompt_ids", "mimo_video_max_pixels",
             "mimo_smart_nframes", "mimo_sample_frames", "mimo_plan_video", "mimo_preprocess_video",
+            "mimo_patch_embed",
             "mimo_status_string", "mimo_version")
 NOALLOC_STAGING_BYTES = 64 << 20
 
@@ -133,6 +134,8 @@ def lib() -> ctypes.CDLL:
             L.mimo_preprocess_video.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _i64, _i32, _i32, _i32,
                                                 _i64, ctypes.POINTER(MimoOutputs), _p]
             L.mimo_preprocess_video.restype = ctypes.c_int
+            L.mimo_patch_embed.argtypes = [_p, _i64, _p, _i32, _p, _i32, _p, _p, _p]
+            L.mimo_patch_embed.restype = ctypes.c_int
             L.mimo_status_string.argtypes = [ctypes.c_int]
             L.mimo_status_string.restype = ctypes.c_char_p
             L.mimo_version.argtypes = []
@@ -463,6 +466,41 @@ def preprocess_video(frames, mean=None, std=None, min_pixels: int | None = None,
     if positions or window_index:
         return out, g, perm, pos, win
     return out, g, perm
+
+
+# ----------------------------------------------------------------- patch embedding (tensor cores)
+class PatchEmbedError(RuntimeError):
+    pass
+
+
+def patch_embed(rows, weight, bias=None, out_dtype=None, out=None, error=None, stream=None, check: bool = True):
+    """out [M, embed_dim] = rows [M, 1536] (bf16, CUDA) @ weight [embed_dim, 1536]^T (bf16) (+ bias fp32).
+
+    ``error`` is an optional int32 CUDA tensor of one element that receives the
+    kernel's status word; with ``check`` the call synchronises and raises if it
+    is nonzero.
+    """
+    import torch
+
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    if rows.dtype != torch.bfloat16 or weight.dtype != torch.bfloat16:
+        raise ValueError("rows and weight must be bfloat16")
+    M = rows.shape[0]
+    N = weight.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=rows.device)
+    if error is None:
+        error = torch.zeros(1, dtype=torch.int32, device=rows.device)
+    _check(lib().mimo_patch_embed(ctypes.c_void_p(rows.data_ptr()), M, ctypes.c_void_p(weight.data_ptr()), N,
+                                  ctypes.c_void_p(bias.data_ptr() if bias is not None else 0), _dtype_code(out.dtype),
+                                  ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(error.data_ptr()),
+                                  _stream_handle(stream, rows.device)), "patch_embed")
+    if check:
+        torch.cuda.current_stream(rows.device).synchronize() if stream is None else stream.synchronize()
+        code = int(error.item())
+        if code != 0:
+            raise PatchEmbedError(f"patch_embed kernel stopped waiting on its pipeline (code {code})")
+    return out
 
 
 # ----------------------------------------------------------------- host-to-host path
