@@ -8,14 +8,19 @@
 //   C[m, n] = sum_k A[m, k] * B[n, k] (+ bias[n]),  A = patch rows (bf16),
 //   B = weight (bf16), accumulated in fp32, C in bf16 or fp32.
 //
-// One CTA per 128 x 256 tile of C. Warp 0 streams 64-wide K blocks of A and B
-// into a 4-stage shared-memory ring with TMA (128-byte swizzle); one lane of
-// warp 1 issues tcgen05.mma (M128 N256 K16, fp32 accumulator in TMEM) as the
-// stages land and frees each stage with tcgen05.commit; warps 2-5 read the
-// finished accumulator with tcgen05.ld, add the bias, convert and store.
+// Persistent kernel, one CTA per SM, walking the 128 x 256 tiles of C in
+// m-major order (the embed_dim / 256 tiles that share rows run side by side, so
+// each row block is read from HBM once). Warp 0 streams 64-wide K blocks of A
+// and B into a 4-stage shared-memory ring with TMA (128-byte swizzle); one lane
+// of warp 1 issues tcgen05.mma (M128 N256 K16, fp32 accumulator in TMEM) as
+// the stages land and frees each stage with tcgen05.commit; warps 2-5 drain
+// the finished accumulator with tcgen05.ld, add the bias, convert and store.
+// TMEM holds two accumulators (2 x 256 columns), so the epilogue of one tile
+// runs under the MMAs of the next.
 // Every wait on an mbarrier is bounded: on expiry the kernel records an error
-// code in *err, stops issuing work, waits (bounded) for copies it started,
-// frees its TMEM and exits.
+// code in *err, every role stops issuing work, the producer waits (bounded) for
+// the copies it started, the MMA lane for the MMAs it issued, and the TMEM is
+// freed before exit.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -37,15 +42,20 @@ constexpr int kATileBytes = kBM * kBK * 2;  // 16 KB
 constexpr int kBTileBytes = kBN * kBK * 2;  // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kGemmThreads = 192;           // 6 warps
-constexpr int kTmemCols = 256;              // fp32 accumulator: 128 lanes x 256 columns
-constexpr uint32_t kWaitLimit = 1u << 20;   // try_wait rounds (about a second) before a wait is declared stuck
+constexpr int kAccCols = kBN;               // one fp32 accumulator: 128 lanes x 256 columns
+constexpr int kTmemCols = 2 * kAccCols;     // double-buffered
+constexpr int kEpiWarps = 4;
+constexpr uint32_t kWaitLimit = 1u << 20;   // try_wait rounds before a wait is declared stuck
 
-enum : int { kErrNone = 0, kErrFullWait = 1, kErrEmptyWait = 2, kErrAccumWait = 3 };
+enum : int { kErrNone = 0, kErrFullWait = 1, kErrEmptyWait = 2, kErrAccumWait = 3, kErrAccumFreeWait = 4,
+             kErrDrainWait = 5 };
 
 struct GemmSmem {
     uint64_t full[kStages];   // TMA -> MMA: stage loaded
     uint64_t empty[kStages];  // MMA -> TMA: stage consumed
-    uint64_t accum;           // MMA -> epilogue: accumulator complete
+    uint64_t acc_full[2];     // MMA -> epilogue: accumulator b complete
+    uint64_t acc_free[2];     // epilogue -> MMA: accumulator b drained
+    uint64_t drain;           // MMA lane: every MMA it issued has completed
     uint32_t tmem_base;
     int32_t failed;           // a role gave up waiting: the others stop too
 };
@@ -61,6 +71,10 @@ __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
 __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Bounded wait for the phase with the given parity to complete; false if the
@@ -81,12 +95,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     return false;
 }
 
+__device__ __forceinline__ bool stopped(const GemmSmem &S) {
+    return *reinterpret_cast<const volatile int32_t *>(&S.failed) != 0;
+}
+
+__device__ __forceinline__ void fail(GemmSmem &S, int32_t *err, int code) {
+    atomicCAS(err, kErrNone, code);
+    *reinterpret_cast<volatile int32_t *>(&S.failed) = 1;
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
         "[%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
 }
 
 // Shared-memory matrix descriptor of a K-major tile stored as 128-byte rows
@@ -104,6 +132,34 @@ __device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t saddr) {
 constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24);
 
 template <bool kOutBF16>
+__device__ __forceinline__ void store_chunk(void *out, int64_t row, int32_t N, int col, const uint32_t (&v)[32],
+                                            const float *__restrict__ bias) {
+    float f[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]) + (bias ? __ldg(bias + col + j) : 0.0f);
+    if constexpr (kOutBF16) {
+        uint4 *o = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + row * N + col);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            __nv_bfloat162 p0 = __floats2bfloat162_rn(f[8 * j + 0], f[8 * j + 1]);
+            __nv_bfloat162 p1 = __floats2bfloat162_rn(f[8 * j + 2], f[8 * j + 3]);
+            __nv_bfloat162 p2 = __floats2bfloat162_rn(f[8 * j + 4], f[8 * j + 5]);
+            __nv_bfloat162 p3 = __floats2bfloat162_rn(f[8 * j + 6], f[8 * j + 7]);
+            uint4 u;
+            u.x = *reinterpret_cast<uint32_t *>(&p0);
+            u.y = *reinterpret_cast<uint32_t *>(&p1);
+            u.z = *reinterpret_cast<uint32_t *>(&p2);
+            u.w = *reinterpret_cast<uint32_t *>(&p3);
+            __stcs(o + j, u);
+        }
+    } else {
+        float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + row * N + col);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) __stcs(o + j, make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]));
+    }
+}
+
+template <bool kOutBF16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     patch_embed_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                        const float *__restrict__ bias, void *__restrict__ out, int64_t M, int32_t N, int32_t K,
@@ -115,8 +171,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = N / kBN;
-    const int64_t m0 = static_cast<int64_t>(blockIdx.x / n_tiles) * kBM;
-    const int n0 = static_cast<int>(blockIdx.x % n_tiles) * kBN;
+    const int64_t m_tiles = (M + kBM - 1) / kBM;
+    const int64_t total_tiles = m_tiles * n_tiles;
     const int kblocks = K / kBK;
 
     if (threadIdx.x == 0) {
@@ -124,7 +180,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&S.full[s], 1);
             mbar_init(&S.empty[s], 1);
         }
-        mbar_init(&S.accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&S.acc_full[b], 1);
+            mbar_init(&S.acc_free[b], kEpiWarps);
+        }
+        mbar_init(&S.drain, 1);
         S.failed = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -140,81 +200,94 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = S.tmem_base;
 
     if (warp == 0) {
-        // ---- producer: TMA into the stage ring
-        int issued = 0;
+        // ---- producer: TMA into the stage ring, k-block counter g runs across tiles
         if (lane == 0) {
-            for (int kb = 0; kb < kblocks; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t use = kb / kStages;
-                if (kb >= kStages && !mbar_wait(&S.empty[s], (use - 1) & 1)) {
-                    atomicCAS(err, kErrNone, kErrEmptyWait);
-                    S.failed = 1;
-                    break;
+            uint32_t g = 0;
+            for (int64_t t = blockIdx.x; t < total_tiles && !stopped(S); t += gridDim.x) {
+                const int m0 = static_cast<int>((t / n_tiles) * kBM);
+                const int n0 = static_cast<int>(t % n_tiles) * kBN;
+                for (int kb = 0; kb < kblocks; ++kb, ++g) {
+                    const uint32_t s = g % kStages, use = g / kStages;
+                    if (use > 0 && !mbar_wait(&S.empty[s], (use - 1) & 1)) {
+                        fail(S, err, kErrEmptyWait);
+                        break;
+                    }
+                    if (stopped(S)) break;
+                    uint8_t *a = tiles + s * kStageBytes;
+                    mbar_expect_tx(&S.full[s], kStageBytes);
+                    tma_load_2d(a, &map_a, &S.full[s], kb * kBK, m0);
+                    tma_load_2d(a + kATileBytes, &map_b, &S.full[s], kb * kBK, n0);
                 }
-                if (*reinterpret_cast<volatile int32_t *>(&S.failed)) break;
-                uint8_t *a = tiles + s * kStageBytes;
-                uint8_t *b = a + kATileBytes;
-                mbar_expect_tx(&S.full[s], kStageBytes);
-                tma_load_2d(a, &map_a, &S.full[s], kb * kBK, static_cast<int>(m0));
-                tma_load_2d(b, &map_b, &S.full[s], kb * kBK, n0);
-                ++issued;
             }
             // copies still in flight land before the CTA can leave (bounded)
-            for (int kb = (issued > kStages ? issued - kStages : 0); kb < issued; ++kb)
-                mbar_wait(&S.full[kb % kStages], (kb / kStages) & 1);
+            for (uint32_t q = (g > kStages ? g - kStages : 0); q < g; ++q)
+                mbar_wait(&S.full[q % kStages], (q / kStages) & 1);
         }
     } else if (warp == 1) {
         // ---- MMA issuer: one lane drives the tensor core
         if (lane == 0) {
-            bool ok = true;
-            for (int kb = 0; kb < kblocks && ok; ++kb) {
-                const int s = kb % kStages;
-                if (!mbar_wait(&S.full[s], (kb / kStages) & 1)) {
-                    atomicCAS(err, kErrNone, kErrFullWait);
-                    S.failed = 1;
-                    ok = false;
+            uint32_t g = 0, i = 0;
+            for (int64_t t = blockIdx.x; t < total_tiles && !stopped(S); t += gridDim.x, ++i) {
+                const uint32_t b = i & 1, use_b = i >> 1;
+                if (use_b > 0 && !mbar_wait(&S.acc_free[b], (use_b - 1) & 1)) {
+                    fail(S, err, kErrAccumFreeWait);
                     break;
                 }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const uint32_t a = smem_u32(tiles + s * kStageBytes);
-                const uint32_t b = a + kATileBytes;
+                const uint32_t acc = tmem + b * kAccCols;
+                bool ok = true;
+                for (int kb = 0; kb < kblocks; ++kb, ++g) {
+                    const uint32_t s = g % kStages;
+                    if (!mbar_wait(&S.full[s], (g / kStages) & 1)) {
+                        fail(S, err, kErrFullWait);
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const uint32_t a = smem_u32(tiles + s * kStageBytes);
+                    const uint32_t bb = a + kATileBytes;
 #pragma unroll
-                for (int k = 0; k < kBK / kUmmaK; ++k) {
-                    // advancing 16 bf16 (32 bytes) inside the swizzled 128-byte row
-                    const uint64_t da = kmajor_sw128_desc(a + k * kUmmaK * 2);
-                    const uint64_t db = kmajor_sw128_desc(b + k * kUmmaK * 2);
-                    const uint32_t accumulate = (kb > 0 || k > 0) ? 1u : 0u;
-                    asm volatile(
-                        "{\n\t.reg .pred p;\n\t"
-                        "setp.ne.b32 p, %4, 0;\n\t"
-                        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
-                        "l"(da), "l"(db), "r"(kInstrDesc), "r"(accumulate)
-                        : "memory");
+                    for (int k = 0; k < kBK / kUmmaK; ++k) {
+                        // advancing 16 bf16 (32 bytes) inside the swizzled 128-byte row
+                        const uint64_t da = kmajor_sw128_desc(a + k * kUmmaK * 2);
+                        const uint64_t db = kmajor_sw128_desc(bb + k * kUmmaK * 2);
+                        const uint32_t accumulate = (kb > 0 || k > 0) ? 1u : 0u;
+                        asm volatile(
+                            "{\n\t.reg .pred p;\n\t"
+                            "setp.ne.b32 p, %4, 0;\n\t"
+                            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(acc),
+                            "l"(da), "l"(db), "r"(kInstrDesc), "r"(accumulate)
+                            : "memory");
+                    }
+                    umma_commit(&S.empty[s]);  // the stage is free once these MMAs have read it
                 }
-                // the stage is free once these MMAs have read it
-                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                                 smem_u32(&S.empty[s]))
-                             : "memory");
+                if (!ok) break;
+                umma_commit(&S.acc_full[b]);
             }
-            if (ok)
-                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                                 smem_u32(&S.accum))
-                             : "memory");
+            // every MMA issued has finished before TMEM can be freed (bounded)
+            umma_commit(&S.drain);
+            if (!mbar_wait(&S.drain, 0)) fail(S, err, kErrDrainWait);
         }
         __syncwarp();
     } else {
         // ---- epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31 (its accessible quarter)
         const int quarter = warp & 3;
-        // uniform across the warp: tcgen05.ld below is a warp-wide instruction
-        const bool ready = __all_sync(0xffffffffu, mbar_wait(&S.accum, 0));
-        if (!ready) {
-            if (lane == 0) atomicCAS(err, kErrNone, kErrAccumWait);
-        } else {
+        uint32_t i = 0;
+        for (int64_t t = blockIdx.x; t < total_tiles; t += gridDim.x, ++i) {
+            const uint32_t b = i & 1;
+            // uniform across the warp: tcgen05.ld below is a warp-wide instruction
+            const bool ready = __all_sync(0xffffffffu, !stopped(S) && mbar_wait(&S.acc_full[b], (i >> 1) & 1));
+            if (!ready) {
+                if (lane == 0) fail(S, err, kErrAccumWait);
+                break;
+            }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const int64_t row = m0 + quarter * 32 + lane;
+            const int64_t row = (t / n_tiles) * kBM + quarter * 32 + lane;
+            const int n0 = static_cast<int>(t % n_tiles) * kBN;
+            const uint32_t base = tmem + b * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
+#pragma unroll 1
             for (int c0 = 0; c0 < kBN; c0 += 32) {
                 uint32_t v[32];
-                const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(c0);
                 asm volatile(
                     "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
                     "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -223,34 +296,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                       "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
                       "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
                       "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-                    : "r"(taddr));
+                    : "r"(base + static_cast<uint32_t>(c0)));
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                if (row < M) {
-                    float f[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]) + (bias ? bias[n0 + c0 + j] : 0.0f);
-                    if constexpr (kOutBF16) {
-                        uint4 *o = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + row * N + n0 + c0);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint4 u;
-                            __nv_bfloat162 p0 = __floats2bfloat162_rn(f[8 * j + 0], f[8 * j + 1]);
-                            __nv_bfloat162 p1 = __floats2bfloat162_rn(f[8 * j + 2], f[8 * j + 3]);
-                            __nv_bfloat162 p2 = __floats2bfloat162_rn(f[8 * j + 4], f[8 * j + 5]);
-                            __nv_bfloat162 p3 = __floats2bfloat162_rn(f[8 * j + 6], f[8 * j + 7]);
-                            u.x = *reinterpret_cast<uint32_t *>(&p0);
-                            u.y = *reinterpret_cast<uint32_t *>(&p1);
-                            u.z = *reinterpret_cast<uint32_t *>(&p2);
-                            u.w = *reinterpret_cast<uint32_t *>(&p3);
-                            __stcs(o + j, u);
-                        }
-                    } else {
-                        float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + row * N + n0 + c0);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            __stcs(o + j, make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]));
-                    }
+                if (c0 + 32 == kBN) {
+                    // the whole accumulator is in registers now: hand it back to the MMA lane
+                    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.acc_free[b]);
                 }
+                if (row < M) store_chunk<kOutBF16>(out, row, N, n0 + c0, v, bias);
             }
         }
     }
@@ -298,20 +352,24 @@ int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_w
     CUtensorMap ma, mb;
     if (!make_map(&ma, d_rows, M, K, kBM) || !make_map(&mb, d_weight, N, K, kBN)) return MIMO_ECUDA;
     const int64_t tiles = ((M + kBM - 1) / kBM) * (N / kBN);
-    if (tiles > INT32_MAX) return MIMO_EOVERFLOW;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return MIMO_ECUDA;
+    const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);  // persistent: one CTA per SM
     const size_t smem = static_cast<size_t>(kStages) * kStageBytes + 1024;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (out_dtype == MIMO_BF16) {
         if (cudaFuncSetAttribute(patch_embed_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
             return MIMO_ECUDA;
-        patch_embed_kernel<true><<<static_cast<unsigned>(tiles), kGemmThreads, smem, s>>>(ma, mb, d_bias, d_out, M, N,
+        patch_embed_kernel<true><<<grid, kGemmThreads, smem, s>>>(ma, mb, d_bias, d_out, M, N,
                                                                                             K, d_err);
     } else {
         if (cudaFuncSetAttribute(patch_embed_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
             return MIMO_ECUDA;
-        patch_embed_kernel<false><<<static_cast<unsigned>(tiles), kGemmThreads, smem, s>>>(ma, mb, d_bias, d_out, M,
+        patch_embed_kernel<false><<<grid, kGemmThreads, smem, s>>>(ma, mb, d_bias, d_out, M,
                                                                                              N, K, d_err);
     }
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
