@@ -8,15 +8,19 @@
 //   C[m, n] = sum_k A[m, k] * B[n, k] (+ bias[n]),  A = patch rows (bf16),
 //   B = weight (bf16), accumulated in fp32, C in bf16 or fp32.
 //
-// Persistent kernel, one CTA per SM, walking the 128 x 256 tiles of C in
-// m-major order (the embed_dim / 256 tiles that share rows run side by side, so
-// each row block is read from HBM once). Warp 0 streams 64-wide K blocks of A
-// and B into a 4-stage shared-memory ring with TMA (128-byte swizzle); one lane
-// of warp 1 issues tcgen05.mma (M128 N256 K16, fp32 accumulator in TMEM) as
-// the stages land and frees each stage with tcgen05.commit; warps 2-5 drain
-// the finished accumulator with tcgen05.ld, add the bias, convert and store.
-// TMEM holds two accumulators (2 x 256 columns), so the epilogue of one tile
-// runs under the MMAs of the next.
+// Persistent kernel on CTA pairs (clusters of two SMs), walking the 256 x 256
+// tiles of C in m-major order (the embed_dim / 256 tiles that share rows run
+// side by side, so each row block is read from HBM once). Each CTA of a pair
+// holds half of A (128 rows) and half of B (128 of the 256 weight rows) per
+// 64-wide K block; warp 0 of each CTA streams them with TMA (128-byte swizzle)
+// into a 6-stage ring and both halves signal the even CTA's barrier. One lane
+// of the even CTA issues tcgen05.mma.cta_group::2 (M256 N256 K16: the tensor
+// cores of both SMs, each reading its own half of A and both halves of B) and
+// frees each stage in both CTAs with a multicast tcgen05.commit. Warps 2-5 of
+// each CTA drain their 128 accumulator rows with tcgen05.ld, add the bias,
+// convert and store. TMEM holds two accumulators (2 x 256 columns) per CTA, so
+// the epilogue of one tile runs under the MMAs of the next. Splitting the tile
+// across the pair halves the weight bytes each SM stages per MMA.
 // Every wait on an mbarrier is bounded: on expiry the kernel records an error
 // code in *err, every role stops issuing work, the producer waits (bounded) for
 // the copies it started, the MMA lane for the MMAs it issued, and the TMEM is
@@ -35,33 +39,55 @@
 namespace mimo {
 namespace {
 
-constexpr int kBM = 128, kBN = 256, kBK = 64;  // tile; kBK * 2 B = one 128-byte swizzle row
-constexpr int kStages = 4;
+constexpr int kPairM = 256;                // rows of C per tile (128 per CTA of the pair)
+constexpr int kBM = 128;                    // rows of A per CTA
+constexpr int kBN = 256;                    // columns of C per tile
+constexpr int kBNHalf = kBN / 2;            // weight rows per CTA
+constexpr int kBK = 64;                     // kBK * 2 B = one 128-byte swizzle row
+constexpr int kStages = 6;
 constexpr int kUmmaK = 16;
-constexpr int kATileBytes = kBM * kBK * 2;  // 16 KB
-constexpr int kBTileBytes = kBN * kBK * 2;  // 32 KB
+constexpr int kATileBytes = kBM * kBK * 2;      // 16 KB
+constexpr int kBTileBytes = kBNHalf * kBK * 2;  // 16 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kGemmThreads = 192;           // 6 warps
-constexpr int kAccCols = kBN;               // one fp32 accumulator: 128 lanes x 256 columns
+constexpr int kAccCols = kBN;               // one fp32 accumulator: 128 lanes x 256 columns per CTA
 constexpr int kTmemCols = 2 * kAccCols;     // double-buffered
 constexpr int kEpiWarps = 4;
+constexpr uint16_t kPairMask = 0x3;         // both CTAs of the cluster
 constexpr uint32_t kWaitLimit = 1u << 20;   // try_wait rounds before a wait is declared stuck
 
 enum : int { kErrNone = 0, kErrFullWait = 1, kErrEmptyWait = 2, kErrAccumWait = 3, kErrAccumFreeWait = 4,
              kErrDrainWait = 5 };
 
 struct GemmSmem {
-    uint64_t full[kStages];   // TMA -> MMA: stage loaded
-    uint64_t empty[kStages];  // MMA -> TMA: stage consumed
-    uint64_t acc_full[2];     // MMA -> epilogue: accumulator b complete
-    uint64_t acc_free[2];     // epilogue -> MMA: accumulator b drained
-    uint64_t drain;           // MMA lane: every MMA it issued has completed
+    uint64_t full[kStages];   // even CTA: both halves of stage s landed (TMA of both CTAs)
+    uint64_t empty[kStages];  // each CTA: the pair's MMAs consumed stage s (multicast commit)
+    uint64_t acc_full[2];     // each CTA: accumulator b complete (multicast commit)
+    uint64_t acc_free[2];     // even CTA: all 8 epilogue warps of the pair drained accumulator b
+    uint64_t drain;           // even CTA: every MMA it issued has completed
     uint32_t tmem_base;
-    int32_t failed;           // a role gave up waiting: the others stop too
+    int32_t failed;           // a role of this CTA gave up waiting: the others stop too
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
@@ -73,19 +99,21 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
                  : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+// Arrive on a barrier given by its shared::cluster address (possibly the peer's).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
 // Bounded wait for the phase with the given parity to complete; false if the
-// limit ran out (the caller records the error and stops).
+// limit ran out (the caller records the error and stops). Cluster scope: some
+// of the arrivals come from the other CTA of the pair.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     const uint32_t a = smem_u32(bar);
     for (uint32_t i = 0; i < kWaitLimit; ++i) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(done)
             : "r"(a), "r"(parity)
@@ -104,16 +132,28 @@ __device__ __forceinline__ void fail(GemmSmem &S, int32_t *err, int code) {
     *reinterpret_cast<volatile int32_t *>(&S.failed) = 1;
 }
 
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
+// TMA tile load into this CTA's shared memory whose completion is counted on
+// the barrier at `cluster_bar` (the even CTA's, for both CTAs of the pair).
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, uint32_t cluster_bar, int x,
+                                                 int y) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-        "[%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(x), "r"(y)
         : "memory");
 }
 
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+// Arrive on the barrier at the same offset in both CTAs once the MMAs issued so far have completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(kPairMask)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_local(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
 }
 
@@ -128,8 +168,8 @@ __device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, N = 256, M = 128.
-constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24);
+// K-major, N = 256, M = 256 (the pair's tile).
+constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kPairM >> 4) << 24);
 
 template <bool kOutBF16>
 __device__ __forceinline__ void store_chunk(void *out, int64_t row, int32_t N, int col, const uint32_t (&v)[32],
@@ -165,13 +205,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                        const float *__restrict__ bias, void *__restrict__ out, int64_t M, int32_t N, int32_t K,
                        int32_t *__restrict__ err) {
     extern __shared__ __align__(1024) uint8_t gemm_smem_raw[];
-    // 1024-byte aligned tiles (the swizzle pattern repeats every 1024 bytes)
+    // 1024-byte aligned tiles (the swizzle pattern repeats every 1024 bytes); the
+    // offset is the same in both CTAs, as the pair MMA requires
     uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ GemmSmem S;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();     // 0: even CTA (issues the MMAs), 1: its peer
+    const bool leader = rank == 0;
+    const int64_t pair = blockIdx.x >> 1, pairs = gridDim.x >> 1;
     const int n_tiles = N / kBN;
-    const int64_t m_tiles = (M + kBM - 1) / kBM;
+    const int64_t m_tiles = (M + kPairM - 1) / kPairM;
     const int64_t total_tiles = m_tiles * n_tiles;
     const int kblocks = K / kBK;
 
@@ -182,30 +226,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&S.acc_full[b], 1);
-            mbar_init(&S.acc_free[b], kEpiWarps);
+            mbar_init(&S.acc_free[b], 2 * kEpiWarps);
         }
         mbar_init(&S.drain, 1);
         S.failed = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem_base)),
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem_base)),
                      "r"(kTmemCols)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = S.tmem_base;
 
     if (warp == 0) {
-        // ---- producer: TMA into the stage ring, k-block counter g runs across tiles
+        // ---- producer (both CTAs): this CTA's halves of A and B, k-block counter g runs across tiles
         if (lane == 0) {
             uint32_t g = 0;
-            for (int64_t t = blockIdx.x; t < total_tiles && !stopped(S); t += gridDim.x) {
-                const int m0 = static_cast<int>((t / n_tiles) * kBM);
-                const int n0 = static_cast<int>(t % n_tiles) * kBN;
+            for (int64_t t = pair; t < total_tiles && !stopped(S); t += pairs) {
+                const int a_row = static_cast<int>((t / n_tiles) * kPairM) + static_cast<int>(rank) * kBM;
+                const int b_row = static_cast<int>(t % n_tiles) * kBN + static_cast<int>(rank) * kBNHalf;
                 for (int kb = 0; kb < kblocks; ++kb, ++g) {
                     const uint32_t s = g % kStages, use = g / kStages;
                     if (use > 0 && !mbar_wait(&S.empty[s], (use - 1) & 1)) {
@@ -214,20 +258,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     if (stopped(S)) break;
                     uint8_t *a = tiles + s * kStageBytes;
-                    mbar_expect_tx(&S.full[s], kStageBytes);
-                    tma_load_2d(a, &map_a, &S.full[s], kb * kBK, m0);
-                    tma_load_2d(a + kATileBytes, &map_b, &S.full[s], kb * kBK, n0);
+                    if (leader) mbar_expect_tx(&S.full[s], 2 * kStageBytes);  // both CTAs' halves
+                    const uint32_t full_bar = cluster_addr(&S.full[s], 0);
+                    tma_load_2d_pair(a, &map_a, full_bar, kb * kBK, a_row);
+                    tma_load_2d_pair(a + kATileBytes, &map_b, full_bar, kb * kBK, b_row);
                 }
             }
-            // copies still in flight land before the CTA can leave (bounded)
-            for (uint32_t q = (g > kStages ? g - kStages : 0); q < g; ++q)
-                mbar_wait(&S.full[q % kStages], (q / kStages) & 1);
+            // copies still in flight land before the CTA can leave (bounded; the even
+            // CTA's barrier counts the peer's copies as well)
+            if (leader)
+                for (uint32_t q = (g > kStages ? g - kStages : 0); q < g; ++q)
+                    mbar_wait(&S.full[q % kStages], (q / kStages) & 1);
         }
     } else if (warp == 1) {
-        // ---- MMA issuer: one lane drives the tensor core
-        if (lane == 0) {
+        // ---- MMA issuer: one lane of the even CTA drives the tensor cores of both SMs
+        if (leader && lane == 0) {
             uint32_t g = 0, i = 0;
-            for (int64_t t = blockIdx.x; t < total_tiles && !stopped(S); t += gridDim.x, ++i) {
+            for (int64_t t = pair; t < total_tiles && !stopped(S); t += pairs, ++i) {
                 const uint32_t b = i & 1, use_b = i >> 1;
                 if (use_b > 0 && !mbar_wait(&S.acc_free[b], (use_b - 1) & 1)) {
                     fail(S, err, kErrAccumFreeWait);
@@ -255,25 +302,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         asm volatile(
                             "{\n\t.reg .pred p;\n\t"
                             "setp.ne.b32 p, %4, 0;\n\t"
-                            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(acc),
+                            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(acc),
                             "l"(da), "l"(db), "r"(kInstrDesc), "r"(accumulate)
                             : "memory");
                     }
-                    umma_commit(&S.empty[s]);  // the stage is free once these MMAs have read it
+                    umma_commit_pair(&S.empty[s]);  // stage s is free in both CTAs once these MMAs have read it
                 }
                 if (!ok) break;
-                umma_commit(&S.acc_full[b]);
+                umma_commit_pair(&S.acc_full[b]);
             }
             // every MMA issued has finished before TMEM can be freed (bounded)
-            umma_commit(&S.drain);
+            umma_commit_local(&S.drain);
             if (!mbar_wait(&S.drain, 0)) fail(S, err, kErrDrainWait);
         }
-        __syncwarp();
     } else {
-        // ---- epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31 (its accessible quarter)
+        // ---- epilogue (both CTAs): warp w reads TMEM lanes 32*(w % 4) .. +31 (its accessible quarter)
         const int quarter = warp & 3;
         uint32_t i = 0;
-        for (int64_t t = blockIdx.x; t < total_tiles; t += gridDim.x, ++i) {
+        for (int64_t t = pair; t < total_tiles; t += pairs, ++i) {
             const uint32_t b = i & 1;
             // uniform across the warp: tcgen05.ld below is a warp-wide instruction
             const bool ready = __all_sync(0xffffffffu, !stopped(S) && mbar_wait(&S.acc_full[b], (i >> 1) & 1));
@@ -282,7 +328,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 break;
             }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const int64_t row = (t / n_tiles) * kBM + quarter * 32 + lane;
+            const int64_t row = (t / n_tiles) * kPairM + rank * kBM + quarter * 32 + lane;
             const int n0 = static_cast<int>(t % n_tiles) * kBN;
             const uint32_t base = tmem + b * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
@@ -302,19 +348,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     // the whole accumulator is in registers now: hand it back to the MMA lane
                     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&S.acc_free[b]);
+                    if (lane == 0) mbar_arrive_cluster(cluster_addr(&S.acc_free[b], 0));
                 }
                 if (row < M) store_chunk<kOutBF16>(out, row, N, n0 + c0, v, bias);
             }
         }
     }
 
+    // both CTAs stay until the pair is done with each other's barriers, shared
+    // memory and TMEM; then each frees its TMEM
+    __syncwarp();
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
-    if (warp == 1) {
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
-    }
+    cluster_sync();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
 // ---------------------------------------------------------------- host side
@@ -350,28 +398,34 @@ bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, in
 int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_weight, int32_t N, const float *d_bias,
                        int32_t out_dtype, void *d_out, int32_t *d_err, void *stream) {
     CUtensorMap ma, mb;
-    if (!make_map(&ma, d_rows, M, K, kBM) || !make_map(&mb, d_weight, N, K, kBN)) return MIMO_ECUDA;
-    const int64_t tiles = ((M + kBM - 1) / kBM) * (N / kBN);
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-        return MIMO_ECUDA;
-    const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);  // persistent: one CTA per SM
+    if (!make_map(&ma, d_rows, M, K, kBM) || !make_map(&mb, d_weight, N, K, kBNHalf)) return MIMO_ECUDA;
+    const int64_t tiles = ((M + kPairM - 1) / kPairM) * (N / kBN);
     const size_t smem = static_cast<size_t>(kStages) * kStageBytes + 1024;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (out_dtype == MIMO_BF16) {
-        if (cudaFuncSetAttribute(patch_embed_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess)
-            return MIMO_ECUDA;
-        patch_embed_kernel<true><<<grid, kGemmThreads, smem, s>>>(ma, mb, d_bias, d_out, M, N,
-                                                                                            K, d_err);
-    } else {
-        if (cudaFuncSetAttribute(patch_embed_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess)
-            return MIMO_ECUDA;
-        patch_embed_kernel<false><<<grid, kGemmThreads, smem, s>>>(ma, mb, d_bias, d_out, M,
-                                                                                             N, K, d_err);
-    }
+    auto kernel = out_dtype == MIMO_BF16 ? patch_embed_kernel<true> : patch_embed_kernel<false>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+        return MIMO_ECUDA;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: as many pairs as can be resident at once (one CTA per SM)
+    int dev = 0, sms = 0, max_pairs = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2)
+        return MIMO_ECUDA;
+    cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
+    if (cudaOccupancyMaxActiveClusters(&max_pairs, kernel, &cfg) != cudaSuccess || max_pairs < 1) return MIMO_ECUDA;
+    const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, kernel, ma, mb, d_bias, d_out, M, N, K, d_err) != cudaSuccess) return MIMO_ECUDA;
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
 }
 
