@@ -55,6 +55,7 @@ def parse():
     ap.add_argument("--workload", default="c5", choices=["c2", "c3", "c4", "c5", "v1", "pe"],
                     help="pe: the patch embedding GEMM on the bf16 rows of c5 (--images sets the image count)")
     ap.add_argument("--embed-dim", type=int, default=1280, help="pe: output width of the patch embedding")
+    ap.add_argument("--gemm-only", action="store_true", help="pe: time the GEMM alone (no cuBLAS, no pixel chain)")
     ap.add_argument("--dtype", default=None, choices=["f32", "bf16"])
     ap.add_argument("--images", type=int, default=None, help="override the workload's image count")
     ap.add_argument("--order", default="merge", choices=["merge", "column"], help="row order of the output")
@@ -74,16 +75,25 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_digest() -> str:
+KERNEL_SOURCES = {
+    "preprocess": ("vision_lm_image_b200/csrc/mimo_preprocess.cu", "vision_lm_image_b200/csrc/mimo_internal.h"),
+    "patch_embed": ("vision_lm_image_b200/csrc/mimo_patch_embed.cu", "vision_lm_image_b200/csrc/mimo_internal.h"),
+}
+
+
+def kernel_source_digest(kernel: str = "preprocess") -> str:
     h = hashlib.sha256()
-    for rel in ("vision_lm_image_b200/csrc/mimo_preprocess.cu", "vision_lm_image_b200/csrc/mimo_internal.h"):
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str, dtype: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+def ncu_traffic(workload: str, dtype: str, kernel: str = "preprocess", rows: int | None = None):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source.
+
+    An entry captured on a smaller case than the launch timed here (``full_rows``
+    differs from ``rows``) is scaled by rows."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -91,9 +101,12 @@ def ncu_traffic(workload: str, dtype: str):
     except Exception:
         return None
     entry = d.get(f"{workload}_{dtype}")
-    if not entry or entry.get("kernel_digest") != kernel_source_digest():
+    if not entry or entry.get("kernel_digest") != kernel_source_digest(kernel):
         return None
-    return entry.get("dram_bytes_per_launch")
+    traffic = entry.get("dram_bytes_per_launch")
+    if rows is not None and entry.get("full_rows") and entry["full_rows"] != rows:
+        traffic = int(round(traffic * rows / entry["full_rows"]))
+    return traffic
 
 
 class ClockSampler:
@@ -269,6 +282,31 @@ def run_video(args, rank, world, local_rank):
         }), flush=True)
 
 
+def compare_patch_embed(args, mimo, w, dev, rows, weight, bias, out, err, stream, timed):
+    """cuBLAS on the same operands, and pixels -> embeddings as two calls vs the chunked entry point."""
+    import torch
+
+    out_ref = torch.empty_like(out)
+    lib_step = lambda: torch.addmm(bias.to(torch.bfloat16), rows, weight.t(), out=out_ref)
+    for _ in range(max(args.warmup, 0)):
+        lib_step()
+    lib_ms = timed(lib_step, args.steps)
+    # the whole chain from uint8 pixels: two calls over the batch vs the chunked entry point
+    params = mimo.make_params(w["mean"], w["std"])
+    packed = mimo.pack_images(w["images"], device=dev)
+    scratch = torch.empty(96 << 20, dtype=torch.uint8, device=dev)
+    two = lambda: (mimo.preprocess_batch_ex(params, packed, rows, None, stream=stream),
+                   mimo.patch_embed(rows, weight, bias, out=out, error=err, stream=stream, check=False))
+    chain = lambda: mimo.preprocess_embed(packed, weight, bias, w["mean"], w["std"], scratch=scratch, stream=stream,
+                                          check=False)
+    for _ in range(max(args.warmup, 0)):
+        two()
+        chain()
+    two_ms = timed(two, args.steps)
+    chain_ms = timed(chain, args.steps)
+    return lib_ms, two_ms, chain_ms
+
+
 def run_patch_embed(args, rank, world, local_rank):
     """Tokens/s of the tensor-core patch embedding on the bf16 rows of the c5 batch (rows resident in HBM)."""
     import numpy as np
@@ -307,12 +345,10 @@ def run_patch_embed(args, rank, world, local_rank):
     code = int(err.item())
     if code:
         raise SystemExit(f"patch_embed reported pipeline error {code}")
-    # library GEMM on the same operands (cuBLAS through torch), for context
-    out_ref = torch.empty_like(out)
-    lib_step = lambda: torch.addmm(bias.to(torch.bfloat16), rows, weight.t(), out=out_ref)
-    for _ in range(max(args.warmup, 0)):
-        lib_step()
-    lib_ms = timed(lib_step, args.steps)
+    lib_ms = two_ms = chain_ms = float("nan")
+    n_img = len(w["images"])
+    if not args.gemm_only:
+        lib_ms, two_ms, chain_ms = compare_patch_embed(args, mimo, w, dev, rows, weight, bias, out, err, stream, timed)
     flops = 2.0 * M * N * K
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -345,9 +381,15 @@ def run_patch_embed(args, rank, world, local_rank):
                        "l2": "rows (%.1f GB) and output larger than L2 (no flush)" % (M * K * 2 / 1e9)},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "frac_of_sustained": achieved / peak_sus, "peak_kind": kind,
-                         "traffic": None, "algorithmic_flops_per_launch": flops, "kernel": "patch_embed_kernel",
+                         "traffic": ncu_traffic("pe", "bf16", "patch_embed", M),
+                         "algorithmic_flops_per_launch": flops, "kernel": "patch_embed_kernel",
+                         "algorithmic_bytes_per_launch": M * K * 2 + N * K * 2 + N * 4 + M * N * 2,
                          "avg_launch_ms": ms},
-            "library_gemm": {"impl": "torch.addmm (cuBLAS)", "ms": lib_ms, "tflops": flops / (lib_ms * 1e-3) / 1e12},
+            "library_gemm": None if args.gemm_only else {
+                "impl": "torch.addmm (cuBLAS)", "ms": lib_ms, "tflops": flops / (lib_ms * 1e-3) / 1e12},
+            "pixels_to_embeddings": None if args.gemm_only else {"images": n_img, "two_calls_ms": two_ms, "chained_ms": chain_ms,
+                                     "two_calls_images_per_s": n_img / (two_ms * 1e-3),
+                                     "chained_images_per_s": n_img / (chain_ms * 1e-3), "scratch_mb": 96},
             "gpu_launches": args.steps, "clocks": clocks.summary(), "e2e": None, "cpu_baseline": cpu,
         }), flush=True)
 

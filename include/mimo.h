@@ -326,6 +326,34 @@ int mimo_preprocess_video(const mimo_params *p, int32_t n_frames, const uint8_t 
 int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int32_t embed_dim,
                      const float *d_bias, int32_t out_dtype, void *d_out, int32_t *d_error, void *stream);
 
+/*
+ * The pixel path followed by the patch embedding, image chunk by image chunk
+ * (vision page, MiMoVisionTransformer.forward: patch rows -> patch embed).
+ * Images are grouped into runs whose bf16 patch rows fit d_scratch; for each
+ * run the pixel kernel writes the rows into the scratch and the
+ * patch-embedding GEMM (as mimo_patch_embed) reads them back, much of them
+ * still in L2, writing embeddings at the run's batch rows. Equal, bit for bit,
+ * to mimo_preprocess_batch_ex with MIMO_BF16 rows followed by
+ * mimo_patch_embed on them.
+ *   p, n, d_src, src_bytes, src_offsets, heights, widths, channels: as in
+ *       mimo_preprocess_batch.
+ *   row_order:  MIMO_ORDER_MERGE or MIMO_ORDER_COLUMN (order of the output rows).
+ *   d_weight, embed_dim, d_bias, out_dtype, d_error: as in mimo_patch_embed.
+ *   d_out:      device [total_rows, embed_dim] of out_dtype; out_rows_capacity
+ *               its row count (MIMO_ECAPACITY if below total_rows).
+ *   d_scratch:  device buffer of scratch_bytes, 16-byte aligned, owned by the
+ *               caller; it must hold one image's rows (rows x 3072 bytes),
+ *               MIMO_ECAPACITY otherwise. Larger runs fill the GPU better,
+ *               smaller ones stay in the 126 MB L2.
+ * No permutation or index tables (mimo_preprocess_batch_ex writes those).
+ * Asynchronous on `stream`.
+ */
+int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src, size_t src_bytes,
+                          const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
+                          const int32_t *channels, int32_t row_order, const void *d_weight, int32_t embed_dim,
+                          const float *d_bias, int32_t out_dtype, void *d_out, int64_t out_rows_capacity,
+                          void *d_scratch, size_t scratch_bytes, int32_t *d_error, void *stream);
+
 /* Static description of a status code. */
 const char *mimo_status_string(int status);
 

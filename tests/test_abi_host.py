@@ -241,3 +241,26 @@ def test_patch_embed_validation_statuses():
     assert call(a=0) == 1 and call(err=0) == 1
     assert call(a=FAKE + 8) == 6 and call(out=FAKE + 2) == 6 and call(bias=FAKE + 4) == 6 and call(err=FAKE + 2) == 6
     assert call(rows=1 << 31) == 8
+
+
+@no_gpu_only
+def test_preprocess_embed_validation_statuses():
+    L = mimo.lib()
+    P = ctypes.c_void_p
+    p = mimo.make_params()
+    offs = np.zeros(1, np.int64)
+    h = np.array([1080], np.int32)
+    w = np.array([1920], np.int32)
+    c = np.array([3], np.int32)
+
+    def call(order=0, n_embed=1280, scratch_bytes=1 << 30, cap=8160, weight=FAKE, scratch=FAKE, err=FAKE):
+        return L.mimo_preprocess_embed(ctypes.byref(p), 1, P(FAKE), 1080 * 1920 * 3, offs.ctypes.data,
+                                       h.ctypes.data, w.ctypes.data, c.ctypes.data, order, P(weight), n_embed,
+                                       P(0), 1, P(FAKE), cap, P(scratch), scratch_bytes, P(err), None)
+
+    assert call(order=5) == 1
+    assert call(n_embed=1000) == 1
+    assert call(cap=8159) == 7
+    assert call(weight=0) == 1 and call(scratch=0) == 1
+    assert call(scratch=FAKE + 8) == 6
+    assert call(scratch_bytes=8160 * 3072 - 2) == 7   # the scratch must hold one image's rows

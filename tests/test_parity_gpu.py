@@ -373,3 +373,41 @@ def test_preprocess_then_patch_embed_chain():
     g_out = out.float().cpu().numpy().astype(np.float64)
     tol = tol_rows + 1e-5 * scale + 2.0 ** -8 * np.abs(ref) + 1e-6
     assert (np.abs(g_out - ref) <= tol).all(), np.abs(g_out - ref).max()
+
+
+@pytest.mark.parametrize("order", ["merge", "column"])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_preprocess_embed_equals_two_step(order, out_dtype):
+    # chunked pixel path + GEMM through a small scratch (several runs) == the two calls on the whole batch
+    imgs = workloads.random_small_batch(701, 12, max_side=400, min_side=1)
+    mean, std = workloads.CLIP_MEAN, workloads.CLIP_STD
+    g = torch.Generator(device="cpu").manual_seed(2)
+    w = (torch.randn((512, 1536), generator=g) * 0.02).to(torch.bfloat16).cuda()
+    bias = torch.randn(512, generator=g).cuda()
+    rows, grid, _ = mimo.preprocess(imgs, mean, std, dtype=torch.bfloat16, order=order)
+    ref = mimo.patch_embed(rows, w, bias, out_dtype=out_dtype)
+    biggest = int((grid[:, 1] * grid[:, 2]).max())
+    emb, grid2 = mimo.preprocess_embed(imgs, w, bias, mean, std, out_dtype=out_dtype, order=order,
+                                       scratch_bytes=(biggest + 300) * 3072)
+    assert torch.equal(grid, grid2)
+    assert torch.equal(emb.view(torch.int16 if out_dtype == torch.bfloat16 else torch.int32),
+                       ref.view(torch.int16 if out_dtype == torch.bfloat16 else torch.int32))
+
+
+def test_preprocess_embed_c5_sample_against_oracle():
+    # full-size geometry (1080x1920 -> 8160 rows each, RGB and RGBA), default scratch; sampled rows vs the oracle chain
+    w5 = workloads.workload("c5", n_images=4)
+    g = torch.Generator(device="cpu").manual_seed(4)
+    w = (torch.randn((1280, 1536), generator=g) * 0.02).to(torch.bfloat16).cuda()
+    emb, grid = mimo.preprocess_embed(w5["images"], w, None, w5["mean"], w5["std"])
+    rng = np.random.Generator(np.random.PCG64(9))
+    wt = w.float().cpu().numpy()
+    for i in (0, 3):
+        rows = oracle.preprocess_image(w5["images"][i], w5["mean"], w5["std"])[0]
+        pick = rng.choice(rows.shape[0], 64, replace=False)
+        a = oracle.bf16_bits_to_f32(oracle.round_to_bf16(rows[pick]))
+        ref = oracle.patch_embed(a, wt)
+        scale = np.abs(a.astype(np.float64)) @ np.abs(wt.astype(np.float64)).T
+        got = emb[i * 8160 + pick].float().cpu().numpy().astype(np.float64)
+        tol = 2.0 ** -8 * scale + 1e-5 * scale + 2.0 ** -8 * np.abs(ref) + 1e-6
+        assert (np.abs(got - ref) <= tol).all(), np.abs(got - ref).max()

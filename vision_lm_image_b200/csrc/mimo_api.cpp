@@ -227,7 +227,7 @@ struct Tables {
 int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_t last, const uint8_t *d_src,
                  size_t src_bytes, const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
                  const int32_t *channels, int32_t out_dtype, void *d_out, int32_t *d_perm, void *stream,
-                 const Tables &tables = Tables()) {
+                 const Tables &tables = Tables(), int64_t row_base = 0) {
     static thread_local mimo::LaunchParams lp;  // 23 KB: kept off the stack
     int32_t i = first;
     while (i < last) {
@@ -246,7 +246,7 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
             const ImagePlan &ip = v.plan.img[i];
             mimo::ImageDesc &d = lp.img[k];
             d.src_off = src_offsets[i];
-            d.row0 = v.plan.row0[i];
+            d.row0 = v.plan.row0[i] - row_base;  // rows land at d_out + (row0 - row_base) * 1536
             d.H = heights[i];
             d.W = widths[i];
             d.Hr = static_cast<int32_t>(ip.Hr);
@@ -570,6 +570,47 @@ int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int
     if (rows > (int64_t(1) << 31) - 1) return MIMO_EOVERFLOW;  // TMA coordinates are int32
     return mimo::launch_patch_embed(d_rows, rows, mimo::kRowWidth, d_weight, embed_dim, d_bias, out_dtype, d_out,
                                     d_error, stream);
+}
+
+int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src, size_t src_bytes,
+                          const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
+                          const int32_t *channels, int32_t row_order, const void *d_weight, int32_t embed_dim,
+                          const float *d_bias, int32_t out_dtype, void *d_out, int64_t out_rows_capacity,
+                          void *d_scratch, size_t scratch_bytes, int32_t *d_error, void *stream) {
+    if (row_order != MIMO_ORDER_MERGE && row_order != MIMO_ORDER_COLUMN) return MIMO_EINVAL;
+    if (embed_dim <= 0 || (embed_dim % 256) != 0) return MIMO_EINVAL;
+    Validated v;
+    int st = validate_batch(p, n, d_src, src_bytes, src_offsets, heights, widths, channels, out_dtype, d_out,
+                            out_rows_capacity, nullptr, &v);
+    if (st != MIMO_OK || n == 0) return st;
+    if (!d_weight || !d_scratch || !d_error) return MIMO_EINVAL;
+    if (!aligned16(d_weight) || !aligned16(d_scratch) || (d_bias && !aligned16(d_bias)) ||
+        (reinterpret_cast<uintptr_t>(d_error) & 3u) != 0)
+        return MIMO_EALIGN;
+    if (v.total_rows > (int64_t(1) << 31) - 1) return MIMO_EOVERFLOW;
+    // a run is a sequence of whole images whose bf16 rows fit the scratch; on one
+    // stream the next run's pixel kernel starts after this run's GEMM has read them
+    const int64_t row_bytes = static_cast<int64_t>(mimo::kRowWidth) * 2;
+    const int64_t run_rows = static_cast<int64_t>(scratch_bytes) / row_bytes;
+    const size_t esz = out_dtype == MIMO_BF16 ? 2 : 4;
+    Tables tables;
+    tables.order = row_order;
+    for (int32_t i0 = 0; i0 < n;) {
+        int32_t i1 = i0;
+        while (i1 < n && v.plan.row0[i1 + 1] - v.plan.row0[i0] <= run_rows) ++i1;
+        if (i1 == i0) return MIMO_ECAPACITY;  // one image's rows exceed the scratch
+        const int64_t row_base = v.plan.row0[i0];
+        const int64_t rows = v.plan.row0[i1] - row_base;
+        st = launch_range(p, v, i0, i1, d_src, src_bytes, src_offsets, heights, widths, channels, MIMO_BF16,
+                          d_scratch, nullptr, stream, tables, row_base);
+        if (st != MIMO_OK) return st;
+        st = mimo::launch_patch_embed(d_scratch, rows, mimo::kRowWidth, d_weight, embed_dim, d_bias, out_dtype,
+                                      static_cast<uint8_t *>(d_out) + static_cast<size_t>(row_base) * embed_dim * esz,
+                                      d_error, stream);
+        if (st != MIMO_OK) return st;
+        i0 = i1;
+    }
+    return MIMO_OK;
 }
 
 const char *mimo_status_string(int status) {

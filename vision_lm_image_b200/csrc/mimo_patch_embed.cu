@@ -53,6 +53,8 @@ constexpr int kGemmThreads = 192;           // 6 warps
 constexpr int kAccCols = kBN;               // one fp32 accumulator: 128 lanes x 256 columns per CTA
 constexpr int kTmemCols = 2 * kAccCols;     // double-buffered
 constexpr int kEpiWarps = 4;
+constexpr int kStagePitch = 128 + 16;       // epilogue staging row: one 128-byte output line + pad (no bank conflicts)
+constexpr int kEpiStageBytes = 32 * kStagePitch;  // per epilogue warp: 32 rows
 constexpr uint16_t kPairMask = 0x3;         // both CTAs of the cluster
 constexpr uint32_t kWaitLimit = 1u << 20;   // try_wait rounds before a wait is declared stuck
 
@@ -171,14 +173,26 @@ __device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t saddr) {
 // K-major, N = 256, M = 256 (the pair's tile).
 constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kPairM >> 4) << 24);
 
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+}
+
+// 32 fp32 accumulator columns of this lane's row (+ bias) -> 128 or 64 bytes
+// of output at byte offset `off` of the lane's staging row.
 template <bool kOutBF16>
-__device__ __forceinline__ void store_chunk(void *out, int64_t row, int32_t N, int col, const uint32_t (&v)[32],
-                                            const float *__restrict__ bias) {
+__device__ __forceinline__ void stage_32(uint8_t *srow, int off, const uint32_t (&v)[32],
+                                         const float *__restrict__ bias, int col) {
     float f[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]) + (bias ? __ldg(bias + col + j) : 0.0f);
     if constexpr (kOutBF16) {
-        uint4 *o = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + row * N + col);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             __nv_bfloat162 p0 = __floats2bfloat162_rn(f[8 * j + 0], f[8 * j + 1]);
@@ -190,12 +204,13 @@ __device__ __forceinline__ void store_chunk(void *out, int64_t row, int32_t N, i
             u.y = *reinterpret_cast<uint32_t *>(&p1);
             u.z = *reinterpret_cast<uint32_t *>(&p2);
             u.w = *reinterpret_cast<uint32_t *>(&p3);
-            __stcs(o + j, u);
+            *reinterpret_cast<uint4 *>(srow + off + 16 * j) = u;
         }
     } else {
-        float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + row * N + col);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) __stcs(o + j, make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]));
+        for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4 *>(srow + off + 16 * j) =
+                make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
     }
 }
 
@@ -318,6 +333,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else {
         // ---- epilogue (both CTAs): warp w reads TMEM lanes 32*(w % 4) .. +31 (its accessible quarter)
         const int quarter = warp & 3;
+        uint8_t *stage = tiles + kStages * kStageBytes + (warp - 2) * kEpiStageBytes;
         uint32_t i = 0;
         for (int64_t t = pair; t < total_tiles; t += pairs, ++i) {
             const uint32_t b = i & 1;
@@ -328,29 +344,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 break;
             }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const int64_t row = (t / n_tiles) * kPairM + rank * kBM + quarter * 32 + lane;
+            // rows of this warp: row0 .. row0 + 31; lane `lane` holds row row0 + lane in TMEM
+            const int64_t row0 = (t / n_tiles) * kPairM + rank * kBM + quarter * 32;
             const int n0 = static_cast<int>(t % n_tiles) * kBN;
             const uint32_t base = tmem + b * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
+            // one output line (128 bytes) per row at a time: 64 bf16 or 32 fp32 columns
+            constexpr int kLineCols = kOutBF16 ? 64 : 32;
+            constexpr int kEsz = kOutBF16 ? 2 : 4;
 #pragma unroll 1
-            for (int c0 = 0; c0 < kBN; c0 += 32) {
+            for (int c0 = 0; c0 < kBN; c0 += kLineCols) {
                 uint32_t v[32];
-                asm volatile(
-                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-                    "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                      "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-                      "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
-                      "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
-                      "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-                    : "r"(base + static_cast<uint32_t>(c0)));
+                tmem_ld32(base + static_cast<uint32_t>(c0), v);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                if (c0 + 32 == kBN) {
-                    // the whole accumulator is in registers now: hand it back to the MMA lane
+                stage_32<kOutBF16>(stage + lane * kStagePitch, 0, v, bias, n0 + c0);
+                if constexpr (kOutBF16) {
+                    tmem_ld32(base + static_cast<uint32_t>(c0 + 32), v);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    stage_32<kOutBF16>(stage + lane * kStagePitch, 64, v, bias, n0 + c0 + 32);
+                }
+                if (c0 + kLineCols == kBN) {
+                    // the whole accumulator has been read: hand it back to the MMA lane
                     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(cluster_addr(&S.acc_free[b], 0));
                 }
-                if (row < M) store_chunk<kOutBF16>(out, row, N, n0 + c0, v, bias);
+                __syncwarp();
+                // 8 lanes per row: each store instruction writes 4 whole 128-byte lines
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = i * 4 + (lane >> 3);
+                    const int64_t row = row0 + r;
+                    const uint4 u = *reinterpret_cast<const uint4 *>(stage + r * kStagePitch + (lane & 7) * 16);
+                    if (row < M)
+                        __stcs(reinterpret_cast<uint4 *>(static_cast<uint8_t *>(out) +
+                                                         (row * N + n0 + c0) * kEsz + (lane & 7) * 16),
+                               u);
+                }
+                __syncwarp();
             }
         }
     }
@@ -400,7 +430,7 @@ int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_w
     CUtensorMap ma, mb;
     if (!make_map(&ma, d_rows, M, K, kBM) || !make_map(&mb, d_weight, N, K, kBNHalf)) return MIMO_ECUDA;
     const int64_t tiles = ((M + kPairM - 1) / kPairM) * (N / kBN);
-    const size_t smem = static_cast<size_t>(kStages) * kStageBytes + 1024;
+    const size_t smem = static_cast<size_t>(kStages) * kStageBytes + kEpiWarps * kEpiStageBytes + 1024;
     auto kernel = out_dtype == MIMO_BF16 ? patch_embed_kernel<true> : patch_embed_kernel<false>;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess)

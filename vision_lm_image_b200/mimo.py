@@ -38,7 +38,7 @@ EXPORTED = ("mimo_params_default", "mimo_smart_resize", "mimo_num_patches", "mim
             "mimo_preprocess_batch", "mimo_preprocess_batch_ex", "mimo_preprocess_batch_host",
             "mimo_preprocess_batch_host_noalloc", "mimo_expand_prompt_ids", "mimo_video_max_pixels",
             "mimo_smart_nframes", "mimo_sample_frames", "mimo_plan_video", "mimo_preprocess_video",
-            "mimo_patch_embed",
+            "mimo_patch_embed", "mimo_preprocess_embed",
             "mimo_status_string", "mimo_version")
 NOALLOC_STAGING_BYTES = 64 << 20
 
@@ -136,6 +136,9 @@ def lib() -> ctypes.CDLL:
             L.mimo_preprocess_video.restype = ctypes.c_int
             L.mimo_patch_embed.argtypes = [_p, _i64, _p, _i32, _p, _i32, _p, _p, _p]
             L.mimo_patch_embed.restype = ctypes.c_int
+            L.mimo_preprocess_embed.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, ctypes.c_size_t, _p, _p, _p, _p,
+                                                _i32, _p, _i32, _p, _i32, _p, _i64, _p, ctypes.c_size_t, _p, _p]
+            L.mimo_preprocess_embed.restype = ctypes.c_int
             L.mimo_status_string.argtypes = [ctypes.c_int]
             L.mimo_status_string.restype = ctypes.c_char_p
             L.mimo_version.argtypes = []
@@ -501,6 +504,45 @@ def patch_embed(rows, weight, bias=None, out_dtype=None, out=None, error=None, s
         if code != 0:
             raise PatchEmbedError(f"patch_embed kernel stopped waiting on its pipeline (code {code})")
     return out
+
+
+def preprocess_embed(images, weight, bias=None, mean=None, std=None, min_pixels: int | None = None,
+                     max_pixels: int | None = None, out_dtype=None, order: str = "merge", scratch_bytes: int = 96 << 20,
+                     scratch=None, device="cuda", stream=None, check: bool = True):
+    """Pixel path + patch embedding chunk by chunk: returns (embeddings [rows, embed_dim], image_grid_thw)."""
+    import torch
+
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    dev = torch.device(device)
+    if dev.type != "cuda":
+        raise ValueError("the MiMo preprocessing library runs on CUDA devices only")
+    if weight.dtype != torch.bfloat16:
+        raise ValueError("weight must be bfloat16")
+    params = make_params(mean, std, min_pixels, max_pixels)
+    packed = pack_images(images, device=dev) if not isinstance(images, PackedBatch) else images
+    grid, offs = plan_batch(packed.heights, packed.widths, params)
+    total = int(offs[-1])
+    N = weight.shape[0]
+    out = torch.empty((total, N), dtype=out_dtype, device=dev)
+    if scratch is None:
+        scratch = torch.empty(scratch_bytes, dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    order_code = {"merge": ORDER_MERGE, "column": ORDER_COLUMN}[order]
+    _check(lib().mimo_preprocess_embed(ctypes.byref(params), packed.n, ctypes.c_void_p(packed.buffer.data_ptr()),
+                                       packed.buffer.numel(), packed.offsets.ctypes.data, packed.heights.ctypes.data,
+                                       packed.widths.ctypes.data, packed.channels.ctypes.data, order_code,
+                                       ctypes.c_void_p(weight.data_ptr()), N,
+                                       ctypes.c_void_p(bias.data_ptr() if bias is not None else 0),
+                                       _dtype_code(out_dtype), ctypes.c_void_p(out.data_ptr()), total,
+                                       ctypes.c_void_p(scratch.data_ptr()), scratch.numel(),
+                                       ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, dev)),
+           "preprocess_embed")
+    if check:
+        (torch.cuda.current_stream(dev) if stream is None else stream).synchronize()
+        code = int(err.item())
+        if code != 0:
+            raise PatchEmbedError(f"patch_embed kernel stopped waiting on its pipeline (code {code})")
+    return out, torch.from_numpy(grid)
 
 
 # ----------------------------------------------------------------- host-to-host path
