@@ -546,7 +546,7 @@ __device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &
 // shared memory and those of block k+2 are in flight (cp.async), and warps
 // 0-1 compute the taps of the block after.
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads, 6) preprocess_kernel(const __grid_constant__ LaunchParams P) {
+__global__ void __launch_bounds__(kThreads, 5) preprocess_kernel(const __grid_constant__ LaunchParams P) {
     extern __shared__ float4 smem4[];
     float *const tile = reinterpret_cast<float *>(smem4);  // [3][rows][stride] | raw bytes
     uint8_t *const raw = reinterpret_cast<uint8_t *>(tile + P.raw);
