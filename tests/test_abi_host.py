@@ -108,6 +108,13 @@ def test_plan_batch_errors():
     assert e.value.status == 5
     g, o = mimo.plan_batch([], [])
     assert g.shape == (0, 3) and list(o) == [0]
+    # a sub-factor sliver upscaled past 2^30 columns (only reachable with a huge max_pixels)
+    big = mimo.make_params(max_pixels=1 << 36)
+    assert oracle.smart_resize(16, (1 << 29) + 1000, 32, 8192, 1 << 36)[1] >= 1 << 30
+    with pytest.raises(mimo.MimoError) as e:
+        mimo.plan_batch([16], [(1 << 29) + 1000], big)
+    assert e.value.status == 8
+    assert mimo.plan_batch([16], [(1 << 28)], big)[0][0, 2] == (1 << 29) // 16
 
 
 # Validation-only calls: every call below must fail before launching. They are

@@ -109,7 +109,9 @@ int plan_image(int64_t H, int64_t W, const mimo_params *p, ImagePlan *ip) {
     int64_t Hr = 0, Wr = 0;
     const int st = smart_resize_impl(H, W, kFactor, p->min_pixels, p->max_pixels, &Hr, &Wr);
     if (st != MIMO_OK) return st;
-    if (Hr > INT32_MAX || Wr > INT32_MAX) return MIMO_EOVERFLOW;
+    // the kernel's tap arithmetic keeps 2 * (resized side) in 32 bits; a side of
+    // 2^30 would mean hundreds of GB of rows anyway
+    if (Hr >= (int64_t(1) << 30) || Wr >= (int64_t(1) << 30)) return MIMO_EOVERFLOW;
     ip->Hr = Hr;
     ip->Wr = Wr;
     ip->rows = (Hr / 16) * (Wr / 16);

@@ -101,8 +101,9 @@ struct TapSet {
 struct AxisCursor {
     int blk = -2, ii = 0, t = 0, bh = 0, bw = 0, tt = 0;  // position of the last block handled
     int img = -1, b = -2;
-    int64_t q = 0, r = 0;
-    int64_t den = 1, step_q = 0, step_r = 0;
+    // q <= in and r < den = 2 * out: both fit 32 bits (only the first numerator needs 64)
+    int32_t q = 0, r = 0;
+    int32_t den = 1, step_q = 0, step_r = 0;
     double inv_den = 1.0;
     float inv_den_f = 1.0f;
 };
@@ -198,12 +199,13 @@ __device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, c
         if (ii != cur.img) {
             cur.img = ii;
             cur.b = -2;
-            cur.den = 2 * out;
+            cur.den = static_cast<int32_t>(2 * out);
             cur.inv_den = 1.0 / static_cast<double>(cur.den);
             cur.inv_den_f = static_cast<float>(cur.inv_den);
             const int64_t step = 2 * kBlock * in;  // numerator change between blocks
-            cur.step_q = step / cur.den;
-            cur.step_r = step - cur.step_q * cur.den;
+            const int64_t sq = step / cur.den;
+            cur.step_q = static_cast<int32_t>(sq);
+            cur.step_r = static_cast<int32_t>(step - sq * cur.den);
         }
         if (b == cur.b + 1) {
             cur.q += cur.step_q;
@@ -227,8 +229,8 @@ __device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, c
                 ++q;
                 r -= cur.den;
             }
-            cur.q = q;
-            cur.r = r;
+            cur.q = static_cast<int32_t>(q);
+            cur.r = static_cast<int32_t>(r);
         }
         cur.b = b;
         // source coordinate clamped at 0: negative quotient -> first pixel, weight 0
@@ -236,7 +238,7 @@ __device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, c
         const int32_t i0 = clamp ? 0 : static_cast<int32_t>(cur.q);
         const int32_t i1 = (static_cast<int64_t>(i0) + 1 < in) ? i0 + 1 : static_cast<int32_t>(in - 1);
         // r < den; below 2^23 the float conversion is exact with the 2^23 bit trick
-        const float rf = (cur.r < (int64_t(1) << 23))
+        const float rf = (cur.r < (1 << 23))
                              ? __uint_as_float(0x4B000000u | static_cast<uint32_t>(cur.r)) - kTwo23
                              : static_cast<float>(cur.r);
         const float lam = clamp ? 0.0f : rf * cur.inv_den_f;
@@ -589,20 +591,44 @@ __global__ void __launch_bounds__(kThreads, 5) preprocess_kernel(const __grid_co
     }
 }
 
+// Launch setup that depends only on the device and the shared-memory size,
+// kept per host thread so that small batches do not pay the driver queries on
+// every call.
+struct LaunchSetup {
+    int dev = -1, sms = 0;
+    size_t attr_smem = 0;        // largest dynamic size opted in so far on this device
+    size_t occ_smem = ~size_t(0);  // shared-memory size the resident count below is for
+    int per_sm = 0;
+};
+
 template <bool kBF16>
 int launch_typed(const LaunchParams &lp, int64_t blocks, size_t smem_bytes, cudaStream_t stream) {
     auto kern = preprocess_kernel<kBF16>;
+    static thread_local LaunchSetup setup;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ECUDA;
+    if (dev != setup.dev) {
+        setup = LaunchSetup();
+        if (cudaDeviceGetAttribute(&setup.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MIMO_ECUDA;
+        setup.dev = dev;
+    }
     // the opt-in covers dynamic + static shared memory above the 48 KB default
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes)) !=
-        cudaSuccess)
-        return MIMO_ECUDA;
+    if (smem_bytes > setup.attr_smem) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes)) !=
+            cudaSuccess)
+            return MIMO_ECUDA;
+        setup.attr_smem = smem_bytes;
+    }
     // persistent grid: as many CTAs as can be resident at once
-    int dev = 0, sms = 0, per_sm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem_bytes) != cudaSuccess ||
-        per_sm <= 0)
-        return MIMO_ECUDA;
+    if (smem_bytes != setup.occ_smem) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem_bytes) != cudaSuccess ||
+            per_sm <= 0)
+            return MIMO_ECUDA;
+        setup.per_sm = per_sm;
+        setup.occ_smem = smem_bytes;
+    }
+    const int sms = setup.sms, per_sm = setup.per_sm;
     const int64_t grid = std::min<int64_t>(blocks, static_cast<int64_t>(sms) * per_sm);
     kern<<<static_cast<unsigned>(grid), kThreads, smem_bytes, stream>>>(lp);
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
