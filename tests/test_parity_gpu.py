@@ -120,6 +120,29 @@ def test_c5_full_size_sampled():
     assert_fp32_close(got, want, "samples")
 
 
+def test_c5_full_size_bf16_sampled():
+    """The bf16 launch of the full batch (as `bench.py --dtype bf16` times it): sampled values within one
+    bf16 ulp of the oracle, the permutation bit-exact, both frames identical."""
+    w = workloads.workload("c5")
+    imgs = w["images"]
+    pv, grid, perm = gpu_run(imgs, w["mean"], w["std"], dtype=torch.bfloat16, column_perm=True)
+    assert pv.shape == (256 * 8160, 1536) and pv.dtype == torch.bfloat16
+    rperm = np.concatenate([oracle.column_permutation(68, 120, 2, 8160 * i) for i in range(256)])
+    assert np.array_equal(perm.cpu().numpy(), rperm)
+    v = pv.view(-1, 3, 2, 256)
+    assert torch.equal(v[:, :, 0], v[:, :, 1])
+    rng = np.random.Generator(np.random.PCG64(56))
+    n = 3000
+    img_idx = rng.integers(0, 256, n)
+    rows = rng.integers(0, 8160, n)
+    cols = rng.integers(0, 1536, n)
+    flat = (torch.from_numpy(img_idx * 8160 + rows) * 1536 + torch.from_numpy(cols)).cuda()
+    got = pv.view(-1).index_select(0, flat)
+    want = np.array([oracle.patch_value(imgs[i], (1088, 1920), int(r), int(c), w["mean"], w["std"])
+                     for i, r, c in zip(img_idx, rows, cols)], np.float32)
+    assert_bf16_close(got, want, "bf16 samples")
+
+
 def test_c5_bf16_subset():
     w = workloads.workload("c5", n_images=6)
     pv, grid, perm = gpu_run(w["images"], w["mean"], w["std"], dtype=torch.bfloat16, column_perm=True)
@@ -373,6 +396,23 @@ def test_preprocess_then_patch_embed_chain():
     g_out = out.float().cpu().numpy().astype(np.float64)
     tol = tol_rows + 1e-5 * scale + 2.0 ** -8 * np.abs(ref) + 1e-6
     assert (np.abs(g_out - ref) <= tol).all(), np.abs(g_out - ref).max()
+
+
+def test_patch_embed_full_bench_size_sampled():
+    # the launch `bench.py --workload pe` times: 2,088,960 rows, embed_dim 1280, ~551 tiles per CTA pair,
+    # so every stage and accumulator phase bit wraps hundreds of times; sampled rows against the oracle
+    M, N = 256 * 8160, 1280
+    g = torch.Generator(device="cuda").manual_seed(11)
+    rows = torch.randn((M, 1536), generator=g, device="cuda").to(torch.bfloat16)
+    w = (torch.randn((N, 1536), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g, device="cuda")
+    out = mimo.patch_embed(rows, w, bias)
+    rng = np.random.Generator(np.random.PCG64(12))
+    pick = np.unique(np.concatenate([[0, 255, 256, M - 256, M - 1], rng.integers(0, M, 120)]))
+    idx = torch.from_numpy(pick).cuda()
+    ref, scale = _embed_ref(rows.index_select(0, idx), w, bias)
+    _assert_embed_close(out.index_select(0, idx), ref, scale, "full-size sample")
+    del rows, out
 
 
 @pytest.mark.parametrize("order", ["merge", "column"])
