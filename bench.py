@@ -195,10 +195,53 @@ def host_cores() -> int:
         return os.cpu_count() or 1
 
 
+def run_reference_other(args, world):
+    """The oracle on the video clip (frames/s) or on the patch embedding (tokens/s)."""
+    import numpy as np
+
+    import oracle
+    import workloads
+
+    oracle.build()
+    cores = host_cores()
+    if args.workload == "v1":
+        # a bounded sample: the first 4 frames of the clip (two temporal patches) per step
+        w = workloads.video_workload("v1", n_frames=4)
+        run = lambda: oracle.preprocess_video(w["frames"], w["mean"], w["std"], total_max_pixels=w["total_max_pixels"])
+        units, unit, sample = 4, "frames/s", "first 4 frames of the 64-frame clip per step, oracle on 1 thread"
+        metric = METRIC + " (video frames)"
+    else:
+        # a bounded sample: 256 rows of the embedding per step, fp64 on one thread
+        rng = np.random.Generator(np.random.PCG64(17))
+        a = rng.standard_normal((256, 1536)).astype(np.float32)
+        wt = (rng.standard_normal((args.embed_dim, 1536)) * 0.02).astype(np.float32)
+        run = lambda: oracle.patch_embed(a, wt)
+        units, unit, sample = 256, "tokens/s", "256 rows x 1536 -> embed_dim per step, fp64 on 1 thread"
+        metric = "patch-embedding tokens/s (Conv3d 3x2x16x16 -> embed_dim as a bf16 GEMM)"
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    t = time.perf_counter() - t0
+    value = units * args.steps / t
+    print(json.dumps({
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def run_reference(args, rank, world):
     import workloads
 
     if rank != 0:
+        return
+    if args.workload in ("v1", "pe"):
+        run_reference_other(args, world)
         return
     w = workloads.workload(args.workload, n_images=args.images)
     if args.dtype:
