@@ -415,11 +415,14 @@ def run_patch_embed(args, rank, world, local_rank):
         sample = 256
         a = rows[:sample].float().cpu().numpy()
         wt = weight.float().cpu().numpy()
-        t0 = time.perf_counter()
-        oracle.patch_embed(a, wt, bias.cpu().numpy())
+        bb = bias.cpu().numpy()
+        done, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < 10.0:
+            oracle.patch_embed(a, wt, bb)
+            done += sample
         dt = time.perf_counter() - t0
-        cpu = {"value": sample / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"first {sample} of {M} rows, one pass, {dt:.1f} s, single thread"}
+        cpu = {"value": done / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"first {sample} of {M} rows, passes repeated for {dt:.1f} s, single thread"}
     if rank == 0:
         print(json.dumps({
             "metric": "patch-embedding tokens/s (Conv3d 3x2x16x16 -> embed_dim as a bf16 GEMM)",
