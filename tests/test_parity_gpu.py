@@ -7,6 +7,8 @@ Bars (from the method's definition and the arithmetic of both sides):
   smaller than 2**-19 (below |v| ~ 2**-12 the fp32 rounding noise of the GPU arithmetic, ~1e-6, is
   larger than a bf16 ulp and may move the rounding by more than one step).
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -296,6 +298,66 @@ def test_column_order_and_tables_match_oracle(dtype):
             assert_fp32_close(pv.cpu().numpy(), ref, order)
         else:
             assert_bf16_close(pv, ref, order)
+
+
+def _kept_width_batch(shapes, seed):
+    rng = workloads.rng_for(seed)
+    imgs = [workloads.rgba_image(rng, h, w) if c == 4 else workloads.uniform_image(rng, h, w, 3) for h, w, c in shapes]
+    for h, w, _ in shapes:
+        assert oracle.smart_resize(h, w)[1] == w  # every width kept: the unstaged kernel takes the launch
+    return imgs
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_kept_width_launches_match_oracle(dtype):
+    # bf16 takes the unstaged kernel for any heights; fp32 only when every height is kept as well
+    shapes = [(1079, 1920, 4), (1088, 640, 3), (97, 352, 4), (64, 160, 3), (720, 1280, 3), (1000, 96, 4)]
+    if dtype == torch.float32:
+        shapes = [(1088, 640, 3), (64, 160, 4), (704, 1280, 3), (96, 352, 4)]
+    imgs = _kept_width_batch(shapes, 909)
+    mean, std = workloads.CLIP_MEAN, workloads.CLIP_STD
+    for order in ("merge", "column"):
+        pv, grid, perm, pos, win = mimo.preprocess(imgs, mean, std, dtype=dtype, column_perm=True, order=order,
+                                                   positions=True, window_index=True)
+        torch.cuda.synchronize()
+        ref, rgrid, rperm, rpos, rwin = oracle.preprocess(imgs, mean, std, column_perm=True, order=order,
+                                                          positions=True, window=True, threads=8)
+        assert np.array_equal(grid.numpy(), rgrid)
+        assert np.array_equal(perm.cpu().numpy(), rperm)
+        assert np.array_equal(pos.cpu().numpy(), rpos)
+        assert np.array_equal(win.cpu().numpy(), rwin)
+        if dtype == torch.float32:
+            assert_fp32_close(pv.cpu().numpy(), ref, order)
+        else:
+            assert_bf16_close(pv, ref, order)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_kept_width_image_ending_at_the_buffer_end(dtype):
+    # an RGB image whose last row ends exactly at the end of the buffer the caller declares: the
+    # unstaged kernel's 16-byte word loads past it must read nothing there
+    h, w = 96, 352
+    img = _kept_width_batch([(h, w, 3)], 910)[0]
+    nbytes = h * w * 3
+    dev_buf = torch.zeros(nbytes + 4096, dtype=torch.uint8, device="cuda")
+    dev_buf[:nbytes] = torch.from_numpy(img.reshape(-1)).cuda()
+    dev_buf[nbytes:] = 255  # bytes beyond the declared end: never used
+    params = mimo.make_params()
+    rows = (h // 16) * (w // 16)
+    out = torch.empty((rows, 1536), dtype=dtype, device="cuda")
+    offs = np.zeros(1, np.int64)
+    hh, ww, cc = (np.array([v], np.int32) for v in (h, w, 3))
+    st = mimo.lib().mimo_preprocess_batch(ctypes.byref(params), 1, ctypes.c_void_p(dev_buf.data_ptr()), nbytes,
+                                          offs.ctypes.data, hh.ctypes.data, ww.ctypes.data, cc.ctypes.data,
+                                          1 if dtype == torch.bfloat16 else 0, ctypes.c_void_p(out.data_ptr()), rows,
+                                          None, None)
+    assert st == 0
+    torch.cuda.synchronize()
+    ref, _ = oracle.preprocess_image(img, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    if dtype == torch.float32:
+        assert_fp32_close(out.cpu().numpy(), ref, "buffer end")
+    else:
+        assert_bf16_close(out, ref, "buffer end")
 
 
 def test_column_order_is_a_row_gather_full_c5():

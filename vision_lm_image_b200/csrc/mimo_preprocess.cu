@@ -18,6 +18,8 @@
 //     page, column_permutation).
 // CTAs are persistent: each takes a contiguous range of blocks and overlaps
 // the source copies of the next blocks with the stores of the current one.
+// Launches whose images all keep their width go to a second, unstaged kernel
+// (direct_kernel below) when that measured faster.
 // There is no inter-CTA communication, no atomics and no global wait; every
 // output element has exactly one writer.
 #include <cuda_bf16.h>
@@ -591,6 +593,199 @@ __global__ void __launch_bounds__(kThreads, 5) preprocess_kernel(const __grid_co
     }
 }
 
+// ---------------------------------------------------------------------------
+// Direct kernel, for launches whose images all keep their width (Wr == W, no
+// video halves). Every output column then samples its own source column, and
+// a block needs no staging. Each thread owns the same 4 pixels x 3 channels of
+// one output row in every block, as in the staged kernel's vertical pass. It
+// reads its one or two source rows straight from global memory (the ~2x reuse
+// between neighbouring output rows hits L1), converts the bytes with the
+// staged kernel's arithmetic, and then interpolates, normalises and stores
+// identically. There is no shared memory and no barrier. The row taps come
+// from the exact quotient, once per block row, and stay in registers.
+// ---------------------------------------------------------------------------
+
+// 16 source bytes from the 4-byte aligned image offset `oa`, zero past the
+// caller's buffer end (the bytes a pixel uses never lie there).
+__device__ __forceinline__ void load_words(const uint8_t *img, int64_t oa, int64_t limit, uint32_t (&w)[4]) {
+    const uint32_t *p = reinterpret_cast<const uint32_t *>(img + oa);
+    if (oa + 16 <= limit) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w[k] = __ldg(p + k);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w[k] = (oa + 4 * k + 4 <= limit) ? __ldg(p + k) : 0u;
+    }
+}
+
+// 4 consecutive pixels of one source row, from the words above, as planar
+// floats on 0..255 (RGBA composited onto white): finish_stage's arithmetic.
+__device__ __forceinline__ void convert4(const uint32_t (&w)[4], int C, uint32_t sh, float4 (&v)[3]) {
+    const float2 m23 = f2(-kTwo23, -kTwo23);
+    float2 R0, R1, G0, G1, B0, B1;
+    if (C == 4) {
+        const float2 A01 = add2(f2(byte_bits<3>(w[0]), byte_bits<3>(w[1])), m23);
+        const float2 A23 = add2(f2(byte_bits<3>(w[2]), byte_bits<3>(w[3])), m23);
+        const float2 wh01 = fma2(A01, f2(-255.0f, -255.0f), f2(65025.0f, 65025.0f));
+        const float2 wh23 = fma2(A23, f2(-255.0f, -255.0f), f2(65025.0f, 65025.0f));
+        R0 = on_white2(add2(f2(byte_bits<0>(w[0]), byte_bits<0>(w[1])), m23), A01, wh01);
+        R1 = on_white2(add2(f2(byte_bits<0>(w[2]), byte_bits<0>(w[3])), m23), A23, wh23);
+        G0 = on_white2(add2(f2(byte_bits<1>(w[0]), byte_bits<1>(w[1])), m23), A01, wh01);
+        G1 = on_white2(add2(f2(byte_bits<1>(w[2]), byte_bits<1>(w[3])), m23), A23, wh23);
+        B0 = on_white2(add2(f2(byte_bits<2>(w[0]), byte_bits<2>(w[1])), m23), A01, wh01);
+        B1 = on_white2(add2(f2(byte_bits<2>(w[2]), byte_bits<2>(w[3])), m23), A23, wh23);
+    } else {
+        // 12 bytes from the shift, realigned as in finish_stage
+        const uint32_t r0 = __funnelshift_r(w[0], w[1], sh);
+        const uint32_t r1 = __funnelshift_r(w[1], w[2], sh);
+        const uint32_t r2 = __funnelshift_r(w[2], w[3], sh);
+        R0 = add2(f2(byte_bits<0>(r0), byte_bits<3>(r0)), m23);
+        R1 = add2(f2(byte_bits<2>(r1), byte_bits<1>(r2)), m23);
+        G0 = add2(f2(byte_bits<1>(r0), byte_bits<0>(r1)), m23);
+        G1 = add2(f2(byte_bits<3>(r1), byte_bits<2>(r2)), m23);
+        B0 = add2(f2(byte_bits<2>(r0), byte_bits<1>(r1)), m23);
+        B1 = add2(f2(byte_bits<0>(r2), byte_bits<3>(r2)), m23);
+    }
+    v[0] = make_float4(R0.x, R0.y, R1.x, R1.y);
+    v[1] = make_float4(G0.x, G0.y, G1.x, G1.y);
+    v[2] = make_float4(B0.x, B0.y, B1.x, B1.y);
+}
+
+template <bool kBF16>
+__global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_constant__ LaunchParams P) {
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int64_t B = P.block_start[P.n];
+    const int begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * B / gridDim.x);
+    const int end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * B / gridDim.x);
+    if (begin >= end) return;
+
+    // this thread's place in every block (the staged kernel's vertical-pass mapping)
+    const int mh = warp >> 2;
+    const int py = ((warp & 3) << 2) | (lane >> 3);
+    const int mw = (lane >> 2) & 1;
+    const int q = lane & 3;
+    const int dy = (mh << 4) | py;
+    const int dx0 = (mw << 4) | (q << 2);
+    const int col = py * 16 + q * 4;
+
+    // position of the first block; later blocks advance one column at a time
+    int ii = find_image(P, begin);
+    int bh, bw;
+    {
+        const ImageDesc &D = P.img[ii];
+        const int g = D.Wr / kBlock;
+        const int local = begin - P.block_start[ii];
+        bh = local / g;
+        bw = local - bh * g;
+    }
+    int tap_ii = -1, tap_bh = -1;
+    int32_t sy0 = 0, sy1 = 0;
+    float ly = 0.0f;
+    for (int blk = begin; blk < end; ++blk) {
+        const ImageDesc &D = P.img[ii];
+        const int32_t H = D.H, W = D.W, Hr = D.Hr, flags = D.flags;
+        const int C = (flags >> kChannelShift) & 0xFF;
+        const bool yident = (flags & kIdentityRows) != 0;
+        if (ii != tap_ii || bh != tap_bh) {
+            // exact taps of output row Y: i0 = floor(((2Y+1)*H - Hr) / (2*Hr)) clamped at 0,
+            // i1 = min(i0+1, H-1), weight = remainder / (2*Hr); compute_taps reaches the same
+            // quotient incrementally
+            const int64_t den = 2 * static_cast<int64_t>(Hr);
+            const double inv_den = 1.0 / static_cast<double>(den);
+            const int64_t Y = static_cast<int64_t>(bh) * kBlock + dy;
+            const int64_t num = (2 * Y + 1) * H - Hr;
+            int64_t qq = static_cast<int64_t>(floor(static_cast<double>(num) * inv_den));
+            int64_t r = num - qq * den;
+            while (r < 0) {
+                --qq;
+                r += den;
+            }
+            while (r >= den) {
+                ++qq;
+                r -= den;
+            }
+            const bool clamp = qq < 0;
+            sy0 = clamp ? 0 : static_cast<int32_t>(qq);
+            sy1 = (static_cast<int64_t>(sy0) + 1 < H) ? sy0 + 1 : H - 1;
+            ly = clamp ? 0.0f : static_cast<float>(r) * static_cast<float>(inv_den);
+            tap_ii = ii;
+            tap_bh = bh;
+        }
+        const uint8_t *img = P.src + D.src_off;
+        const int64_t x = static_cast<int64_t>(bw) * kBlock + dx0;
+        const int64_t oA = (static_cast<int64_t>(sy0) * W + x) * C;
+        uint32_t wa[4], wb[4];
+        load_words(img, oA & ~int64_t(3), D.limit, wa);
+        float4 va[3], vb[3];
+        if (!yident) {
+            const int64_t oB = (static_cast<int64_t>(sy1) * W + x) * C;
+            load_words(img, oB & ~int64_t(3), D.limit, wb);
+            convert4(wb, C, static_cast<uint32_t>(oB & 3) * 8u, vb);
+        }
+        convert4(wa, C, static_cast<uint32_t>(oA & 3) * 8u, va);
+
+        // merge order lists units by (block row, block col), column order by (block col, block row)
+        const int gw2 = D.Wr / kBlock, gh2 = Hr / kBlock;
+        const int64_t unit = P.order ? static_cast<int64_t>(bw) * gh2 + bh : static_cast<int64_t>(bh) * gw2 + bw;
+        const int64_t row = D.row0 + 4 * unit + (mh * 2 + mw);
+        const float2 ly2 = f2(ly, ly), nly2 = f2(-ly, -ly);
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+            float2 v01 = f2(va[c].x, va[c].y), v23 = f2(va[c].z, va[c].w);
+            if (!yident) {
+                v01 = fma2(ly2, f2(vb[c].x, vb[c].y), fma2(nly2, v01, v01));
+                v23 = fma2(ly2, f2(vb[c].z, vb[c].w), fma2(nly2, v23, v23));
+            }
+            const float2 k2 = f2(P.k[c], P.k[c]), b2 = f2(P.b[c], P.b[c]);
+            const float2 n01 = fma2(v01, k2, b2);
+            const float2 n23 = fma2(v23, k2, b2);
+            // an image fills both temporal slots with its one frame
+            if constexpr (!kBF16) {
+                float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col;
+                const float4 f4 = make_float4(n01.x, n01.y, n23.x, n23.y);
+                __stcs(reinterpret_cast<float4 *>(o), f4);
+                __stcs(reinterpret_cast<float4 *>(o + 256), f4);
+            } else {
+                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col;
+                const __nv_bfloat162 lo2 = __floats2bfloat162_rn(n01.x, n01.y);
+                const __nv_bfloat162 hi2 = __floats2bfloat162_rn(n23.x, n23.y);
+                uint2 u;
+                u.x = *reinterpret_cast<const uint32_t *>(&lo2);
+                u.y = *reinterpret_cast<const uint32_t *>(&hi2);
+                __stcs(reinterpret_cast<uint2 *>(o), u);
+                __stcs(reinterpret_cast<uint2 *>(o + 256), u);
+            }
+        }
+        // the merge unit's table entries: permutation (thread 0), rotary positions (thread 1),
+        // window index (thread 2), as in emit_block
+        if (tid < 3) {
+            const int64_t src_unit = static_cast<int64_t>(bh) * gw2 + bw;  // merge order
+            const int64_t dst_unit = static_cast<int64_t>(bw) * gh2 + bh;  // column order
+            if (tid == 0 && P.perm != nullptr) {
+                const int32_t s0 = static_cast<int32_t>(D.row0 + 4 * src_unit);
+                __stcs(reinterpret_cast<int4 *>(P.perm + D.row0 + 4 * dst_unit), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
+            } else if (tid == 1 && P.pos != nullptr) {
+                const int32_t h = 2 * bh, w = 2 * bw;
+                int4 *d = reinterpret_cast<int4 *>(P.pos + 2 * (D.row0 + 4 * unit));
+                __stcs(d, make_int4(h, w, h, w + 1));
+                __stcs(d + 1, make_int4(h + 1, w, h + 1, w + 1));
+            } else if (tid == 2 && P.win != nullptr) {
+                const int64_t u0 = D.row0 / 4;
+                P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
+            }
+        }
+        // next block: one column on, then the next block row, then the next image
+        if (++bw == gw2) {
+            bw = 0;
+            if (++bh == gh2) {
+                bh = 0;
+                ++ii;
+            }
+        }
+    }
+}
+
 // Launch setup that depends only on the device and the shared-memory size,
 // kept per host thread so that small batches do not pay the driver queries on
 // every call.
@@ -634,12 +829,42 @@ int launch_typed(const LaunchParams &lp, int64_t blocks, size_t smem_bytes, cuda
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
 }
 
+template <bool kBF16>
+int launch_direct(const LaunchParams &lp, int64_t blocks, cudaStream_t stream) {
+    auto kern = direct_kernel<kBF16>;
+    static thread_local LaunchSetup setup;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ECUDA;
+    if (dev != setup.dev) {
+        setup = LaunchSetup();
+        int per_sm = 0;
+        if (cudaDeviceGetAttribute(&setup.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess || per_sm <= 0)
+            return MIMO_ECUDA;
+        setup.per_sm = per_sm;
+        setup.dev = dev;
+    }
+    // persistent grid, as the staged kernel's
+    const int64_t grid = std::min<int64_t>(blocks, static_cast<int64_t>(setup.sms) * setup.per_sm);
+    kern<<<static_cast<unsigned>(grid), kThreads, 0, stream>>>(lp);
+    return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
+}
+
 }  // namespace
 
 int launch_preprocess(const LaunchParams &lp, int64_t blocks, int out_dtype, size_t smem_bytes, void *stream) {
     if (blocks <= 0) return MIMO_OK;
     if (blocks > static_cast<int64_t>(INT32_MAX)) return MIMO_EOVERFLOW;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // every width kept, no video halves: the direct kernel, unless fp32 rows are written for resized
+    // heights (there the staged kernel's burst reads keep the write stream faster, as measured)
+    bool widths_kept = true, heights_kept = true;
+    for (int i = 0; i < lp.n; ++i) {
+        widths_kept = widths_kept && (lp.img[i].flags & kIdentityCols) != 0 && (lp.img[i].flags & kVideo) == 0;
+        heights_kept = heights_kept && (lp.img[i].flags & kIdentityRows) != 0;
+    }
+    if (widths_kept && (out_dtype == MIMO_BF16 || heights_kept))
+        return out_dtype == MIMO_BF16 ? launch_direct<true>(lp, blocks, s) : launch_direct<false>(lp, blocks, s);
     return out_dtype == MIMO_BF16 ? launch_typed<true>(lp, blocks, smem_bytes, s)
                                   : launch_typed<false>(lp, blocks, smem_bytes, s);
 }
