@@ -602,25 +602,34 @@ __global__ void __launch_bounds__(kThreads, 5) preprocess_kernel(const __grid_co
 // between neighbouring output rows hits L1), converts the bytes with the
 // staged kernel's arithmetic, and then interpolates, normalises and stores
 // identically. There is no shared memory and no barrier. The row taps come
-// from the exact quotient, once per block row, and stay in registers.
+// from the exact quotient, once per block row, and stay in registers. Each
+// row quad is one 16-byte load (RGBA) or three 4-byte loads (RGB).
 // ---------------------------------------------------------------------------
 
-// 16 source bytes from the 4-byte aligned image offset `oa`, zero past the
-// caller's buffer end (the bytes a pixel uses never lie there).
-__device__ __forceinline__ void load_words(const uint8_t *img, int64_t oa, int64_t limit, uint32_t (&w)[4]) {
-    const uint32_t *p = reinterpret_cast<const uint32_t *>(img + oa);
-    if (oa + 16 <= limit) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) w[k] = __ldg(p + k);
+// The 4-pixel quad a thread reads from one source row. Every width on this
+// path is a multiple of 32 (Wr == W) and a thread's first column a multiple of
+// 4, so an RGB quad (12 bytes) starts 4-byte aligned and an RGBA quad (16
+// bytes) 16-byte aligned, both wholly inside the image (image offsets are
+// 16-byte aligned).
+__device__ __forceinline__ void load_quad(const uint8_t *p, int C, uint32_t (&w)[4]) {
+    if (C == 4) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p));
+        w[0] = v.x;
+        w[1] = v.y;
+        w[2] = v.z;
+        w[3] = v.w;
     } else {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) w[k] = (oa + 4 * k + 4 <= limit) ? __ldg(p + k) : 0u;
+        const uint32_t *q = reinterpret_cast<const uint32_t *>(p);
+        w[0] = __ldg(q);
+        w[1] = __ldg(q + 1);
+        w[2] = __ldg(q + 2);
+        w[3] = 0u;
     }
 }
 
-// 4 consecutive pixels of one source row, from the words above, as planar
-// floats on 0..255 (RGBA composited onto white): finish_stage's arithmetic.
-__device__ __forceinline__ void convert4(const uint32_t (&w)[4], int C, uint32_t sh, float4 (&v)[3]) {
+// The quad as planar floats on 0..255 (RGBA composited onto white), with
+// finish_stage's arithmetic.
+__device__ __forceinline__ void convert4(const uint32_t (&w)[4], int C, float4 (&v)[3]) {
     const float2 m23 = f2(-kTwo23, -kTwo23);
     float2 R0, R1, G0, G1, B0, B1;
     if (C == 4) {
@@ -635,16 +644,13 @@ __device__ __forceinline__ void convert4(const uint32_t (&w)[4], int C, uint32_t
         B0 = on_white2(add2(f2(byte_bits<2>(w[0]), byte_bits<2>(w[1])), m23), A01, wh01);
         B1 = on_white2(add2(f2(byte_bits<2>(w[2]), byte_bits<2>(w[3])), m23), A23, wh23);
     } else {
-        // 12 bytes from the shift, realigned as in finish_stage
-        const uint32_t r0 = __funnelshift_r(w[0], w[1], sh);
-        const uint32_t r1 = __funnelshift_r(w[1], w[2], sh);
-        const uint32_t r2 = __funnelshift_r(w[2], w[3], sh);
-        R0 = add2(f2(byte_bits<0>(r0), byte_bits<3>(r0)), m23);
-        R1 = add2(f2(byte_bits<2>(r1), byte_bits<1>(r2)), m23);
-        G0 = add2(f2(byte_bits<1>(r0), byte_bits<0>(r1)), m23);
-        G1 = add2(f2(byte_bits<3>(r1), byte_bits<2>(r2)), m23);
-        B0 = add2(f2(byte_bits<2>(r0), byte_bits<1>(r1)), m23);
-        B1 = add2(f2(byte_bits<0>(r2), byte_bits<3>(r2)), m23);
+        // bytes: w0 = R0 G0 B0 R1 | w1 = G1 B1 R2 G2 | w2 = B2 R3 G3 B3
+        R0 = add2(f2(byte_bits<0>(w[0]), byte_bits<3>(w[0])), m23);
+        R1 = add2(f2(byte_bits<2>(w[1]), byte_bits<1>(w[2])), m23);
+        G0 = add2(f2(byte_bits<1>(w[0]), byte_bits<0>(w[1])), m23);
+        G1 = add2(f2(byte_bits<3>(w[1]), byte_bits<2>(w[2])), m23);
+        B0 = add2(f2(byte_bits<2>(w[0]), byte_bits<1>(w[1])), m23);
+        B1 = add2(f2(byte_bits<0>(w[2]), byte_bits<3>(w[2])), m23);
     }
     v[0] = make_float4(R0.x, R0.y, R1.x, R1.y);
     v[1] = make_float4(G0.x, G0.y, G1.x, G1.y);
@@ -714,16 +720,14 @@ __global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_consta
         }
         const uint8_t *img = P.src + D.src_off;
         const int64_t x = static_cast<int64_t>(bw) * kBlock + dx0;
-        const int64_t oA = (static_cast<int64_t>(sy0) * W + x) * C;
         uint32_t wa[4], wb[4];
-        load_words(img, oA & ~int64_t(3), D.limit, wa);
         float4 va[3], vb[3];
+        load_quad(img + (static_cast<int64_t>(sy0) * W + x) * C, C, wa);
         if (!yident) {
-            const int64_t oB = (static_cast<int64_t>(sy1) * W + x) * C;
-            load_words(img, oB & ~int64_t(3), D.limit, wb);
-            convert4(wb, C, static_cast<uint32_t>(oB & 3) * 8u, vb);
+            load_quad(img + (static_cast<int64_t>(sy1) * W + x) * C, C, wb);
+            convert4(wb, C, vb);
         }
-        convert4(wa, C, static_cast<uint32_t>(oA & 3) * 8u, va);
+        convert4(wa, C, va);
 
         // merge order lists units by (block row, block col), column order by (block col, block row)
         const int gw2 = D.Wr / kBlock, gh2 = Hr / kBlock;
