@@ -49,8 +49,10 @@ static_assert(sizeof(ImageDesc) == 56, "descriptor layout");
 
 // Everything one launch needs travels by value as the kernel's parameter
 // block (__grid_constant__), so a launch needs no device-side table and no
-// host-to-device copy.
-struct LaunchParams {
+// host-to-device copy. The block is sized for kCap images: the driver copies
+// all of it on every launch, so launches of a few images use a small one.
+template <int kCap>
+struct LaunchParamsT {
     const uint8_t *src;
     void *out;
     int32_t *perm;       // may be null
@@ -64,9 +66,12 @@ struct LaunchParams {
     int32_t tile_stride; // row stride (floats, multiple of 4) of the tile
     int32_t raw;         // float offset of the raw staging rows
     int32_t raw_stride;  // bytes per raw staging row (multiple of 16)
-    int32_t block_start[kMaxImagesPerLaunch + 1];  // prefix sum of blocks (video blocks are halves)
-    ImageDesc img[kMaxImagesPerLaunch];
+    int32_t block_start[kCap + 1];  // prefix sum of blocks (video blocks are halves)
+    ImageDesc img[kCap];
 };
+using LaunchParams = LaunchParamsT<kMaxImagesPerLaunch>;
+constexpr int kSmallLaunch = 32;  // launches of up to this many images use the small block
+using SmallLaunchParams = LaunchParamsT<kSmallLaunch>;
 static_assert(sizeof(LaunchParams) <= 32764 - 64, "kernel parameter limit");
 
 // Bilinear taps of output index d along an axis of size in -> out under the

@@ -26,6 +26,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstddef>
+#include <cstring>
 
 #include "mimo.h"
 #include "mimo_internal.h"
@@ -63,7 +65,8 @@ __device__ __forceinline__ float2 on_white2(float2 c2, float2 a2, float2 white2)
 }
 
 // last i with block_start[i] <= blk
-__device__ __forceinline__ int find_image(const LaunchParams &P, int blk) {
+template <class Params>
+__device__ __forceinline__ int find_image(const Params &P, int blk) {
     int lo = 0, hi = P.n - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -112,7 +115,8 @@ struct AxisCursor {
 
 // Warps 0 (rows) and 1 (columns): taps of block blk into T. `prev` holds the
 // taps of the block before blk in this CTA's order.
-__device__ __forceinline__ void compute_taps(const LaunchParams &P, TapSet &T, const TapSet &prev, int blk,
+template <class Params>
+__device__ __forceinline__ void compute_taps(const Params &P, TapSet &T, const TapSet &prev, int blk,
                                              AxisCursor &cur, int warp, int lane) {
     // block position: consecutive blocks advance one column (or start the
     // next block row / temporal patch / item), a video first through its
@@ -318,7 +322,8 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src, int nbyte
 // raw buffer: row j's bytes [rs, rs + C*ncols) are covered by 16-byte aligned
 // chunks stored at raw + j*raw_stride. A chunk reaching past the caller's
 // buffer is zero-filled there.
-__device__ __forceinline__ void issue_stage(const LaunchParams &P, const TapSet &T, uint8_t *raw, int tid) {
+template <class Params>
+__device__ __forceinline__ void issue_stage(const Params &P, const TapSet &T, uint8_t *raw, int tid) {
     const int flags = T.flags;
     if ((flags & kGatherCols) == 0) {
         const uint8_t *img = P.src + T.src_off;
@@ -348,7 +353,8 @@ __device__ __forceinline__ void issue_stage(const LaunchParams &P, const TapSet 
 // Converts block T's staged bytes to planar fp32 in the tile (RGBA
 // composited onto white): a job = 4 consecutive pixels of one tile row.
 // Gathered columns are loaded here directly from global memory.
-__device__ __forceinline__ void finish_stage(const LaunchParams &P, const TapSet &T, const uint8_t *raw, float *tile,
+template <class Params>
+__device__ __forceinline__ void finish_stage(const Params &P, const TapSet &T, const uint8_t *raw, float *tile,
                                              int TS, int plane, int tid) {
     const int flags = T.flags;
     const int nrows = T.nrows;
@@ -442,8 +448,8 @@ __device__ __forceinline__ void finish_stage(const LaunchParams &P, const TapSet
 }
 
 // Interpolation, normalisation and stores of one staged block.
-template <bool kBF16>
-__device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &T, float *tile, int TS, int plane,
+template <bool kBF16, class Params>
+__device__ __forceinline__ void emit_block(const Params &P, const TapSet &T, float *tile, int TS, int plane,
                                            int tid, int warp, int lane) {
     const int flags = T.flags;
     const int nrows = T.nrows;
@@ -549,8 +555,8 @@ __device__ __forceinline__ void emit_block(const LaunchParams &P, const TapSet &
 // interpolated and stored, the source bytes of block k+1 are already in
 // shared memory and those of block k+2 are in flight (cp.async), and warps
 // 0-1 compute the taps of the block after.
-template <bool kBF16>
-__global__ void __launch_bounds__(kThreads, 5) preprocess_kernel(const __grid_constant__ LaunchParams P) {
+template <bool kBF16, class Params>
+__global__ void __launch_bounds__(kThreads, 5) preprocess_kernel(const __grid_constant__ Params P) {
     extern __shared__ float4 smem4[];
     float *const tile = reinterpret_cast<float *>(smem4);  // [3][rows][stride] | raw bytes
     uint8_t *const raw = reinterpret_cast<uint8_t *>(tile + P.raw);
@@ -657,8 +663,8 @@ __device__ __forceinline__ void convert4(const uint32_t (&w)[4], int C, float4 (
     v[2] = make_float4(B0.x, B0.y, B1.x, B1.y);
 }
 
-template <bool kBF16>
-__global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_constant__ LaunchParams P) {
+template <bool kBF16, class Params>
+__global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_constant__ Params P) {
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int64_t B = P.block_start[P.n];
@@ -800,9 +806,9 @@ struct LaunchSetup {
     int per_sm = 0;
 };
 
-template <bool kBF16>
-int launch_typed(const LaunchParams &lp, int64_t blocks, size_t smem_bytes, cudaStream_t stream) {
-    auto kern = preprocess_kernel<kBF16>;
+template <bool kBF16, class Params>
+int launch_typed(const Params &lp, int64_t blocks, size_t smem_bytes, cudaStream_t stream) {
+    auto kern = preprocess_kernel<kBF16, Params>;
     static thread_local LaunchSetup setup;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ECUDA;
@@ -833,9 +839,9 @@ int launch_typed(const LaunchParams &lp, int64_t blocks, size_t smem_bytes, cuda
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
 }
 
-template <bool kBF16>
-int launch_direct(const LaunchParams &lp, int64_t blocks, cudaStream_t stream) {
-    auto kern = direct_kernel<kBF16>;
+template <bool kBF16, class Params>
+int launch_direct(const Params &lp, int64_t blocks, cudaStream_t stream) {
+    auto kern = direct_kernel<kBF16, Params>;
     static thread_local LaunchSetup setup;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ECUDA;
@@ -854,14 +860,12 @@ int launch_direct(const LaunchParams &lp, int64_t blocks, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
 }
 
-}  // namespace
-
-int launch_preprocess(const LaunchParams &lp, int64_t blocks, int out_dtype, size_t smem_bytes, void *stream) {
-    if (blocks <= 0) return MIMO_OK;
-    if (blocks > static_cast<int64_t>(INT32_MAX)) return MIMO_EOVERFLOW;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // every width kept, no video halves: the direct kernel, unless fp32 rows are written for resized
-    // heights (there the staged kernel's burst reads keep the write stream faster, as measured)
+// Both kernels for one parameter block type, chosen as measured: the direct
+// kernel when every width is kept and no image is a video half, unless fp32
+// rows are written for resized heights (there the staged kernel's burst reads
+// keep the write stream faster).
+template <class Params>
+int launch_kernels(const Params &lp, int64_t blocks, int out_dtype, size_t smem_bytes, cudaStream_t s) {
     bool widths_kept = true, heights_kept = true;
     for (int i = 0; i < lp.n; ++i) {
         widths_kept = widths_kept && (lp.img[i].flags & kIdentityCols) != 0 && (lp.img[i].flags & kVideo) == 0;
@@ -871,6 +875,23 @@ int launch_preprocess(const LaunchParams &lp, int64_t blocks, int out_dtype, siz
         return out_dtype == MIMO_BF16 ? launch_direct<true>(lp, blocks, s) : launch_direct<false>(lp, blocks, s);
     return out_dtype == MIMO_BF16 ? launch_typed<true>(lp, blocks, smem_bytes, s)
                                   : launch_typed<false>(lp, blocks, smem_bytes, s);
+}
+
+}  // namespace
+
+int launch_preprocess(const LaunchParams &lp, int64_t blocks, int out_dtype, size_t smem_bytes, void *stream) {
+    if (blocks <= 0) return MIMO_OK;
+    if (blocks > static_cast<int64_t>(INT32_MAX)) return MIMO_EOVERFLOW;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (lp.n <= kSmallLaunch) {
+        // a few images: copy into the small parameter block (the launch then costs about half)
+        static thread_local SmallLaunchParams sp;
+        std::memcpy(&sp, &lp, offsetof(LaunchParams, block_start));
+        std::memcpy(sp.block_start, lp.block_start, sizeof(int32_t) * (lp.n + 1));
+        std::memcpy(sp.img, lp.img, sizeof(ImageDesc) * lp.n);
+        return launch_kernels(sp, blocks, out_dtype, smem_bytes, s);
+    }
+    return launch_kernels(lp, blocks, out_dtype, smem_bytes, s);
 }
 
 }  // namespace mimo

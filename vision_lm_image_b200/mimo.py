@@ -261,6 +261,9 @@ class PackedBatch:
         self.heights = np.ascontiguousarray(heights, np.int32)
         self.widths = np.ascontiguousarray(widths, np.int32)
         self.channels = np.ascontiguousarray(channels, np.int32)
+        # host addresses of the four arrays, looked up once (they are passed on every call)
+        self.ptrs = (self.offsets.ctypes.data, self.heights.ctypes.data, self.widths.ctypes.data,
+                     self.channels.ctypes.data)
 
     @property
     def n(self) -> int:
@@ -306,8 +309,7 @@ def preprocess_batch(params: MimoParams, packed: PackedBatch, out, perm=None, st
     buf = packed.buffer
     st = lib().mimo_preprocess_batch(
         ctypes.byref(params), packed.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
-        packed.offsets.ctypes.data, packed.heights.ctypes.data, packed.widths.ctypes.data,
-        packed.channels.ctypes.data, _dtype_code(out.dtype), ctypes.c_void_p(out.data_ptr()),
+        *packed.ptrs, _dtype_code(out.dtype), ctypes.c_void_p(out.data_ptr()),
         out.shape[0] if out.ndim == 2 else 0, ctypes.c_void_p(perm.data_ptr() if perm is not None else 0),
         _stream_handle(stream, buf.device))
     _check(st, "preprocess_batch")
@@ -337,8 +339,7 @@ def preprocess_batch_ex(params: MimoParams, packed: PackedBatch, out, perm=None,
     o.d_window_index = window.data_ptr() if window is not None else None
     st = lib().mimo_preprocess_batch_ex(
         ctypes.byref(params), packed.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
-        packed.offsets.ctypes.data, packed.heights.ctypes.data, packed.widths.ctypes.data,
-        packed.channels.ctypes.data, ctypes.byref(o), _stream_handle(stream, buf.device))
+        *packed.ptrs, ctypes.byref(o), _stream_handle(stream, buf.device))
     _check(st, "preprocess_batch_ex")
 
 
