@@ -390,6 +390,35 @@ def test_video_matches_oracle(n, shape, c):
         assert_fp32_close(pv.cpu().numpy(), want, f"video {order}")
 
 
+@pytest.mark.parametrize("dtype,shape", [(torch.bfloat16, (100, 128)), (torch.float32, (96, 128)),
+                                         (torch.bfloat16, (1080, 1920))])
+@pytest.mark.parametrize("n,c", [(3, 3), (4, 4)])
+def test_video_with_kept_width_matches_oracle(dtype, shape, n, c):
+    # frames whose width is kept go to the unstaged kernel (bf16 for any height, fp32 when the
+    # height is kept too): halves pick frame 2t + tt, an odd count repeats its last frame
+    assert oracle.smart_resize(*shape)[1] == shape[1]
+    rng = workloads.rng_for(700 + n + shape[0])
+    frames = np.stack([workloads.uniform_image(rng, shape[0], shape[1], 3) if c == 3
+                       else workloads.rgba_image(rng, shape[0], shape[1]) for _ in range(n)])
+    mean, std = workloads.CLIP_MEAN, workloads.CLIP_STD
+    ref, g = oracle.preprocess_video(frames, mean, std)
+    gt, gh, gw = g
+    for order in ("merge", "column"):
+        pv, grid, perm, pos, win = mimo.preprocess_video(frames, mean, std, dtype=dtype, column_perm=True,
+                                                         order=order, positions=True, window_index=True)
+        torch.cuda.synchronize()
+        assert tuple(grid[0].tolist()) == g
+        rperm = oracle.column_permutation(gh, gw, 2, 0, gt)
+        assert np.array_equal(perm.cpu().numpy(), rperm)
+        assert np.array_equal(win.cpu().numpy(), oracle.window_index(gh, gw, 2, 0, gt))
+        assert np.array_equal(pos.cpu().numpy(), oracle.rotary_positions(gh, gw, 2, order == "column", gt))
+        want = ref if order == "merge" else ref[rperm]
+        if dtype == torch.float32:
+            assert_fp32_close(pv.cpu().numpy(), want, f"video {order}")
+        else:
+            assert_bf16_close(pv, want, f"video {order}")
+
+
 def test_video_budget_and_bf16_full_hd():
     rng = workloads.rng_for(600)
     frames = np.stack([workloads.uniform_image(rng, 1080, 1920, 3) for _ in range(6)])

@@ -18,8 +18,8 @@
 //     page, column_permutation).
 // CTAs are persistent: each takes a contiguous range of blocks and overlaps
 // the source copies of the next blocks with the stores of the current one.
-// Launches whose images all keep their width go to a second, unstaged kernel
-// (direct_kernel below) when that measured faster.
+// Launches whose images or frames all keep their width go to a second,
+// unstaged kernel (direct_kernel below) when that measured faster.
 // There is no inter-CTA communication, no atomics and no global wait; every
 // output element has exactly one writer.
 #include <cuda_bf16.h>
@@ -600,8 +600,8 @@ __global__ void __launch_bounds__(kThreads, 5) preprocess_kernel(const __grid_co
 }
 
 // ---------------------------------------------------------------------------
-// Direct kernel, for launches whose images all keep their width (Wr == W, no
-// video halves). Every output column then samples its own source column, and
+// Direct kernel, for launches whose images (or video frames) all keep their
+// width (Wr == W). Every output column then samples its own source column, and
 // a block needs no staging. Each thread owns the same 4 pixels x 3 channels of
 // one output row in every block, as in the staged kernel's vertical pass. It
 // reads its one or two source rows straight from global memory (the ~2x reuse
@@ -681,13 +681,20 @@ __global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_consta
     const int dx0 = (mw << 4) | (q << 2);
     const int col = py * 16 + q * 4;
 
-    // position of the first block; later blocks advance one column at a time
+    // position of the first block (a video's blocks are (t, block row, block col, tt) halves, tt
+    // innermost); later blocks advance one step at a time
     int ii = find_image(P, begin);
-    int bh, bw;
+    int t, bh, bw, tt;
     {
         const ImageDesc &D = P.img[ii];
         const int g = D.Wr / kBlock;
-        const int local = begin - P.block_start[ii];
+        int local = begin - P.block_start[ii];
+        const bool vid = (D.flags & kVideo) != 0;
+        tt = vid ? (local & 1) : 0;
+        if (vid) local >>= 1;
+        const int units = (D.Hr / kBlock) * g;
+        t = local / units;
+        local -= t * units;
         bh = local / g;
         bw = local - bh * g;
     }
@@ -724,7 +731,10 @@ __global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_consta
             tap_ii = ii;
             tap_bh = bh;
         }
-        const uint8_t *img = P.src + D.src_off;
+        const bool video = (flags & kVideo) != 0;
+        // a video half reads frame 2t + tt, the last frame standing in past the end
+        const int64_t f = video ? min(2 * t + tt, D.frames - 1) : 0;
+        const uint8_t *img = P.src + D.src_off + f * D.frame_stride;
         const int64_t x = static_cast<int64_t>(bw) * kBlock + dx0;
         uint32_t wa[4], wb[4];
         float4 va[3], vb[3];
@@ -735,10 +745,13 @@ __global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_consta
         }
         convert4(wa, C, va);
 
-        // merge order lists units by (block row, block col), column order by (block col, block row)
+        // merge order lists units by (t, block row, block col), column order by (t, block col, block row)
         const int gw2 = D.Wr / kBlock, gh2 = Hr / kBlock;
-        const int64_t unit = P.order ? static_cast<int64_t>(bw) * gh2 + bh : static_cast<int64_t>(bh) * gw2 + bw;
+        const int64_t t_units = static_cast<int64_t>(t) * gh2 * gw2;
+        const int64_t unit =
+            t_units + (P.order ? static_cast<int64_t>(bw) * gh2 + bh : static_cast<int64_t>(bh) * gw2 + bw);
         const int64_t row = D.row0 + 4 * unit + (mh * 2 + mw);
+        const int slot0 = video ? 256 * tt : 0;
         const float2 ly2 = f2(ly, ly), nly2 = f2(-ly, -ly);
 #pragma unroll
         for (int c = 0; c < 3; ++c) {
@@ -750,28 +763,28 @@ __global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_consta
             const float2 k2 = f2(P.k[c], P.k[c]), b2 = f2(P.b[c], P.b[c]);
             const float2 n01 = fma2(v01, k2, b2);
             const float2 n23 = fma2(v23, k2, b2);
-            // an image fills both temporal slots with its one frame
+            // an image fills both temporal slots with its one frame; a video half fills slot tt
             if constexpr (!kBF16) {
-                float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col;
+                float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
                 const float4 f4 = make_float4(n01.x, n01.y, n23.x, n23.y);
                 __stcs(reinterpret_cast<float4 *>(o), f4);
-                __stcs(reinterpret_cast<float4 *>(o + 256), f4);
+                if (!video) __stcs(reinterpret_cast<float4 *>(o + 256), f4);
             } else {
-                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col;
+                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
                 const __nv_bfloat162 lo2 = __floats2bfloat162_rn(n01.x, n01.y);
                 const __nv_bfloat162 hi2 = __floats2bfloat162_rn(n23.x, n23.y);
                 uint2 u;
                 u.x = *reinterpret_cast<const uint32_t *>(&lo2);
                 u.y = *reinterpret_cast<const uint32_t *>(&hi2);
                 __stcs(reinterpret_cast<uint2 *>(o), u);
-                __stcs(reinterpret_cast<uint2 *>(o + 256), u);
+                if (!video) __stcs(reinterpret_cast<uint2 *>(o + 256), u);
             }
         }
-        // the merge unit's table entries: permutation (thread 0), rotary positions (thread 1),
-        // window index (thread 2), as in emit_block
-        if (tid < 3) {
-            const int64_t src_unit = static_cast<int64_t>(bh) * gw2 + bw;  // merge order
-            const int64_t dst_unit = static_cast<int64_t>(bw) * gh2 + bh;  // column order
+        // the merge unit's table entries (once per unit: a video's tt = 0 half): permutation
+        // (thread 0), rotary positions (thread 1), window index (thread 2), as in emit_block
+        if (tid < 3 && (!video || tt == 0)) {
+            const int64_t src_unit = t_units + static_cast<int64_t>(bh) * gw2 + bw;  // merge order
+            const int64_t dst_unit = t_units + static_cast<int64_t>(bw) * gh2 + bh;  // column order
             if (tid == 0 && P.perm != nullptr) {
                 const int32_t s0 = static_cast<int32_t>(D.row0 + 4 * src_unit);
                 __stcs(reinterpret_cast<int4 *>(P.perm + D.row0 + 4 * dst_unit), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
@@ -785,12 +798,21 @@ __global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_consta
                 P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
             }
         }
-        // next block: one column on, then the next block row, then the next image
-        if (++bw == gw2) {
-            bw = 0;
-            if (++bh == gh2) {
-                bh = 0;
-                ++ii;
+        // next block: the other half of a video unit, else one column on, then the next block row,
+        // then the next temporal patch; a new item starts where the block prefix sum says
+        if (ii + 1 < P.n && P.block_start[ii + 1] <= blk + 1) {
+            ++ii;
+            t = bh = bw = tt = 0;
+        } else if (video && tt == 0) {
+            tt = 1;
+        } else {
+            tt = 0;
+            if (++bw == gw2) {
+                bw = 0;
+                if (++bh == gh2) {
+                    bh = 0;
+                    ++t;
+                }
             }
         }
     }
@@ -861,14 +883,13 @@ int launch_direct(const Params &lp, int64_t blocks, cudaStream_t stream) {
 }
 
 // Both kernels for one parameter block type, chosen as measured: the direct
-// kernel when every width is kept and no image is a video half, unless fp32
-// rows are written for resized heights (there the staged kernel's burst reads
-// keep the write stream faster).
+// kernel when every width is kept, unless fp32 rows are written for resized
+// heights (there the staged kernel's burst reads keep the write stream faster).
 template <class Params>
 int launch_kernels(const Params &lp, int64_t blocks, int out_dtype, size_t smem_bytes, cudaStream_t s) {
     bool widths_kept = true, heights_kept = true;
     for (int i = 0; i < lp.n; ++i) {
-        widths_kept = widths_kept && (lp.img[i].flags & kIdentityCols) != 0 && (lp.img[i].flags & kVideo) == 0;
+        widths_kept = widths_kept && (lp.img[i].flags & kIdentityCols) != 0;
         heights_kept = heights_kept && (lp.img[i].flags & kIdentityRows) != 0;
     }
     if (widths_kept && (out_dtype == MIMO_BF16 || heights_kept))
