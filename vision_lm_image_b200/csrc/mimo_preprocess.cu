@@ -663,8 +663,8 @@ __device__ __forceinline__ void convert4(const uint32_t (&w)[4], int C, float4 (
     v[2] = make_float4(B0.x, B0.y, B1.x, B1.y);
 }
 
-template <bool kBF16, class Params>
-__global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_constant__ Params P) {
+template <bool kBF16, bool kVideoLaunch, class Params>
+__global__ void __launch_bounds__(kThreads, kVideoLaunch ? 5 : 6) direct_kernel(const __grid_constant__ Params P) {
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int64_t B = P.block_start[P.n];
@@ -731,7 +731,8 @@ __global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_consta
             tap_ii = ii;
             tap_bh = bh;
         }
-        const bool video = (flags & kVideo) != 0;
+        // a launch holds images only, or one video (kVideoLaunch): the image code carries no video work
+        const bool video = kVideoLaunch;
         // a video half reads frame 2t + tt, the last frame standing in past the end
         const int64_t f = video ? min(2 * t + tt, D.frames - 1) : 0;
         const uint8_t *img = P.src + D.src_off + f * D.frame_stride;
@@ -798,20 +799,28 @@ __global__ void __launch_bounds__(kThreads, 6) direct_kernel(const __grid_consta
                 P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
             }
         }
-        // next block: the other half of a video unit, else one column on, then the next block row,
-        // then the next temporal patch; a new item starts where the block prefix sum says
-        if (ii + 1 < P.n && P.block_start[ii + 1] <= blk + 1) {
-            ++ii;
-            t = bh = bw = tt = 0;
-        } else if (video && tt == 0) {
-            tt = 1;
+        if constexpr (kVideoLaunch) {
+            // next half: the other temporal slot of the unit, else one column on, then the next
+            // block row, then the next temporal patch (the launch's only item)
+            if (tt == 0) {
+                tt = 1;
+            } else {
+                tt = 0;
+                if (++bw == gw2) {
+                    bw = 0;
+                    if (++bh == gh2) {
+                        bh = 0;
+                        ++t;
+                    }
+                }
+            }
         } else {
-            tt = 0;
+            // next block: one column on, then the next block row, then the next image
             if (++bw == gw2) {
                 bw = 0;
                 if (++bh == gh2) {
                     bh = 0;
-                    ++t;
+                    ++ii;
                 }
             }
         }
@@ -861,9 +870,9 @@ int launch_typed(const Params &lp, int64_t blocks, size_t smem_bytes, cudaStream
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
 }
 
-template <bool kBF16, class Params>
+template <bool kBF16, bool kVideoLaunch, class Params>
 int launch_direct(const Params &lp, int64_t blocks, cudaStream_t stream) {
-    auto kern = direct_kernel<kBF16, Params>;
+    auto kern = direct_kernel<kBF16, kVideoLaunch, Params>;
     static thread_local LaunchSetup setup;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ECUDA;
@@ -887,13 +896,20 @@ int launch_direct(const Params &lp, int64_t blocks, cudaStream_t stream) {
 // heights (there the staged kernel's burst reads keep the write stream faster).
 template <class Params>
 int launch_kernels(const Params &lp, int64_t blocks, int out_dtype, size_t smem_bytes, cudaStream_t s) {
-    bool widths_kept = true, heights_kept = true;
+    bool widths_kept = true, heights_kept = true, video = false;
     for (int i = 0; i < lp.n; ++i) {
         widths_kept = widths_kept && (lp.img[i].flags & kIdentityCols) != 0;
         heights_kept = heights_kept && (lp.img[i].flags & kIdentityRows) != 0;
+        video = video || (lp.img[i].flags & kVideo) != 0;
     }
-    if (widths_kept && (out_dtype == MIMO_BF16 || heights_kept))
-        return out_dtype == MIMO_BF16 ? launch_direct<true>(lp, blocks, s) : launch_direct<false>(lp, blocks, s);
+    // a video launch carries exactly one clip
+    if (widths_kept && (out_dtype == MIMO_BF16 || heights_kept) && (!video || lp.n == 1)) {
+        if (video)
+            return out_dtype == MIMO_BF16 ? launch_direct<true, true>(lp, blocks, s)
+                                          : launch_direct<false, true>(lp, blocks, s);
+        return out_dtype == MIMO_BF16 ? launch_direct<true, false>(lp, blocks, s)
+                                      : launch_direct<false, false>(lp, blocks, s);
+    }
     return out_dtype == MIMO_BF16 ? launch_typed<true>(lp, blocks, smem_bytes, s)
                                   : launch_typed<false>(lp, blocks, smem_bytes, s);
 }
