@@ -344,7 +344,7 @@ def compare_patch_embed(args, mimo, w, dev, rows, weight, bias, out, err, stream
     # the whole chain from uint8 pixels: two calls over the batch vs the chunked entry point
     params = mimo.make_params(w["mean"], w["std"])
     packed = mimo.pack_images(w["images"], device=dev)
-    scratch = torch.empty(96 << 20, dtype=torch.uint8, device=dev)
+    scratch = torch.empty(192 << 20, dtype=torch.uint8, device=dev)
     two = lambda: (mimo.preprocess_batch_ex(params, packed, rows, None, stream=stream),
                    mimo.patch_embed(rows, weight, bias, out=out, error=err, stream=stream, check=False))
     chain = lambda: mimo.preprocess_embed(packed, weight, bias, w["mean"], w["std"], scratch=scratch, stream=stream,
@@ -442,7 +442,7 @@ def run_patch_embed(args, rank, world, local_rank):
                 "impl": "torch.addmm (cuBLAS)", "ms": lib_ms, "tflops": flops / (lib_ms * 1e-3) / 1e12},
             "pixels_to_embeddings": None if args.gemm_only else {"images": n_img, "two_calls_ms": two_ms, "chained_ms": chain_ms,
                                      "two_calls_images_per_s": n_img / (two_ms * 1e-3),
-                                     "chained_images_per_s": n_img / (chain_ms * 1e-3), "scratch_mb": 96},
+                                     "chained_images_per_s": n_img / (chain_ms * 1e-3), "scratch_mb": 192},
             "gpu_launches": args.steps, "clocks": clocks.summary(), "e2e": None, "cpu_baseline": cpu,
         }), flush=True)
 

@@ -327,14 +327,16 @@ int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int
                      const float *d_bias, int32_t out_dtype, void *d_out, int32_t *d_error, void *stream);
 
 /*
- * The pixel path followed by the patch embedding, image chunk by image chunk
+ * The pixel path followed by the patch embedding, image run by image run
  * (vision page, MiMoVisionTransformer.forward: patch rows -> patch embed).
- * Images are grouped into runs whose bf16 patch rows fit d_scratch; for each
- * run the pixel kernel writes the rows into the scratch and the
- * patch-embedding GEMM (as mimo_patch_embed) reads them back, much of them
- * still in L2, writing embeddings at the run's batch rows. Equal, bit for bit,
- * to mimo_preprocess_batch_ex with MIMO_BF16 rows followed by
- * mimo_patch_embed on them.
+ * Images are grouped into runs whose bf16 patch rows fit half of d_scratch;
+ * the runs alternate between the two halves. The pixel kernel writes a run's
+ * rows on `stream`, and the patch-embedding GEMM (as mimo_patch_embed) reads
+ * them on a second stream the library keeps per host thread and device, so it
+ * overlaps the next run's pixel kernel. Events order each GEMM after its rows
+ * and each reuse of a half after the GEMM that read it; `stream` finally waits
+ * for the last GEMMs. Equal, bit for bit, to mimo_preprocess_batch_ex with
+ * MIMO_BF16 rows followed by mimo_patch_embed on them.
  *   p, n, d_src, src_bytes, src_offsets, heights, widths, channels: as in
  *       mimo_preprocess_batch.
  *   row_order:  MIMO_ORDER_MERGE or MIMO_ORDER_COLUMN (order of the output rows).
@@ -342,9 +344,9 @@ int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int
  *   d_out:      device [total_rows, embed_dim] of out_dtype; out_rows_capacity
  *               its row count (MIMO_ECAPACITY if below total_rows).
  *   d_scratch:  device buffer of scratch_bytes, 16-byte aligned, owned by the
- *               caller; it must hold one image's rows (rows x 3072 bytes),
- *               MIMO_ECAPACITY otherwise. Larger runs fill the GPU better,
- *               smaller ones stay in the 126 MB L2.
+ *               caller; half of it must hold one image's rows (rows x 3072
+ *               bytes), MIMO_ECAPACITY otherwise. About 2 x 96 MB or more
+ *               keeps the GEMMs' last waves full.
  * No permutation or index tables (mimo_preprocess_batch_ex writes those).
  * Asynchronous on `stream`.
  */

@@ -270,4 +270,4 @@ def test_preprocess_embed_validation_statuses():
     assert call(cap=8159) == 7
     assert call(weight=0) == 1 and call(scratch=0) == 1
     assert call(scratch=FAKE + 8) == 6
-    assert call(scratch_bytes=8160 * 3072 - 2) == 7   # the scratch must hold one image's rows
+    assert call(scratch_bytes=2 * 8160 * 3072 - 2) == 7   # half the scratch must hold one image's rows

@@ -590,28 +590,62 @@ int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src,
         (reinterpret_cast<uintptr_t>(d_error) & 3u) != 0)
         return MIMO_EALIGN;
     if (v.total_rows > (int64_t(1) << 31) - 1) return MIMO_EOVERFLOW;
-    // a run is a sequence of whole images whose bf16 rows fit the scratch; on one
-    // stream the next run's pixel kernel starts after this run's GEMM has read them
+    // runs of whole images alternate between the two halves of the scratch. The pixel kernel of run r
+    // goes on the caller's stream, the GEMM of run r on a second stream of the library's, so that it
+    // overlaps the pixel kernel of run r + 1 (the unstaged pixel kernel holds no shared memory and fits
+    // beside the GEMM's CTAs). Events order each GEMM after its run's rows and each reuse of a half after
+    // the GEMM that read it; the caller's stream finally waits for the last GEMMs.
     const int64_t row_bytes = static_cast<int64_t>(mimo::kRowWidth) * 2;
-    const int64_t run_rows = static_cast<int64_t>(scratch_bytes) / row_bytes;
+    const int64_t run_rows = static_cast<int64_t>(scratch_bytes / 2) / row_bytes;
+    for (int32_t i = 0; i < n; ++i)
+        if (v.plan.row0[i + 1] - v.plan.row0[i] > run_rows) return MIMO_ECAPACITY;  // exceeds half the scratch
+    struct Aux {
+        int dev = -1;
+        cudaStream_t s = nullptr;
+        cudaEvent_t rows_ready[2] = {nullptr, nullptr}, rows_read[2] = {nullptr, nullptr};
+    };
+    static thread_local Aux aux;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ECUDA;
+    if (aux.dev != dev) {
+        aux = Aux();
+        if (cudaStreamCreateWithFlags(&aux.s, cudaStreamNonBlocking) != cudaSuccess) return MIMO_ECUDA;
+        for (int k = 0; k < 2; ++k)
+            if (cudaEventCreateWithFlags(&aux.rows_ready[k], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&aux.rows_read[k], cudaEventDisableTiming) != cudaSuccess)
+                return MIMO_ECUDA;
+        aux.dev = dev;
+    }
+    cudaStream_t main_s = static_cast<cudaStream_t>(stream);
+    uint8_t *halves[2] = {static_cast<uint8_t *>(d_scratch), static_cast<uint8_t *>(d_scratch) + run_rows * row_bytes};
     const size_t esz = out_dtype == MIMO_BF16 ? 2 : 4;
     Tables tables;
     tables.order = row_order;
-    for (int32_t i0 = 0; i0 < n;) {
+    int run = 0;
+    for (int32_t i0 = 0; i0 < n; ++run) {
         int32_t i1 = i0;
         while (i1 < n && v.plan.row0[i1 + 1] - v.plan.row0[i0] <= run_rows) ++i1;
-        if (i1 == i0) return MIMO_ECAPACITY;  // one image's rows exceed the scratch
+        if (i1 == i0) return MIMO_ECAPACITY;  // one image's rows exceed half the scratch
+        const int h = run & 1;
         const int64_t row_base = v.plan.row0[i0];
         const int64_t rows = v.plan.row0[i1] - row_base;
+        if (run >= 2 && cudaStreamWaitEvent(main_s, aux.rows_read[h], 0) != cudaSuccess) return MIMO_ECUDA;
         st = launch_range(p, v, i0, i1, d_src, src_bytes, src_offsets, heights, widths, channels, MIMO_BF16,
-                          d_scratch, nullptr, stream, tables, row_base);
+                          halves[h], nullptr, stream, tables, row_base);
         if (st != MIMO_OK) return st;
-        st = mimo::launch_patch_embed(d_scratch, rows, mimo::kRowWidth, d_weight, embed_dim, d_bias, out_dtype,
+        if (cudaEventRecord(aux.rows_ready[h], main_s) != cudaSuccess ||
+            cudaStreamWaitEvent(aux.s, aux.rows_ready[h], 0) != cudaSuccess)
+            return MIMO_ECUDA;
+        st = mimo::launch_patch_embed(halves[h], rows, mimo::kRowWidth, d_weight, embed_dim, d_bias, out_dtype,
                                       static_cast<uint8_t *>(d_out) + static_cast<size_t>(row_base) * embed_dim * esz,
-                                      d_error, stream);
+                                      d_error, aux.s);
         if (st != MIMO_OK) return st;
+        if (cudaEventRecord(aux.rows_read[h], aux.s) != cudaSuccess) return MIMO_ECUDA;
         i0 = i1;
     }
+    // the caller's stream sees every GEMM done
+    for (int h = 0; h < 2 && h < run; ++h)
+        if (cudaStreamWaitEvent(main_s, aux.rows_read[h], 0) != cudaSuccess) return MIMO_ECUDA;
     return MIMO_OK;
 }
 

@@ -508,7 +508,7 @@ def patch_embed(rows, weight, bias=None, out_dtype=None, out=None, error=None, s
 
 
 def preprocess_embed(images, weight, bias=None, mean=None, std=None, min_pixels: int | None = None,
-                     max_pixels: int | None = None, out_dtype=None, order: str = "merge", scratch_bytes: int = 96 << 20,
+                     max_pixels: int | None = None, out_dtype=None, order: str = "merge", scratch_bytes: int = 192 << 20,
                      scratch=None, device="cuda", stream=None, check: bool = True):
     """Pixel path + patch embedding chunk by chunk: returns (embeddings [rows, embed_dim], image_grid_thw)."""
     import torch
