@@ -1,0 +1,51 @@
+"""Host-side logic of bench.py that decides what the JSON line reports (no GPU needed)."""
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_traffic_is_reported_only_for_the_captured_kernel_source(tmp_path, monkeypatch):
+    digest = bench.kernel_source_digest("preprocess")
+    table = {"c5_f32": {"kernel_digest": digest, "dram_bytes_per_launch": 1000},
+             "c5_bf16": {"kernel_digest": "0000000000000000", "dram_bytes_per_launch": 500},
+             "pe_bf16": {"kernel_digest": bench.kernel_source_digest("patch_embed"), "dram_bytes_per_launch": 800,
+                         "full_rows": 400}}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(table))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    # the digests are computed from the sources under ROOT: point them back at the repository
+    monkeypatch.setattr(bench, "kernel_source_digest",
+                        lambda kernel="preprocess": table["c5_f32"]["kernel_digest"] if kernel == "preprocess"
+                        else table["pe_bf16"]["kernel_digest"])
+    assert bench.ncu_traffic("c5", "f32") == 1000
+    assert bench.ncu_traffic("c5", "bf16") is None           # captured on another kernel source
+    assert bench.ncu_traffic("c3", "f32") is None            # never captured
+    assert bench.ncu_traffic("pe", "bf16", "patch_embed", rows=400) == 800
+    assert bench.ncu_traffic("pe", "bf16", "patch_embed", rows=100) == 200   # scaled by rows
+
+
+def test_committed_traffic_table_is_consistent():
+    # entries name the kernel sources they were captured on (bench.py reports null for any other source)
+    with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+        table = json.load(f)
+    for key in ("c5_f32", "c5_bf16", "pe_bf16"):
+        e = table[key]
+        assert len(e["kernel_digest"]) == 16 and int(e["kernel_digest"], 16) >= 0
+        assert e["dram_bytes_per_launch"] == e["read"] + e["write"]
+
+
+def test_algorithmic_bytes_of_c5():
+    class Packed:
+        heights = [1080] * 256
+        widths = [1920] * 256
+        channels = [3, 4] * 128
+    nb = bench.algorithmic_bytes(Packed(), 256 * 8160, 4, True)
+    assert nb["read"] == 1_857_945_600
+    assert nb["write_rows"] == 12_834_570_240
+    assert nb["write_perm"] == 8_355_840
+    assert nb["total"] == 14_700_871_680
