@@ -542,3 +542,53 @@ def test_preprocess_embed_c5_sample_against_oracle():
         got = emb[i * 8160 + pick].float().cpu().numpy().astype(np.float64)
         tol = 2.0 ** -8 * scale + 1e-5 * scale + 2.0 ** -8 * np.abs(ref) + 1e-6
         assert (np.abs(got - ref) <= tol).all(), np.abs(got - ref).max()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_calls_replay_from_a_cuda_graph(dtype):
+    # the launches a call makes can be captured once and replayed (planning runs at capture); replays on
+    # new pixels in the same buffers equal fresh calls, for the staged and the unstaged kernel
+    for seed, shapes in ((31, [(1079, 1920, 4), (1088, 640, 3)]), (32, [(300, 200, 3), (47, 512, 4)])):
+        rng = workloads.rng_for(seed)
+        make = lambda: [workloads.rgba_image(rng, h, w) if c == 4 else workloads.uniform_image(rng, h, w, 3)
+                        for h, w, c in shapes]
+        params = mimo.make_params(workloads.CLIP_MEAN, workloads.CLIP_STD)
+        packed = mimo.pack_images(make(), device="cuda")
+        grid, offs = mimo.plan_batch(packed.heights, packed.widths, params)
+        total = int(offs[-1])
+        out = torch.empty((total, 1536), dtype=dtype, device="cuda")
+        perm = torch.empty(total, dtype=torch.int32, device="cuda")
+        g = torch.Generator(device="cpu").manual_seed(seed)
+        w = (torch.randn((256, 1536), generator=g) * 0.02).to(torch.bfloat16).cuda()
+        emb = torch.empty((total, 256), dtype=torch.bfloat16, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        rows_bf16 = out if dtype == torch.bfloat16 else None
+        mimo.preprocess_batch_ex(params, packed, out, perm)  # warm-up outside the capture
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            mimo.preprocess_batch_ex(params, packed, out, perm)
+            if rows_bf16 is not None:
+                mimo.patch_embed(rows_bf16, w, None, out=emb, error=err, check=False)
+        # new pixels into the same device buffer, then replay
+        fresh = mimo.pack_images(make(), device="cpu")
+        packed.buffer.copy_(fresh.buffer)
+        graph.replay()
+        torch.cuda.synchronize()
+        imgs = [np.ascontiguousarray(x) for x in _unpack(fresh)]
+        want_rows, _, want_perm = mimo.preprocess(imgs, workloads.CLIP_MEAN, workloads.CLIP_STD, dtype=dtype,
+                                                  column_perm=True)
+        assert torch.equal(perm, want_perm)
+        assert torch.equal(out.view(torch.int16 if dtype == torch.bfloat16 else torch.int32),
+                           want_rows.view(torch.int16 if dtype == torch.bfloat16 else torch.int32))
+        if rows_bf16 is not None:
+            assert int(err.item()) == 0
+            assert torch.equal(emb.view(torch.int16), mimo.patch_embed(want_rows, w).view(torch.int16))
+        del graph
+
+
+def _unpack(packed):
+    """The HWC images of a host PackedBatch."""
+    buf = packed.buffer.numpy()
+    return [buf[o:o + h * w * c].reshape(h, w, c)
+            for o, h, w, c in zip(packed.offsets, packed.heights, packed.widths, packed.channels)]
