@@ -123,14 +123,16 @@ int mimo_num_patches(int64_t height, int64_t width, const mimo_params *p, int64_
  *   grid_thw:       out, [n*3] int64, rows (1, H'/16, W'/16).
  *   row_offsets:    out, [n+1] int64, first output row of each image; the
  *                   last entry is the total number of rows.
- * The first image whose geometry fails decides the returned status.
+ * The first image whose geometry fails decides the returned status. A
+ * resized side of 2^30 pixels or more is MIMO_EOVERFLOW (reachable only with
+ * a max_pixels far above the default).
  */
 int mimo_plan_batch(int32_t n, const int32_t *heights, const int32_t *widths,
                     const mimo_params *p, int64_t *grid_thw, int64_t *row_offsets);
 
 /*
  * The fused pixel path for a batch, on the GPU.
- *   d_src:        device, packed interleaved HWC uint8 images.
+ *   d_src:        device, packed interleaved HWC uint8 images, 16-byte aligned.
  *   src_bytes:    size of the d_src buffer; every image must lie inside it
  *                 (MIMO_ERANGE otherwise).
  *   src_offsets:  host [n], byte offset of image i in d_src, a multiple of 16.
