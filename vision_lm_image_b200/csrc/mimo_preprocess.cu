@@ -447,6 +447,57 @@ __device__ __forceinline__ void finish_stage(const Params &P, const TapSet &T, c
     }
 }
 
+// Normalises one channel's 4 interpolated values (x*k + b) and stores them at
+// column `col` of output row `row`: into both temporal slots for an image
+// (`both`), into the slot at `slot0` for a video half. Streaming stores.
+template <bool kBF16, class Params>
+__device__ __forceinline__ void store_quad(const Params &P, int64_t row, int c, int col, int slot0, bool both,
+                                           float2 v01, float2 v23) {
+    const float2 k2 = f2(P.k[c], P.k[c]), b2 = f2(P.b[c], P.b[c]);
+    const float2 n01 = fma2(v01, k2, b2);
+    const float2 n23 = fma2(v23, k2, b2);
+    if constexpr (!kBF16) {
+        float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
+        const float4 f4 = make_float4(n01.x, n01.y, n23.x, n23.y);
+        __stcs(reinterpret_cast<float4 *>(o), f4);
+        if (both) __stcs(reinterpret_cast<float4 *>(o + 256), f4);
+    } else {
+        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
+        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(n01.x, n01.y);
+        const __nv_bfloat162 hi2 = __floats2bfloat162_rn(n23.x, n23.y);
+        uint2 u;
+        u.x = *reinterpret_cast<const uint32_t *>(&lo2);
+        u.y = *reinterpret_cast<const uint32_t *>(&hi2);
+        __stcs(reinterpret_cast<uint2 *>(o), u);
+        if (both) __stcs(reinterpret_cast<uint2 *>(o + 256), u);
+    }
+}
+
+// The merge unit's table entries, written by threads 0-2 of the block: the
+// column-order permutation (thread 0), the rotary positions of the unit's 4
+// emitted rows starting at `row_base` (thread 1), the window index (thread 2).
+// `row0` is the item's first row, `t_units` the units of its earlier temporal
+// patches.
+template <class Params>
+__device__ __forceinline__ void write_unit_tables(const Params &P, int tid, int64_t row0, int64_t t_units, int bh,
+                                                  int bw, int gh2, int gw2, int64_t row_base) {
+    const int64_t src_unit = t_units + static_cast<int64_t>(bh) * gw2 + bw;  // merge order
+    const int64_t dst_unit = t_units + static_cast<int64_t>(bw) * gh2 + bh;  // column order
+    if (tid == 0 && P.perm != nullptr) {
+        const int32_t s0 = static_cast<int32_t>(row0 + 4 * src_unit);
+        __stcs(reinterpret_cast<int4 *>(P.perm + row0 + 4 * dst_unit), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
+    } else if (tid == 1 && P.pos != nullptr) {
+        // rows (mh, mw) = (0,0), (0,1), (1,0), (1,1) of the unit
+        const int32_t h = 2 * bh, w = 2 * bw;
+        int4 *d = reinterpret_cast<int4 *>(P.pos + 2 * row_base);
+        __stcs(d, make_int4(h, w, h, w + 1));
+        __stcs(d + 1, make_int4(h + 1, w, h + 1, w + 1));
+    } else if (tid == 2 && P.win != nullptr) {
+        const int64_t u0 = row0 / 4;
+        P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
+    }
+}
+
 // Interpolation, normalisation and stores of one staged block.
 template <bool kBF16, class Params>
 __device__ __forceinline__ void emit_block(const Params &P, const TapSet &T, float *tile, int TS, int plane,
@@ -507,47 +558,14 @@ __device__ __forceinline__ void emit_block(const Params &P, const TapSet &T, flo
             v01 = fma2(ly2, f2(B.x, B.y), fma2(nly2, v01, v01));
             v23 = fma2(ly2, f2(B.z, B.w), fma2(nly2, v23, v23));
         }
-        const float2 k2 = f2(P.k[c], P.k[c]), b2 = f2(P.b[c], P.b[c]);
-        const float2 n01 = fma2(v01, k2, b2);
-        const float2 n23 = fma2(v23, k2, b2);
         // an image fills both temporal slots with its one frame; a video half fills slot tt
-        if constexpr (!kBF16) {
-            float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
-            const float4 f4 = make_float4(n01.x, n01.y, n23.x, n23.y);
-            __stcs(reinterpret_cast<float4 *>(o), f4);
-            if (both) __stcs(reinterpret_cast<float4 *>(o + 256), f4);
-        } else {
-            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
-            const __nv_bfloat162 lo2 = __floats2bfloat162_rn(n01.x, n01.y);
-            const __nv_bfloat162 hi2 = __floats2bfloat162_rn(n23.x, n23.y);
-            uint2 u;
-            u.x = *reinterpret_cast<const uint32_t *>(&lo2);
-            u.y = *reinterpret_cast<const uint32_t *>(&hi2);
-            __stcs(reinterpret_cast<uint2 *>(o), u);
-            if (both) __stcs(reinterpret_cast<uint2 *>(o + 256), u);
-        }
+        store_quad<kBF16>(P, row, c, col, slot0, both, v01, v23);
     }
 
-    // the merge unit's table entries: permutation (thread 0), rotary
-    // positions of its 4 emitted rows (thread 1), window index (thread 2)
-    if (tid < 3 && (!video || T.tt == 0)) {
-        const int64_t t_units = static_cast<int64_t>(T.t) * T.gh2 * T.gw2;
-        const int64_t src_unit = t_units + static_cast<int64_t>(T.bh) * T.gw2 + T.bw;  // merge order
-        const int64_t dst_unit = t_units + static_cast<int64_t>(T.bw) * T.gh2 + T.bh;  // column order
-        if (tid == 0 && P.perm != nullptr) {
-            const int32_t s0 = static_cast<int32_t>(T.row0 + 4 * src_unit);
-            __stcs(reinterpret_cast<int4 *>(P.perm + T.row0 + 4 * dst_unit), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
-        } else if (tid == 1 && P.pos != nullptr) {
-            // rows (mh, mw) = (0,0), (0,1), (1,0), (1,1) of the unit
-            const int32_t h = 2 * T.bh, w = 2 * T.bw;
-            int4 *d = reinterpret_cast<int4 *>(P.pos + 2 * T.row_base);
-            __stcs(d, make_int4(h, w, h, w + 1));
-            __stcs(d + 1, make_int4(h + 1, w, h + 1, w + 1));
-        } else if (tid == 2 && P.win != nullptr) {
-            const int64_t u0 = T.row0 / 4;
-            P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
-        }
-    }
+    // the merge unit's table entries (once per unit: a video's tt = 0 half)
+    if (tid < 3 && (!video || T.tt == 0))
+        write_unit_tables(P, tid, T.row0, static_cast<int64_t>(T.t) * T.gh2 * T.gw2, T.bh, T.bw, T.gh2, T.gw2,
+                          T.row_base);
 }
 
 // Persistent CTAs: CTA c takes the contiguous block range
@@ -761,28 +779,12 @@ __global__ void __launch_bounds__(kThreads, kVideoLaunch ? 5 : 6) direct_kernel(
                 v01 = fma2(ly2, f2(vb[c].x, vb[c].y), fma2(nly2, v01, v01));
                 v23 = fma2(ly2, f2(vb[c].z, vb[c].w), fma2(nly2, v23, v23));
             }
-            const float2 k2 = f2(P.k[c], P.k[c]), b2 = f2(P.b[c], P.b[c]);
-            const float2 n01 = fma2(v01, k2, b2);
-            const float2 n23 = fma2(v23, k2, b2);
             // an image fills both temporal slots with its one frame; a video half fills slot tt
-            if constexpr (!kBF16) {
-                float *o = static_cast<float *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
-                const float4 f4 = make_float4(n01.x, n01.y, n23.x, n23.y);
-                __stcs(reinterpret_cast<float4 *>(o), f4);
-                if (!video) __stcs(reinterpret_cast<float4 *>(o + 256), f4);
-            } else {
-                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
-                const __nv_bfloat162 lo2 = __floats2bfloat162_rn(n01.x, n01.y);
-                const __nv_bfloat162 hi2 = __floats2bfloat162_rn(n23.x, n23.y);
-                uint2 u;
-                u.x = *reinterpret_cast<const uint32_t *>(&lo2);
-                u.y = *reinterpret_cast<const uint32_t *>(&hi2);
-                __stcs(reinterpret_cast<uint2 *>(o), u);
-                if (!video) __stcs(reinterpret_cast<uint2 *>(o + 256), u);
-            }
+            store_quad<kBF16>(P, row, c, col, slot0, !video, v01, v23);
         }
-        // the merge unit's table entries (once per unit: a video's tt = 0 half): permutation
-        // (thread 0), rotary positions (thread 1), window index (thread 2), as in emit_block
+        // the merge unit's table entries (once per unit: a video's tt = 0 half): the same entries
+        // as write_unit_tables, written inline here because calling that helper from this loop
+        // made the bf16 image launch about 1.4% slower
         if (tid < 3 && (!video || tt == 0)) {
             const int64_t src_unit = t_units + static_cast<int64_t>(bh) * gw2 + bw;  // merge order
             const int64_t dst_unit = t_units + static_cast<int64_t>(bw) * gh2 + bh;  // column order
