@@ -226,7 +226,8 @@ int mimo_preprocess_batch_host(const mimo_params *p, int32_t n,
  *   - Arguments and results are those of mimo_preprocess_batch_host without
  *     the three device staging buffers. The call runs on the current device;
  *     `stream` must belong to it. Synchronous: returns after the last copy
- *     to h_out has completed.
+ *     to h_out has completed. A CUDA error part-way still waits for the
+ *     work already queued on `stream` before it returns MIMO_ECUDA.
  *   - The batch is processed in chunks of whole images. An image whose
  *     uint8 bytes plus output rows (plus permutation entries when asked for)
  *     exceed the area, rounded up as the staging layout needs, is rejected
@@ -350,7 +351,9 @@ int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int
  *               bytes), MIMO_ECAPACITY otherwise. About 2 x 96 MB or more
  *               keeps the GEMMs' last waves full.
  * No permutation or index tables (mimo_preprocess_batch_ex writes those).
- * Asynchronous on `stream`.
+ * Asynchronous on `stream`. Argument errors return before anything is
+ * queued; a CUDA error part-way waits for the second stream's queued GEMMs
+ * before it returns, so none of them runs after the call.
  */
 int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src, size_t src_bytes,
                           const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,

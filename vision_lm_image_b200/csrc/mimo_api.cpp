@@ -230,7 +230,7 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
                  size_t src_bytes, const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
                  const int32_t *channels, int32_t out_dtype, void *d_out, int32_t *d_perm, void *stream,
                  const Tables &tables = Tables(), int64_t row_base = 0) {
-    static thread_local mimo::LaunchParams lp;  // 23 KB: kept off the stack
+    static thread_local mimo::LaunchParams lp;  // 31 KB: kept off the stack
     int32_t i = first;
     while (i < last) {
         std::memset(&lp, 0, sizeof(lp));
@@ -486,6 +486,12 @@ int mimo_preprocess_batch_host_noalloc(const mimo_params *p, int32_t n, const ui
     if (rc != MIMO_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const uintptr_t base = reinterpret_cast<uintptr_t>(stage);
+    // an error after the first enqueue still waits for what was queued, so
+    // that no copy touches the caller's host buffers after the return
+    auto bail = [s](int status) {
+        cudaStreamSynchronize(s);
+        return status;
+    };
 
     // the launch helper reads source offsets by batch index: chunk-local
     // positions go into a batch-sized table
@@ -510,7 +516,7 @@ int mimo_preprocess_batch_host_noalloc(const mimo_params *p, int32_t n, const ui
             const size_t bytes = static_cast<size_t>(heights[k]) * widths[k] * channels[k];
             if (cudaMemcpyAsync(reinterpret_cast<void *>(base + static_cast<uintptr_t>(local_off[k])),
                                 h_src + src_offsets[k], bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
-                return MIMO_ECUDA;
+                return bail(MIMO_ECUDA);
         }
         // The kernel addresses rows and permutation entries by batch-global
         // row index; shifting the bases down by the chunk's first row puts
@@ -520,15 +526,15 @@ int mimo_preprocess_batch_host_noalloc(const mimo_params *p, int32_t n, const ui
             perm ? reinterpret_cast<int32_t *>(perm_at - static_cast<uintptr_t>(row0) * sizeof(int32_t)) : nullptr;
         rc = launch_range(p, v, first, i, reinterpret_cast<const uint8_t *>(base), src_used, local_off.data(),
                           heights, widths, channels, out_dtype, out_base, perm_base, s);
-        if (rc != MIMO_OK) return rc;
+        if (rc != MIMO_OK) return bail(rc);
         if (cudaMemcpyAsync(static_cast<char *>(h_out) + static_cast<size_t>(row0) * row_bytes,
                             reinterpret_cast<void *>(out_at), static_cast<size_t>(rows) * row_bytes,
                             cudaMemcpyDeviceToHost, s) != cudaSuccess)
-            return MIMO_ECUDA;
+            return bail(MIMO_ECUDA);
         if (perm && cudaMemcpyAsync(h_column_perm + row0, reinterpret_cast<void *>(perm_at),
                                     static_cast<size_t>(rows) * sizeof(int32_t), cudaMemcpyDeviceToHost,
                                     s) != cudaSuccess)
-            return MIMO_ECUDA;
+            return bail(MIMO_ECUDA);
     }
     return cudaStreamSynchronize(s) == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
 }
@@ -599,24 +605,35 @@ int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src,
     const int64_t run_rows = static_cast<int64_t>(scratch_bytes / 2) / row_bytes;
     for (int32_t i = 0; i < n; ++i)
         if (v.plan.row0[i + 1] - v.plan.row0[i] > run_rows) return MIMO_ECAPACITY;  // exceeds half the scratch
+    // the second stream and its events, made once per host thread and device
     struct Aux {
-        int dev = -1;
+        bool ready = false;
         cudaStream_t s = nullptr;
         cudaEvent_t rows_ready[2] = {nullptr, nullptr}, rows_read[2] = {nullptr, nullptr};
     };
-    static thread_local Aux aux;
+    constexpr int kMaxDevices = 64;
+    static thread_local Aux aux_of[kMaxDevices];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ECUDA;
-    if (aux.dev != dev) {
-        aux = Aux();
-        if (cudaStreamCreateWithFlags(&aux.s, cudaStreamNonBlocking) != cudaSuccess) return MIMO_ECUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MIMO_ECUDA;
+    Aux &aux = aux_of[dev];
+    if (!aux.ready) {
+        // handles made before a failed creation are kept and reused by the next attempt
+        if (!aux.s && cudaStreamCreateWithFlags(&aux.s, cudaStreamNonBlocking) != cudaSuccess) return MIMO_ECUDA;
         for (int k = 0; k < 2; ++k)
-            if (cudaEventCreateWithFlags(&aux.rows_ready[k], cudaEventDisableTiming) != cudaSuccess ||
-                cudaEventCreateWithFlags(&aux.rows_read[k], cudaEventDisableTiming) != cudaSuccess)
+            if ((!aux.rows_ready[k] && cudaEventCreateWithFlags(&aux.rows_ready[k], cudaEventDisableTiming) !=
+                                           cudaSuccess) ||
+                (!aux.rows_read[k] &&
+                 cudaEventCreateWithFlags(&aux.rows_read[k], cudaEventDisableTiming) != cudaSuccess))
                 return MIMO_ECUDA;
-        aux.dev = dev;
+        aux.ready = true;
     }
     cudaStream_t main_s = static_cast<cudaStream_t>(stream);
+    // an error after the first enqueue waits for the second stream's work, so
+    // that no GEMM still reads the scratch or writes d_out after the return
+    auto bail = [&aux](int status) {
+        cudaStreamSynchronize(aux.s);
+        return status;
+    };
     uint8_t *halves[2] = {static_cast<uint8_t *>(d_scratch), static_cast<uint8_t *>(d_scratch) + run_rows * row_bytes};
     const size_t esz = out_dtype == MIMO_BF16 ? 2 : 4;
     Tables tables;
@@ -625,27 +642,27 @@ int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src,
     for (int32_t i0 = 0; i0 < n; ++run) {
         int32_t i1 = i0;
         while (i1 < n && v.plan.row0[i1 + 1] - v.plan.row0[i0] <= run_rows) ++i1;
-        if (i1 == i0) return MIMO_ECAPACITY;  // one image's rows exceed half the scratch
+        if (i1 == i0) return bail(MIMO_ECAPACITY);  // one image's rows exceed half the scratch
         const int h = run & 1;
         const int64_t row_base = v.plan.row0[i0];
         const int64_t rows = v.plan.row0[i1] - row_base;
-        if (run >= 2 && cudaStreamWaitEvent(main_s, aux.rows_read[h], 0) != cudaSuccess) return MIMO_ECUDA;
+        if (run >= 2 && cudaStreamWaitEvent(main_s, aux.rows_read[h], 0) != cudaSuccess) return bail(MIMO_ECUDA);
         st = launch_range(p, v, i0, i1, d_src, src_bytes, src_offsets, heights, widths, channels, MIMO_BF16,
                           halves[h], nullptr, stream, tables, row_base);
-        if (st != MIMO_OK) return st;
+        if (st != MIMO_OK) return bail(st);
         if (cudaEventRecord(aux.rows_ready[h], main_s) != cudaSuccess ||
             cudaStreamWaitEvent(aux.s, aux.rows_ready[h], 0) != cudaSuccess)
-            return MIMO_ECUDA;
+            return bail(MIMO_ECUDA);
         st = mimo::launch_patch_embed(halves[h], rows, mimo::kRowWidth, d_weight, embed_dim, d_bias, out_dtype,
                                       static_cast<uint8_t *>(d_out) + static_cast<size_t>(row_base) * embed_dim * esz,
                                       d_error, aux.s);
-        if (st != MIMO_OK) return st;
-        if (cudaEventRecord(aux.rows_read[h], aux.s) != cudaSuccess) return MIMO_ECUDA;
+        if (st != MIMO_OK) return bail(st);
+        if (cudaEventRecord(aux.rows_read[h], aux.s) != cudaSuccess) return bail(MIMO_ECUDA);
         i0 = i1;
     }
     // the caller's stream sees every GEMM done
     for (int h = 0; h < 2 && h < run; ++h)
-        if (cudaStreamWaitEvent(main_s, aux.rows_read[h], 0) != cudaSuccess) return MIMO_ECUDA;
+        if (cudaStreamWaitEvent(main_s, aux.rows_read[h], 0) != cudaSuccess) return bail(MIMO_ECUDA);
     return MIMO_OK;
 }
 
