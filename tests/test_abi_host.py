@@ -271,3 +271,33 @@ def test_preprocess_embed_validation_statuses():
     assert call(weight=0) == 1 and call(scratch=0) == 1
     assert call(scratch=FAKE + 8) == 6
     assert call(scratch_bytes=2 * 8160 * 3072 - 2) == 7   # half the scratch must hold one image's rows
+
+
+def test_binding_checks_tensors_before_the_library_sees_them():
+    """The library gets bare pointers and one row count: the binding rejects tensors whose width, layout,
+    element type or device the library could not check, and folds the table sizes into that count."""
+    imgs = workloads.random_small_batch(7, 3, max_side=90)
+    params = mimo.make_params()
+    host = mimo.pack_images(imgs, device="cpu")
+    _, offs = mimo.plan_batch(host.heights, host.widths, params)
+    total = int(offs[-1])
+    with pytest.raises(ValueError, match="shape"):
+        mimo.preprocess_batch_host_noalloc(params, host, torch.empty((total, 768)))
+    with pytest.raises(ValueError, match="contiguous"):
+        mimo.preprocess_batch_host_noalloc(params, host, torch.empty((1536, total)).t())
+    with pytest.raises(ValueError, match="dtype"):
+        mimo.preprocess_batch_host_noalloc(params, host, torch.empty((total, 1536), dtype=torch.float16))
+    with pytest.raises(ValueError, match="int32"):
+        mimo.preprocess_batch_host_noalloc(params, host, torch.empty((total, 1536)),
+                                           torch.empty(total, dtype=torch.int64))
+    # a table shorter than the rows lowers the row count the library is given (MIMO_ECAPACITY there)
+    out = torch.empty((total, 1536))
+    assert mimo._row_capacity(out, "out", host=True) == total
+    assert mimo._row_capacity(out, "out", host=True, perm=torch.empty(total - 1, dtype=torch.int32)) == total - 1
+    # device entry points take device tensors only
+    with pytest.raises(ValueError, match="CUDA"):
+        mimo.preprocess_batch(params, host, torch.empty((total, 1536)))
+    with pytest.raises(ValueError, match="CUDA"):
+        mimo.patch_embed(torch.empty((4, 1536), dtype=torch.bfloat16), torch.empty((256, 1536), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="shape"):
+        mimo.patch_embed(torch.empty((4, 1500), dtype=torch.bfloat16), torch.empty((256, 1536), dtype=torch.bfloat16))

@@ -49,3 +49,11 @@ def test_algorithmic_bytes_of_c5():
     assert nb["write_rows"] == 12_834_570_240
     assert nb["write_perm"] == 8_355_840
     assert nb["total"] == 14_700_871_680
+
+
+def test_l2_note_states_whether_inputs_outgrow_l2():
+    # the default batch: 1.86 GB of uint8 inputs, 12.8 GB of fp32 rows
+    assert "larger than L2" in bench.l2_note(1_857_945_600, 12_842_926_080)
+    # 16 RGBA 480x640 images: 19.7 MB of inputs, below the L2 size
+    note = bench.l2_note(16 * 480 * 640 * 4, 19_200 * 6_144)
+    assert "smaller than the 126 MB L2" in note and "19.7 MB" in note

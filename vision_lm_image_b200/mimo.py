@@ -14,6 +14,7 @@ permutation (docs.rs "cortiq_engine::mimo_vision", column_permutation).
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -159,6 +160,72 @@ def _check(status: int, what: str = ""):
         raise MimoError(status, what)
 
 
+def _tensor(t, name: str, device=None, dtype=None, cols: int | None = None, host: bool = False):
+    """Checks a tensor that goes to the library as a bare pointer.
+
+    The library sees only the address and a count, so what it cannot see is
+    checked here: dense layout, element type, the row width and the device
+    (a CUDA tensor on ``device``, or a host tensor with ``host``). One
+    combined test on the common path; the message is worked out on failure."""
+    if (not t.is_contiguous() or (dtype is not None and t.dtype != dtype)
+            or (cols is not None and (t.dim() != 2 or t.shape[1] != cols)) or t.is_cuda == host
+            or (device is not None and t.get_device() != device.index)):
+        _tensor_error(t, name, device, dtype, cols, host)
+
+
+def _tensor_error(t, name, device, dtype, cols, host):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if cols is not None and (t.dim() != 2 or t.shape[1] != cols):
+        raise ValueError(f"{name} must have shape [rows, {cols}], got {tuple(t.shape)}")
+    if host:
+        raise ValueError(f"{name} must be a host tensor, got {t.device}")
+    raise ValueError(f"{name} must be a CUDA tensor on {device if device is not None else 'a CUDA device'}, "
+                     f"got {t.device}")
+
+
+_DTYPES = None  # (float32, bfloat16, int32, uint8), looked up once
+
+
+def _dtypes():
+    global _DTYPES
+    if _DTYPES is None:
+        import torch
+
+        _DTYPES = (torch.float32, torch.bfloat16, torch.int32, torch.uint8)
+    return _DTYPES
+
+
+def _row_capacity(out, name: str, device=None, host: bool = False, perm=None, positions=None, window=None) -> int:
+    """Rows the output tensors can hold: the pixel rows' count, lowered to what
+    the permutation (1 per row), positions (2 per row) and window index (1 per
+    4 rows) hold, so that the library's capacity check covers all of them."""
+    f32, bf16, i32, _ = _DTYPES or _dtypes()
+    if out.dtype is not f32 and out.dtype is not bf16:
+        raise ValueError(f"unsupported output dtype {out.dtype}")
+    _tensor(out, name, device, cols=ROW_WIDTH, host=host)
+    cap = out.shape[0]
+    if perm is not None:
+        _tensor(perm, "perm", device, i32, host=host)
+        cap = min(cap, perm.numel())
+    if positions is not None:
+        _tensor(positions, "positions", device, i32)
+        cap = min(cap, positions.numel() // 2)
+    if window is not None:
+        _tensor(window, "window", device, i32)
+        cap = min(cap, window.numel() * 4)
+    return cap
+
+
+def _packed_buffer(packed: "PackedBatch", device=None, host: bool = False):
+    """The packed images' buffer, checked as a uint8 tensor on ``device`` (or the host)."""
+    buf = packed.buffer
+    _tensor(buf, "packed.buffer", device, (_DTYPES or _dtypes())[3], host=host)
+    return buf
+
+
 # ----------------------------------------------------------------- knobs
 def make_params(mean=None, std=None, min_pixels: int | None = None, max_pixels: int | None = None,
                 patch_size: int = 16, temporal_patch_size: int = 2, merge_size: int = 2) -> MimoParams:
@@ -296,6 +363,14 @@ def pack_images(images, device="cpu", pin_memory: bool = False) -> PackedBatch:
 
 
 # ----------------------------------------------------------------- device path
+def _on_stream(stream):
+    """Context that makes ``stream`` (when given) torch's current stream, so that the packing
+    copies and allocations of a high-level call are ordered with its library call."""
+    import torch
+
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
 def _stream_handle(stream, device):
     import torch
 
@@ -306,11 +381,12 @@ def _stream_handle(stream, device):
 
 def preprocess_batch(params: MimoParams, packed: PackedBatch, out, perm=None, stream=None) -> None:
     """Raw ABI call on device buffers (``packed.buffer``, ``out`` and ``perm`` on the same CUDA device)."""
-    buf = packed.buffer
+    buf = _packed_buffer(packed)
+    cap = _row_capacity(out, "out", buf.device, perm=perm)
     st = lib().mimo_preprocess_batch(
         ctypes.byref(params), packed.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
         *packed.ptrs, _dtype_code(out.dtype), ctypes.c_void_p(out.data_ptr()),
-        out.shape[0] if out.ndim == 2 else 0, ctypes.c_void_p(perm.data_ptr() if perm is not None else 0),
+        cap, ctypes.c_void_p(perm.data_ptr() if perm is not None else 0),
         _stream_handle(stream, buf.device))
     _check(st, "preprocess_batch")
 
@@ -328,12 +404,12 @@ def _dtype_code(dtype) -> int:
 def preprocess_batch_ex(params: MimoParams, packed: PackedBatch, out, perm=None, positions=None, window=None,
                         order: str = "merge", stream=None) -> None:
     """Raw ABI call of mimo_preprocess_batch_ex: row order and the optional index tables (device tensors)."""
-    buf = packed.buffer
+    buf = _packed_buffer(packed)
     o = MimoOutputs()
     o.out_dtype = _dtype_code(out.dtype)
     o.row_order = {"merge": ORDER_MERGE, "column": ORDER_COLUMN}[order]
     o.d_out = out.data_ptr()
-    o.out_rows_capacity = out.shape[0] if out.ndim == 2 else 0
+    o.out_rows_capacity = _row_capacity(out, "out", buf.device, perm=perm, positions=positions, window=window)
     o.d_column_perm = perm.data_ptr() if perm is not None else None
     o.d_positions = positions.data_ptr() if positions is not None else None
     o.d_window_index = window.data_ptr() if window is not None else None
@@ -363,14 +439,15 @@ def preprocess(images, mean=None, std=None, min_pixels: int | None = None, max_p
     if dev.type != "cuda":
         raise ValueError("the MiMo preprocessing library runs on CUDA devices only")
     params = make_params(mean, std, min_pixels, max_pixels)
-    packed = pack_images(images, device=dev)
-    grid, offs = plan_batch(packed.heights, packed.widths, params)
-    total = int(offs[-1])
-    out = torch.empty((total, ROW_WIDTH), dtype=dtype, device=dev)
-    perm = torch.empty(total, dtype=torch.int32, device=dev) if column_perm else None
-    pos = torch.empty((total, 2), dtype=torch.int32, device=dev) if positions else None
-    win = torch.empty(total // 4, dtype=torch.int32, device=dev) if window_index else None
-    preprocess_batch_ex(params, packed, out, perm, pos, win, order, stream)
+    with _on_stream(stream):
+        packed = pack_images(images, device=dev)
+        grid, offs = plan_batch(packed.heights, packed.widths, params)
+        total = int(offs[-1])
+        out = torch.empty((total, ROW_WIDTH), dtype=dtype, device=dev)
+        perm = torch.empty(total, dtype=torch.int32, device=dev) if column_perm else None
+        pos = torch.empty((total, 2), dtype=torch.int32, device=dev) if positions else None
+        win = torch.empty(total // 4, dtype=torch.int32, device=dev) if window_index else None
+        preprocess_batch_ex(params, packed, out, perm, pos, win, order, stream)
     if positions or window_index:
         return out, torch.from_numpy(grid), perm, pos, win
     return out, torch.from_numpy(grid), perm
@@ -414,11 +491,14 @@ def preprocess_video_raw(params: MimoParams, d_frames, n_frames: int, frame_stri
                          channels: int, out, total_max_pixels: int = 0, perm=None, positions=None, window=None,
                          order: str = "merge", stream=None) -> None:
     """Raw ABI call of mimo_preprocess_video on frames already in device memory (uint8 tensor)."""
+    import torch
+
+    _tensor(d_frames, "d_frames", dtype=torch.uint8)
     o = MimoOutputs()
     o.out_dtype = _dtype_code(out.dtype)
     o.row_order = {"merge": ORDER_MERGE, "column": ORDER_COLUMN}[order]
     o.d_out = out.data_ptr()
-    o.out_rows_capacity = out.shape[0]
+    o.out_rows_capacity = _row_capacity(out, "out", d_frames.device, perm=perm, positions=positions, window=window)
     o.d_column_perm = perm.data_ptr() if perm is not None else None
     o.d_positions = positions.data_ptr() if positions is not None else None
     o.d_window_index = window.data_ptr() if window is not None else None
@@ -448,24 +528,15 @@ def preprocess_video(frames, mean=None, std=None, min_pixels: int | None = None,
     n, H, W, C = (int(v) for v in t.shape)
     frame_bytes = H * W * C
     stride = (frame_bytes + ALIGN - 1) // ALIGN * ALIGN
-    buf = torch.zeros(n * stride, dtype=torch.uint8, device=dev)
-    buf.view(n, stride)[:, :frame_bytes].copy_(t.reshape(n, frame_bytes), non_blocking=True)
-    grid, rows = plan_video(n, H, W, total_max_pixels, params)
-    out = torch.empty((rows, ROW_WIDTH), dtype=dtype, device=dev)
-    perm = torch.empty(rows, dtype=torch.int32, device=dev) if column_perm else None
-    pos = torch.empty((rows, 2), dtype=torch.int32, device=dev) if positions else None
-    win = torch.empty(rows // 4, dtype=torch.int32, device=dev) if window_index else None
-    o = MimoOutputs()
-    o.out_dtype = _dtype_code(dtype)
-    o.row_order = {"merge": ORDER_MERGE, "column": ORDER_COLUMN}[order]
-    o.d_out = out.data_ptr()
-    o.out_rows_capacity = rows
-    o.d_column_perm = perm.data_ptr() if perm is not None else None
-    o.d_positions = pos.data_ptr() if pos is not None else None
-    o.d_window_index = win.data_ptr() if win is not None else None
-    _check(lib().mimo_preprocess_video(ctypes.byref(params), n, ctypes.c_void_p(buf.data_ptr()), buf.numel(), stride,
-                                       H, W, C, total_max_pixels, ctypes.byref(o), _stream_handle(stream, dev)),
-           "preprocess_video")
+    with _on_stream(stream):
+        buf = torch.zeros(n * stride, dtype=torch.uint8, device=dev)
+        buf.view(n, stride)[:, :frame_bytes].copy_(t.reshape(n, frame_bytes), non_blocking=True)
+        grid, rows = plan_video(n, H, W, total_max_pixels, params)
+        out = torch.empty((rows, ROW_WIDTH), dtype=dtype, device=dev)
+        perm = torch.empty(rows, dtype=torch.int32, device=dev) if column_perm else None
+        pos = torch.empty((rows, 2), dtype=torch.int32, device=dev) if positions else None
+        win = torch.empty(rows // 4, dtype=torch.int32, device=dev) if window_index else None
+        preprocess_video_raw(params, buf, n, stride, H, W, C, out, total_max_pixels, perm, pos, win, order, stream)
     g = torch.from_numpy(grid.reshape(1, 3))
     if positions or window_index:
         return out, g, perm, pos, win
@@ -487,14 +558,23 @@ def patch_embed(rows, weight, bias=None, out_dtype=None, out=None, error=None, s
     import torch
 
     out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
-    if rows.dtype != torch.bfloat16 or weight.dtype != torch.bfloat16:
-        raise ValueError("rows and weight must be bfloat16")
+    _tensor(rows, "rows", dtype=torch.bfloat16, cols=ROW_WIDTH)
+    dev = rows.device
+    _tensor(weight, "weight", dev, torch.bfloat16, cols=ROW_WIDTH)
     M = rows.shape[0]
     N = weight.shape[0]
+    if bias is not None:
+        _tensor(bias, "bias", dev, torch.float32)
+        if bias.numel() != N:
+            raise ValueError(f"bias must hold {N} values, got {bias.numel()}")
     if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=rows.device)
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    _tensor(out, "out", dev, cols=N)
+    if int(out.shape[0]) != M:
+        raise ValueError(f"out must have {M} rows, got {out.shape[0]}")
     if error is None:
-        error = torch.zeros(1, dtype=torch.int32, device=rows.device)
+        error = torch.zeros(1, dtype=torch.int32, device=dev)
+    _tensor(error, "error", dev, torch.int32)
     _check(lib().mimo_patch_embed(ctypes.c_void_p(rows.data_ptr()), M, ctypes.c_void_p(weight.data_ptr()), N,
                                   ctypes.c_void_p(bias.data_ptr() if bias is not None else 0), _dtype_code(out.dtype),
                                   ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(error.data_ptr()),
@@ -508,8 +588,8 @@ def patch_embed(rows, weight, bias=None, out_dtype=None, out=None, error=None, s
 
 
 def preprocess_embed(images, weight, bias=None, mean=None, std=None, min_pixels: int | None = None,
-                     max_pixels: int | None = None, out_dtype=None, order: str = "merge", scratch_bytes: int = 192 << 20,
-                     scratch=None, device="cuda", stream=None, check: bool = True):
+                     max_pixels: int | None = None, out_dtype=None, order: str = "merge",
+                     scratch_bytes: int = 192 << 20, scratch=None, device="cuda", stream=None, check: bool = True):
     """Pixel path + patch embedding chunk by chunk: returns (embeddings [rows, embed_dim], image_grid_thw)."""
     import torch
 
@@ -517,27 +597,33 @@ def preprocess_embed(images, weight, bias=None, mean=None, std=None, min_pixels:
     dev = torch.device(device)
     if dev.type != "cuda":
         raise ValueError("the MiMo preprocessing library runs on CUDA devices only")
-    if weight.dtype != torch.bfloat16:
-        raise ValueError("weight must be bfloat16")
-    params = make_params(mean, std, min_pixels, max_pixels)
-    packed = pack_images(images, device=dev) if not isinstance(images, PackedBatch) else images
-    grid, offs = plan_batch(packed.heights, packed.widths, params)
-    total = int(offs[-1])
+    if dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    _tensor(weight, "weight", dev, torch.bfloat16, cols=ROW_WIDTH)
     N = weight.shape[0]
-    out = torch.empty((total, N), dtype=out_dtype, device=dev)
-    if scratch is None:
-        scratch = torch.empty(scratch_bytes, dtype=torch.uint8, device=dev)
-    err = torch.zeros(1, dtype=torch.int32, device=dev)
-    order_code = {"merge": ORDER_MERGE, "column": ORDER_COLUMN}[order]
-    _check(lib().mimo_preprocess_embed(ctypes.byref(params), packed.n, ctypes.c_void_p(packed.buffer.data_ptr()),
-                                       packed.buffer.numel(), packed.offsets.ctypes.data, packed.heights.ctypes.data,
-                                       packed.widths.ctypes.data, packed.channels.ctypes.data, order_code,
-                                       ctypes.c_void_p(weight.data_ptr()), N,
-                                       ctypes.c_void_p(bias.data_ptr() if bias is not None else 0),
-                                       _dtype_code(out_dtype), ctypes.c_void_p(out.data_ptr()), total,
-                                       ctypes.c_void_p(scratch.data_ptr()), scratch.numel(),
-                                       ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, dev)),
-           "preprocess_embed")
+    if bias is not None:
+        _tensor(bias, "bias", dev, torch.float32)
+        if bias.numel() != N:
+            raise ValueError(f"bias must hold {N} values, got {bias.numel()}")
+    params = make_params(mean, std, min_pixels, max_pixels)
+    with _on_stream(stream):
+        packed = pack_images(images, device=dev) if not isinstance(images, PackedBatch) else images
+        _packed_buffer(packed, dev)
+        grid, offs = plan_batch(packed.heights, packed.widths, params)
+        total = int(offs[-1])
+        out = torch.empty((total, N), dtype=out_dtype, device=dev)
+        if scratch is None:
+            scratch = torch.empty(scratch_bytes, dtype=torch.uint8, device=dev)
+        _tensor(scratch, "scratch", dev, torch.uint8)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        order_code = {"merge": ORDER_MERGE, "column": ORDER_COLUMN}[order]
+        st = lib().mimo_preprocess_embed(
+            ctypes.byref(params), packed.n, ctypes.c_void_p(packed.buffer.data_ptr()), packed.buffer.numel(),
+            *packed.ptrs, order_code, ctypes.c_void_p(weight.data_ptr()), N,
+            ctypes.c_void_p(bias.data_ptr() if bias is not None else 0), _dtype_code(out_dtype),
+            ctypes.c_void_p(out.data_ptr()), total, ctypes.c_void_p(scratch.data_ptr()), scratch.numel(),
+            ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, dev))
+        _check(st, "preprocess_embed")
     if check:
         (torch.cuda.current_stream(dev) if stream is None else stream).synchronize()
         code = int(err.item())
@@ -551,14 +637,23 @@ def preprocess_batch_host(params: MimoParams, packed_host: PackedBatch, out_host
                           out_stage, perm_stage=None, stream=None) -> None:
     """Raw ABI call of mimo_preprocess_batch_host: host input and output buffers (pinned for full
     bandwidth), caller-provided device staging buffers. Returns when ``out_host`` is filled."""
-    buf = packed_host.buffer
+    import torch
+
+    buf = _packed_buffer(packed_host, host=True)
+    cap = _row_capacity(out_host, "out_host", host=True, perm=perm_host)
+    _tensor(src_stage, "src_stage", dtype=torch.uint8)
+    if out_stage.dtype != out_host.dtype:
+        raise ValueError("out_stage and out_host must have the same dtype")
+    # the permutation is staged only when it is asked for
+    stage_cap = _row_capacity(out_stage, "out_stage", src_stage.device,
+                              perm=perm_stage if perm_host is not None else None)
     st = lib().mimo_preprocess_batch_host(
         ctypes.byref(params), packed_host.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
         packed_host.offsets.ctypes.data, packed_host.heights.ctypes.data, packed_host.widths.ctypes.data,
         packed_host.channels.ctypes.data, _dtype_code(out_host.dtype), ctypes.c_void_p(out_host.data_ptr()),
-        out_host.shape[0], ctypes.c_void_p(perm_host.data_ptr() if perm_host is not None else 0),
+        cap, ctypes.c_void_p(perm_host.data_ptr() if perm_host is not None else 0),
         ctypes.c_void_p(src_stage.data_ptr()), src_stage.numel(), ctypes.c_void_p(out_stage.data_ptr()),
-        out_stage.shape[0], ctypes.c_void_p(perm_stage.data_ptr() if perm_stage is not None else 0),
+        stage_cap, ctypes.c_void_p(perm_stage.data_ptr() if perm_stage is not None else 0),
         _stream_handle(stream, src_stage.device))
     _check(st, "preprocess_batch_host")
 
@@ -569,11 +664,12 @@ def preprocess_batch_host_noalloc(params: MimoParams, packed_host: PackedBatch, 
     cannot allocate device memory. Runs on the current CUDA device; returns when ``out_host`` is filled."""
     import torch
 
-    buf = packed_host.buffer
+    buf = _packed_buffer(packed_host, host=True)
+    cap = _row_capacity(out_host, "out_host", host=True, perm=perm_host)
     st = lib().mimo_preprocess_batch_host_noalloc(
         ctypes.byref(params), packed_host.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
         packed_host.offsets.ctypes.data, packed_host.heights.ctypes.data, packed_host.widths.ctypes.data,
         packed_host.channels.ctypes.data, _dtype_code(out_host.dtype), ctypes.c_void_p(out_host.data_ptr()),
-        out_host.shape[0], ctypes.c_void_p(perm_host.data_ptr() if perm_host is not None else 0),
+        cap, ctypes.c_void_p(perm_host.data_ptr() if perm_host is not None else 0),
         _stream_handle(stream, torch.device("cuda", torch.cuda.current_device())))
     _check(st, "preprocess_batch_host_noalloc")
