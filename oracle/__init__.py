@@ -25,6 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lib = None
+_lib_override = None  # another build of oracle.c, set by load_build()
 _lock = threading.Lock()
 
 OK, EINVAL, EASPECT, EDEGENERATE, ECAPACITY, ENOMEM = range(6)
@@ -43,12 +44,22 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def load_build(path: str | None) -> None:
+    """Test hook: later calls run the oracle compiled at ``path`` (None: the
+    default build of oracle.c). The mutation check of the pins uses it to run
+    copies of oracle.c with planted mistakes; the arithmetic here is unchanged."""
+    global _lib, _lib_override
+    with _lock:
+        _lib = None
+        _lib_override = path
+
+
 def lib():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            L = ctypes.CDLL(_LIB_PATH)
+            path = _lib_override if _lib_override is not None else build()
+            L = ctypes.CDLL(path)
             L.oracle_smart_resize.argtypes = [_i64, _i64, _i64, _i64, _i64,
                                               ctypes.POINTER(_i64), ctypes.POINTER(_i64)]
             L.oracle_smart_resize.restype = ctypes.c_int
