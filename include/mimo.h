@@ -21,11 +21,16 @@
  *
  * Conventions for every entry point:
  *   - Return value: a mimo_status (0 = MIMO_OK). Every argument problem the
- *     host can see is reported before anything is launched or copied; the
- *     device code contains no traps and no waits.
+ *     host can see is reported before anything is launched or copied. The
+ *     device code contains no traps. The pixel kernels contain no waits. The
+ *     patch-embedding kernel's waits are bounded and report through d_error.
  *   - Ownership: the caller owns every buffer. The library never allocates
- *     or frees device memory at run time. Apart from the fixed staging area
- *     of mimo_preprocess_batch_host_noalloc it keeps no state between calls.
+ *     or frees device memory at run time. Between calls it keeps:
+ *       - the fixed staging area of mimo_preprocess_batch_host_noalloc;
+ *       - the second stream and events of mimo_preprocess_embed, per host
+ *         thread and device;
+ *       - cached device attributes (SM count, occupancy, shared-memory
+ *         opt-in).
  *   - "d_" pointers are device pointers, "h_" pointers host pointers; the
  *     other arrays (sizes, offsets) are host arrays read during the call.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
@@ -203,9 +208,9 @@ int mimo_preprocess_batch_ex(const mimo_params *p, int32_t n,
  * out_dtype; d_perm_stage >= total_rows int32 when h_column_perm is not
  * NULL), so the call allocates nothing. Host buffers should be page-locked
  * for full copy bandwidth. The batch is cut into chunks of images whose
- * upload, kernel and download overlap on the caller's stream plus library-
- * created streams that live only for the call. Synchronous: returns after
- * the last copy to h_out has completed.
+ * upload, kernel and download overlap on two library-created streams that
+ * live only for the call, ordered after the work already on the caller's
+ * stream. Synchronous: returns after the last copy to h_out has completed.
  */
 int mimo_preprocess_batch_host(const mimo_params *p, int32_t n,
                                const uint8_t *h_src, size_t src_bytes, const int64_t *src_offsets,
@@ -324,7 +329,10 @@ int mimo_preprocess_video(const mimo_params *p, int32_t n_frames, const uint8_t 
  *   d_error:  device int32, read after the stream synchronises: 0, or a
  *             nonzero code if the kernel gave up waiting on its own pipeline
  *             (its output is then incomplete). The call does not clear it.
- * All pointers 16-byte aligned (MIMO_EALIGN). Asynchronous on `stream`.
+ * d_rows, d_weight, d_bias and d_out 16-byte aligned, d_error 4-byte aligned
+ * (MIMO_EALIGN). An embed_dim that is not a positive multiple of 256 is
+ * MIMO_EINVAL; rows above 2^31 - 1 is MIMO_EOVERFLOW (the tensor-map
+ * coordinates are 32-bit). Asynchronous on `stream`.
  */
 int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int32_t embed_dim,
                      const float *d_bias, int32_t out_dtype, void *d_out, int32_t *d_error, void *stream);
