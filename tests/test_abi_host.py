@@ -43,11 +43,54 @@ def test_library_exports_every_declared_symbol():
     assert set(mimo.EXPORTED) == names
 
 
+def header_enum_values():
+    text = open(os.path.join(ROOT, "include", "mimo.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return {k: int(v) for k, v in re.findall(r"\b(MIMO_[A-Z0-9_]+)\s*=\s*(\d+)", text)}
+
+
 def test_version_and_status_strings():
     L = mimo.lib()
     assert L.mimo_version() >= 10000
-    for s in range(11):
+    statuses = {k: v for k, v in header_enum_values().items() if k == "MIMO_OK" or k.startswith("MIMO_E")}
+    for s in statuses.values():
         assert L.mimo_status_string(s) and L.mimo_status_string(s) != b"unknown status"
+    assert L.mimo_status_string(max(statuses.values()) + 1) == b"unknown status"
+
+
+def test_binding_constants_match_the_header():
+    enums = header_enum_values()
+    assert {v: k for k, v in enums.items() if k == "MIMO_OK" or k.startswith("MIMO_E")} == mimo.STATUS_NAMES
+    assert (enums["MIMO_F32"], enums["MIMO_BF16"]) == (mimo.F32, mimo.BF16)
+    assert (enums["MIMO_ORDER_MERGE"], enums["MIMO_ORDER_COLUMN"]) == (mimo.ORDER_MERGE, mimo.ORDER_COLUMN)
+    text = open(os.path.join(ROOT, "include", "mimo.h")).read()
+    m = re.search(r"#define MIMO_NOALLOC_STAGING_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == mimo.NOALLOC_STAGING_BYTES
+
+
+def test_ctypes_structs_match_the_c_layout(tmp_path):
+    """The binding's ctypes mirrors of mimo_params and mimo_outputs have the C compiler's sizes and offsets."""
+    structs = {"mimo_params": mimo.MimoParams, "mimo_outputs": mimo.MimoOutputs}
+    lines = ["#include <stddef.h>", "#include <stdio.h>", '#include "mimo.h"', "int main(void) {"]
+    for cname, cls in structs.items():
+        lines.append(f'    printf("{cname} sizeof %zu\\n", sizeof({cname}));')
+        for field, _ in cls._fields_:
+            lines.append(f'    printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    lines += ["    return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    import subprocess
+
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = {}
+    for line in subprocess.check_output([str(exe)], text=True).splitlines():
+        cname, field, value = line.split()
+        got[(cname, field)] = int(value)
+    for cname, cls in structs.items():
+        assert got[(cname, "sizeof")] == ctypes.sizeof(cls), cname
+        for field, _ in cls._fields_:
+            assert got[(cname, field)] == getattr(cls, field).offset, (cname, field)
 
 
 def test_defaults_match_processor_constructor():
