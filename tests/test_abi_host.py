@@ -344,3 +344,46 @@ def test_binding_checks_tensors_before_the_library_sees_them():
         mimo.patch_embed(torch.empty((4, 1536), dtype=torch.bfloat16), torch.empty((256, 1536), dtype=torch.bfloat16))
     with pytest.raises(ValueError, match="shape"):
         mimo.patch_embed(torch.empty((4, 1500), dtype=torch.bfloat16), torch.empty((256, 1536), dtype=torch.bfloat16))
+
+
+def header_prototypes():
+    """name -> list of parameter C types, from the prototypes in include/mimo.h."""
+    text = open(os.path.join(ROOT, "include", "mimo.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = {}
+    for ret, name, params in re.findall(r"\b(int|void|const char \*)\s*(mimo_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", text):
+        ps = [" ".join(p.split()) for p in params.split(",") if p.strip() and p.strip() != "void"]
+        protos[name] = ps
+    return protos
+
+
+def _category(c_param: str) -> str:
+    if "*" in c_param:
+        return "pointer"
+    base = c_param.replace("const ", "").split()[0]
+    return {"int32_t": "i32", "int64_t": "i64", "size_t": "size", "double": "f64", "int": "i32"}[base]
+
+
+def _ctypes_category(t) -> str:
+    if t is ctypes.c_void_p or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "pointer"
+    if t is ctypes.c_size_t:
+        return "size"
+    if t is ctypes.c_double:
+        return "f64"
+    if t in (ctypes.c_int32, ctypes.c_int):
+        return "i32"
+    if t is ctypes.c_int64:
+        return "i64"
+    raise AssertionError(f"unexpected ctypes type {t}")
+
+
+def test_binding_argtypes_match_the_prototypes():
+    """Every exported function's ctypes argument list has the header prototype's count, order and widths."""
+    protos = header_prototypes()
+    assert set(mimo.EXPORTED) <= set(protos)
+    L = mimo.lib()
+    for name in mimo.EXPORTED:
+        want = [_category(p) for p in protos[name]]
+        got = [_ctypes_category(t) for t in getattr(L, name).argtypes]
+        assert got == want, (name, got, want)
