@@ -353,7 +353,7 @@ def header_prototypes():
     protos = {}
     for ret, name, params in re.findall(r"\b(int|void|const char \*)\s*(mimo_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", text):
         ps = [" ".join(p.split()) for p in params.split(",") if p.strip() and p.strip() != "void"]
-        protos[name] = ps
+        protos[name] = (ret.strip(), ps)
     return protos
 
 
@@ -383,7 +383,10 @@ def test_binding_argtypes_match_the_prototypes():
     protos = header_prototypes()
     assert set(mimo.EXPORTED) <= set(protos)
     L = mimo.lib()
+    restypes = {"int": ctypes.c_int, "void": None, "const char *": ctypes.c_char_p}
     for name in mimo.EXPORTED:
-        want = [_category(p) for p in protos[name]]
+        ret, params = protos[name]
+        want = [_category(p) for p in params]
         got = [_ctypes_category(t) for t in getattr(L, name).argtypes]
         assert got == want, (name, got, want)
+        assert getattr(L, name).restype is restypes[ret], (name, ret)
