@@ -206,6 +206,19 @@ def cpu_baseline(w, sample_images: int, threads: int, min_seconds: float = 0.0):
             return done / dt, dt
 
 
+def image_cpu_baseline(w, n_img: int, cores: int, min_seconds: float = 10.0, single_seconds: float = 5.0) -> dict:
+    """The oracle on `cores` host threads over the first 64 images (the reported baseline), plus a
+    single-threaded figure over the first 8."""
+    sample_n = max(1, min(n_img, 64))
+    v, dt = cpu_baseline(w, sample_n, cores, min_seconds=min_seconds)
+    single_n = max(1, min(n_img, 8))
+    v1, dt1 = cpu_baseline(w, single_n, 1, min_seconds=single_seconds)
+    return {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"first {sample_n} of the {n_img} workload images, passes repeated for {dt:.1f} s",
+            "single_thread": {"value": v1, "unit": UNIT, "cores": 1,
+                              "sample": f"first {single_n} images, passes repeated for {dt1:.1f} s"}}
+
+
 def host_cores() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -574,11 +587,7 @@ def run_ours(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cores = host_cores()
-        sample_n = max(1, min(n_img, 64))
-        v, dt = cpu_baseline(w, sample_n, cores, min_seconds=10.0)
-        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": f"first {sample_n} of the {n_img} workload images, passes repeated for {dt:.1f} s"}
+        cpu = image_cpu_baseline(w, n_img, host_cores())
 
     if dist is not None:
         dist.barrier()

@@ -57,3 +57,12 @@ def test_l2_note_states_whether_inputs_outgrow_l2():
     # 16 RGBA 480x640 images: 19.7 MB of inputs, below the L2 size
     note = bench.l2_note(16 * 480 * 640 * 4, 19_200 * 6_144)
     assert "smaller than the 126 MB L2" in note and "19.7 MB" in note
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    import workloads
+
+    cpu = bench.image_cpu_baseline(workloads.workload("c1"), 1, 2, min_seconds=0.0, single_seconds=0.0)
+    assert cpu["kind"] == "oracle" and cpu["cores"] == 2 and cpu["value"] > 0
+    assert cpu["single_thread"]["cores"] == 1 and cpu["single_thread"]["value"] > 0
+    assert cpu["unit"] == cpu["single_thread"]["unit"] == bench.UNIT
