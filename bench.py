@@ -206,6 +206,18 @@ def cpu_baseline(w, sample_images: int, threads: int, min_seconds: float = 0.0):
             return done / dt, dt
 
 
+def dominant_kernel(grid, heights, widths, out_dtype: str) -> str:
+    """The pixel kernel an image launch runs, by the library's dispatch rule: the unstaged
+    direct_kernel when every width is kept and either the rows are bf16 or every height is kept too,
+    else the staged preprocess_kernel."""
+    import numpy as np
+
+    grid = np.asarray(grid)
+    widths_kept = bool(np.all(grid[:, 2] * 16 == np.asarray(widths)))
+    heights_kept = bool(np.all(grid[:, 1] * 16 == np.asarray(heights)))
+    return "direct_kernel" if widths_kept and (out_dtype == "bf16" or heights_kept) else "preprocess_kernel"
+
+
 def image_cpu_baseline(w, n_img: int, cores: int, min_seconds: float = 10.0, single_seconds: float = 5.0) -> dict:
     """The oracle on `cores` host threads over the first 64 images (the reported baseline), plus a
     single-threaded figure over the first 8."""
@@ -606,7 +618,8 @@ def run_ours(args, rank, world, local_rank):
                          "frac": achieved / peak, "peak_kind": peak_kind,
                          "traffic": ncu_traffic(args.workload, out_dtype),
                          "algorithmic_bytes_per_launch": nbytes["total"] // launches_per_step,
-                         "kernel": "preprocess_kernel", "avg_launch_ms": avg_launch_ms},
+                         "kernel": dominant_kernel(grid, host.heights, host.widths, out_dtype),
+                         "avg_launch_ms": avg_launch_ms},
             "gpu_launches": K * launches_per_step,
             "clocks": clocks.summary(),
             "e2e": e2e,

@@ -66,3 +66,19 @@ def test_cpu_baseline_reports_all_cores_and_one_thread():
     assert cpu["kind"] == "oracle" and cpu["cores"] == 2 and cpu["value"] > 0
     assert cpu["single_thread"]["cores"] == 1 and cpu["single_thread"]["value"] > 0
     assert cpu["unit"] == cpu["single_thread"]["unit"] == bench.UNIT
+
+
+def test_dominant_kernel_follows_the_dispatch_rule():
+    import workloads
+    from vision_lm_image_b200 import mimo
+
+    def kernel(name, dtype):
+        w = workloads.workload(name)
+        host = mimo.pack_images(w["images"][:8], device="cpu")
+        grid, _ = mimo.plan_batch(host.heights, host.widths, mimo.make_params(w["mean"], w["std"]))
+        return bench.dominant_kernel(grid, host.heights, host.widths, dtype)
+
+    assert kernel("c5", "f32") == "preprocess_kernel"   # 1080 -> 1088 rows: heights resized
+    assert kernel("c5", "bf16") == "direct_kernel"      # widths kept, bf16 rows
+    assert kernel("c2", "f32") == "direct_kernel"       # identity resize
+    assert kernel("c3", "f32") == "preprocess_kernel"   # widths resized
