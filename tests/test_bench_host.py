@@ -73,7 +73,7 @@ def test_dominant_kernel_follows_the_dispatch_rule():
     from vision_lm_image_b200 import mimo
 
     def kernel(name, dtype):
-        w = workloads.workload(name)
+        w = workloads.workload(name, n_images=8 if name == "c5" else None)
         host = mimo.pack_images(w["images"][:8], device="cpu")
         grid, _ = mimo.plan_batch(host.heights, host.widths, mimo.make_params(w["mean"], w["std"]))
         return bench.dominant_kernel(grid, host.heights, host.widths, dtype)
