@@ -10,6 +10,7 @@ not a crash.
 """
 import json
 import os
+import shutil
 import subprocess
 import sys
 
@@ -111,7 +112,19 @@ MUTANTS = [
     ("bias_dropped", "double acc = bias ? bias[n] : 0.0;", "double acc = 0.0;"),
 ]
 
+# the same for the Python half of the oracle (oracle/__init__.py): batch assembly and bf16 rounding
+PY_SRC = os.path.join(ROOT, "oracle", "__init__.py")
+PY_MUTANTS = [
+    ("pymod_perm_offset_in_units", "            row0 += gh * gw\n", "            row0 += (gh * gw) // 4\n"),
+    ("pymod_window_offset_in_rows", "        unit0 += (gh // merge) * (gw // merge)\n", "        unit0 += gh * gw\n"),
+    ("pymod_positions_always_merge_order", "rotary_positions(gh, gw, merge, column_order=(order == \"column\"))",
+     "rotary_positions(gh, gw, merge, column_order=False)"),
+    ("pymod_no_flatten", "            flat.extend(item)\n", "            flat.append(item)\n"),
+    ("pymod_bf16_ties_up", "    rounding = 0x7FFF + ((bits >> 16) & 1)\n", "    rounding = 0x8000 + 0 * bits\n"),
+]
+
 CONTROL = "control"
+PY_CONTROL = "pymod_control"
 
 # Readings that no pin fixes ("parity unpinned"): their mutants are expected to pass every pin. Strict, so
 # that a new pin which catches one shows up here.
@@ -123,6 +136,9 @@ UNPINNED = {
 
 @pytest.fixture(scope="module")
 def results(tmp_path_factory):
+    # the runner tells the two kinds apart by the name's prefix
+    assert not any(n.startswith("pymod_") for n, _, _ in MUTANTS)
+    assert all(n.startswith("pymod_") for n, _, _ in PY_MUTANTS)
     src = open(SRC).read()
     d = tmp_path_factory.mktemp("oracle_mutants")
     builds = [(CONTROL, src)]
@@ -136,8 +152,21 @@ def results(tmp_path_factory):
         procs.append(subprocess.Popen(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", str(d / f"{name}.so"),
                                        str(c), "-lm"]))
     assert all(p.wait() == 0 for p in procs)
+    # Python mutants: a copy of the oracle package with one changed line, built from the control library
+    py_src = open(PY_SRC).read()
+    py_builds = [(PY_CONTROL, py_src)]
+    for name, old, new in PY_MUTANTS:
+        assert py_src.count(old) == 1, f"{name}: the text to mutate must occur once in oracle/__init__.py"
+        py_builds.append((name, py_src.replace(old, new)))
+    for name, text in py_builds:
+        pkg = d / name / "oracle"
+        pkg.mkdir(parents=True)
+        (pkg / "__init__.py").write_text(text)
+        shutil.copy(SRC, pkg / "oracle.c")
+        shutil.copy(d / f"{CONTROL}.so", pkg / "liboracle.so")  # newer than oracle.c: not rebuilt
     r = subprocess.run([sys.executable, os.path.join(ROOT, "tests", "_oracle_mutation_runner.py"), str(d),
-                        *[n for n, _ in builds]], cwd=ROOT, capture_output=True, text=True, timeout=900)
+                        *[n for n, _ in builds], *[n for n, _ in py_builds]],
+                       cwd=ROOT, capture_output=True, text=True, timeout=900)
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("RESULTS ")]
     assert r.returncode == 0 and lines, r.stdout[-3000:] + r.stderr[-3000:]
     return json.loads(lines[-1][len("RESULTS "):])
@@ -145,11 +174,12 @@ def results(tmp_path_factory):
 
 def test_unmodified_copy_passes_every_pin(results):
     assert results[CONTROL] == 0
+    assert results[PY_CONTROL] == 0
 
 
 @pytest.mark.parametrize("name", [
     pytest.param(m[0], marks=pytest.mark.xfail(strict=True, reason=UNPINNED[m[0]])) if m[0] in UNPINNED else m[0]
-    for m in MUTANTS])
+    for m in MUTANTS + PY_MUTANTS])
 def test_pins_catch_planted_mistake(results, name):
     # pytest exit code 1: a pin failed (0 would mean the mistake went unnoticed)
     assert results[name] == 1, f"planted mistake '{name}' passed every pin (exit code {results[name]})"
