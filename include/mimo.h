@@ -116,8 +116,8 @@ int mimo_smart_resize(int64_t height, int64_t width, int64_t factor,
 
 /*
  * get_number_of_image_patches (processing page): grid_h * grid_w of the
- * resized image, before the merge_size**2 reduction (vision tokens =
- * *out_patches / 4). Host only.
+ * resized image, counted before each merge_size**2 patches merge into one
+ * token (vision tokens = *out_patches / 4). Host only.
  */
 int mimo_num_patches(int64_t height, int64_t width, const mimo_params *p, int64_t *out_patches);
 
@@ -278,8 +278,9 @@ int mimo_expand_prompt_ids(const int32_t *ids, int64_t n_ids, int32_t pad_id,
  * mimo_video_max_pixels: per-frame pixel ceiling for n sampled frames,
  *   max(min_pixels, min(total_max_pixels * temporal_patch_size // n,
  *   max_pixels)); total_max_pixels = 0 means no overall budget (max_pixels).
- * mimo_smart_nframes: total / fps_src * fps, clamped to [min_frames,
- *   max_frames] and to total, floored to even; MIMO_EINVAL if that is 0.
+ * mimo_smart_nframes: the number of frames to sample: total / fps_src * fps,
+ *   kept inside [min_frames, max_frames] and no larger than total, then
+ *   rounded down to an even number; MIMO_EINVAL if that leaves 0.
  * mimo_sample_frames: idx = unique(int64(linspace(0, total - 1, n))) and
  *   ts = float32(idx) / fps_src; idx and ts hold n entries, *count gets the
  *   number of distinct indices written.

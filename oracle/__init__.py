@@ -2,9 +2,9 @@
 
 A plain, slow restatement of what the path computes (``oracle.c``, fp64),
 plus the batch assembly of ``MimoV2ImageProcessor.__call__`` (NeMo Automodel,
-"mimo_v2_flash.processing", class MimoV2ImageProcessor: nested input is
-flattened one level, per-image patch rows are concatenated, ``image_grid_thw``
-is ``[n, 3]``).
+"mimo_v2_flash.processing", class MimoV2ImageProcessor: a list of
+per-sample lists is unpacked by one level, the images' patch rows are
+stacked in order, and ``image_grid_thw`` is ``[n, 3]``).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package. The product library

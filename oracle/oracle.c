@@ -61,10 +61,12 @@ static double py_round(double v)
 
 /*
  * [P] smart_resize / [C] smart_resize.
- * Same algorithm as the HF (Qwen2-VL) smart_resize except:
- *   - a short side below `factor` is first scaled up to `factor` (both sides
- *     scaled by the same ratio), and that branch skips the aspect guard;
- *   - a zero side produced by the max_pixels shrink is an error, not clamped.
+ * The HF (Qwen2-VL) smart_resize with two differences:
+ *   - when the shorter side is under `factor`, both sides are first scaled by
+ *     one ratio that brings it to exactly `factor`, and no aspect guard
+ *     applies on that path;
+ *   - when the max_pixels shrink floors a side to zero, that is an error
+ *     rather than a value clamped up to `factor`.
  * HF algorithm as used here: aspect guard max/min > 200 is an error; round each
  * side to the nearest multiple of factor; if the area is above max_pixels,
  * shrink by beta = sqrt(h*w/max_pixels) and floor to the factor; else if the
@@ -171,8 +173,8 @@ static void axis_taps(int64_t d, int64_t in, int64_t out, int64_t *i0, int64_t *
 /*
  * [P] class doc: F.interpolate(mode="bilinear", align_corners=False), no
  * antialias; [C] resize_bilinear: the same on a planar [c][h][w] image, taps
- * taken along W on the two source rows first, then along H. No rounding back
- * to 8 bits. One plane, fp64.
+ * blended horizontally inside each of the two source rows, then those two
+ * results blended vertically. No rounding back to 8 bits. One plane, fp64.
  */
 void oracle_resize_plane(const double *in, int64_t in_h, int64_t in_w,
                          double *out, int64_t out_h, int64_t out_w)
@@ -205,10 +207,10 @@ void oracle_normalize_planes(double *planes, int64_t HW, const double mean[3], c
 }
 
 /*
- * [C] conventions: the image becomes T identical frames (T = temporal patch
- * size); each patch row is the Conv3d kernel flattened as (c, tt, py, px);
- * rows are in merge-block order (t, block row, block col, mh, mw). [P] class
- * doc: "emit patches in the Qwen2VL merge-block order".
+ * [C] conventions, [P] class doc: one image stands for T identical frames
+ * (T = temporal patch size). A patch row holds the values one Conv3d window
+ * sees, in (c, tt, py, px) order, and the rows follow Qwen2-VL's merge-block
+ * order (t, block row, block col, mh, mw).
  * planes: normalised [3, Hr, Wr]; out: [grid_t*grid_h*grid_w, 3*T*p*p] fp32.
  */
 void oracle_patchify(const double *planes, int64_t Hr, int64_t Wr,
@@ -336,10 +338,11 @@ int oracle_patch_value(const uint8_t *src, int64_t H, int64_t W, int32_t C,
 }
 
 /*
- * [C] column_permutation: row permutation into column order. Merge units are
- * listed by (t, block col, block row); the m*m rows of a unit stay together;
- * perm[dst] = src. Indices are offset by row0 (the image's first row in a
- * batch), so they index the concatenated batch directly.
+ * [C] column_permutation: the permutation that puts the rows into column
+ * order. It visits merge units by (t, block col, block row) and keeps the m*m
+ * rows of each unit adjacent and in their own order; perm[dst] = src.
+ * Indices are offset by row0 (the image's first row in a batch), so they
+ * index the concatenated batch directly.
  */
 void oracle_column_permutation(int64_t grid_t, int64_t grid_h, int64_t grid_w,
                                int32_t merge, int64_t row0, int32_t *perm)
@@ -354,10 +357,9 @@ void oracle_column_permutation(int64_t grid_t, int64_t grid_h, int64_t grid_w,
 }
 
 /*
- * [C] conventions: "whole merge units are listed by (t, block col, block
- * row)" -- the same rows as oracle_patchify, emitted in column order: units
- * by (t, block col, block row), the m*m rows of a unit kept together in
- * (mh, mw) order. Equals the merge-order rows gathered with
+ * [C] conventions, column order: the rows of oracle_patchify, with whole
+ * merge units visited by (t, block col, block row) and the m*m rows of each
+ * unit adjacent in (mh, mw) order. Equals the merge-order rows gathered with
  * oracle_column_permutation.
  */
 void oracle_patchify_column(const double *planes, int64_t Hr, int64_t Wr,
@@ -389,8 +391,8 @@ void oracle_patchify_column(const double *planes, int64_t Hr, int64_t Wr,
  * MiMoVisionRotaryEmbedding: two-dimensional frequencies): for every patch
  * row, its patch row index and patch column index in the grid, in the order
  * the rows are emitted (merge-block order, or column order when
- * column_order != 0, [C] conventions: "the RoPE tables are permuted the same
- * way"). pos has 2 entries per row: (h, w).
+ * column_order != 0: [C] conventions, the rotary tables follow the rows'
+ * permutation). pos has 2 entries per row: (h, w).
  */
 void oracle_rotary_positions(int64_t grid_t, int64_t grid_h, int64_t grid_w, int32_t merge,
                              int32_t column_order, int32_t *pos)
@@ -473,9 +475,10 @@ int64_t oracle_video_max_pixels(int64_t n_sampled, int64_t total_max, int32_t te
 }
 
 /*
- * [C] smart_nframes: total / fps_src * fps, clamped to [min_frames,
- * max_frames] and to total, floored to even. A result of 0 frames is an
- * error (OR_EINVAL), as is a non-positive count or rate.
+ * [C] smart_nframes: the number of frames to sample. Start from
+ * total / fps_src * fps, keep it inside [min_frames, max_frames] and no
+ * larger than total, then round it down to an even number. A result of 0
+ * frames is an error (OR_EINVAL), as is a non-positive count or rate.
  */
 int oracle_smart_nframes(int64_t total, double fps_src, double fps, int64_t min_frames, int64_t max_frames,
                          int64_t *out)
@@ -578,7 +581,7 @@ int oracle_preprocess_video(const uint8_t *frames, int64_t n, int64_t frame_stri
                             for (int64_t tt = 0; tt < T; ++tt) {
                                 int64_t f = t * T + tt;
                                 if (f > n - 1)
-                                    f = n - 1; /* even padding: repeat the last frame */
+                                    f = n - 1; /* an odd count reuses its final frame */
                                 const double *pl = resized + f * 3 * Hr * Wr + c * Hr * Wr;
                                 for (int64_t py = 0; py < p; ++py)
                                     for (int64_t px = 0; px < p; ++px, ++col) {

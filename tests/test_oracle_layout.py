@@ -1,9 +1,9 @@
 """Pins for the oracle's whole path, row layout and column permutation.
 
-The patch layout is stated on docs.rs 'cortiq_engine::mimo_vision' (conventions list): T = 2 identical
-frames, rows flattened as (c, tt, py, px), rows in merge-block order (t, block row, block col, mh, mw);
-column_permutation lists merge units by (t, block col, block row) with each unit's m*m rows kept
-together, perm[dst] = src. Here that layout is re-expressed independently with torch reshape/permute
+The patch layout comes from docs.rs 'cortiq_engine::mimo_vision' (conventions list). There are
+T = 2 identical frames. A row holds its values in (c, tt, py, px) order, and rows follow the
+merge-block order (t, block row, block col, mh, mw). column_permutation visits merge units by
+(t, block col, block row), keeps each unit's m*m rows adjacent, and maps perm[dst] = src. Here that layout is re-expressed independently with torch reshape/permute
 on planes produced by PIL compositing and torch's F.interpolate (the routines the NeMo Automodel
 'mimo_v2_flash.processing' page names), and compared with the oracle's loop nest.
 """

@@ -425,7 +425,7 @@ def preprocess(images, mean=None, std=None, min_pixels: int | None = None, max_p
     """The processor call on the GPU: returns (pixel_values, image_grid_thw, perm | None).
 
     ``images``: HWC uint8 numpy arrays or torch tensors (CPU or CUDA), RGB or
-    RGBA, or a list of such lists (flattened one level). ``pixel_values`` is a
+    RGBA, or a list of such lists (unpacked by one level). ``pixel_values`` is a
     CUDA tensor [total_patches, 1536] (float32 by default, bfloat16 on
     request); ``image_grid_thw`` a CPU int64 tensor [n, 3]. ``order="column"``
     emits the rows in column order. With ``positions`` or ``window_index`` the
