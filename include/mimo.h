@@ -102,7 +102,9 @@ void mimo_params_default(mimo_params *p);
  * smart_resize (processing page, function smart_resize; cortiq page,
  * smart_resize). Resized (height, width), both multiples of `factor`:
  *  - a side below `factor` first scales both sides so the short side equals
- *    `factor`; that branch skips the aspect guard;
+ *    `factor` and the long side becomes floor(long * factor / short), the
+ *    integer sizes the MiMo processor (sglang semantics) continues with; that
+ *    branch skips the aspect guard;
  *  - otherwise long/short > 200 -> MIMO_EASPECT;
  *  - each side rounds to the nearest multiple of factor (exact halves to
  *    even); an area above max_pixels shrinks by sqrt(area/max_pixels) with

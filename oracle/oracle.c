@@ -29,11 +29,13 @@
  * in full before the next one starts, in the order the processor page lists
  * them.
  *
- * Parity pins live in tests/test_oracle_*.py. One reading is NOT pinned by
- * anything outside this file ("parity unpinned"): in the sub-factor upscale
- * branch of smart_resize, the long side scaled by a non-integer ratio is kept
- * as an unrounded fp64 value (long * factor / short). Every case whose scaled
- * long side is an integer is pinned by closed forms.
+ * Parity pins live in tests/test_oracle_*.py: closed forms, brute force,
+ * invariants and library routines (transformers' Qwen2-VL smart_resize, PIL,
+ * torch F.interpolate / conv3d, numpy). The one reading the pages leave open,
+ * whether the long side scaled in the sub-factor upscale branch of
+ * smart_resize is truncated to an integer, follows the MiMo-V2 processor of
+ * the same serving lineage that is installed as a library (vLLM's MiMo-V2
+ * Omni processor): it truncates, and the pins call it.
  */
 #include <math.h>
 #include <stdint.h>
@@ -71,6 +73,10 @@ static double py_round(double v)
  * side to the nearest multiple of factor; if the area is above max_pixels,
  * shrink by beta = sqrt(h*w/max_pixels) and floor to the factor; else if the
  * area is below min_pixels, grow by beta = sqrt(min_pixels/(h*w)) and ceil.
+ * The page names the sglang MiMoProcessor semantics for the upscale branch;
+ * in that processor lineage the scaled long side is an integer, the float
+ * quotient long*factor/short truncated (Python int()), and the later steps
+ * run on the upscaled integer sizes.
  */
 int oracle_smart_resize(int64_t height, int64_t width, int64_t factor,
                         int64_t min_pixels, int64_t max_pixels,
@@ -84,12 +90,13 @@ int oracle_smart_resize(int64_t height, int64_t width, int64_t factor,
     double f = (double)factor;
 
     if (height < factor || width < factor) {
-        /* upscale branch: the short side becomes exactly `factor` */
+        /* upscale branch: the short side becomes exactly `factor`, the long
+           side the truncated quotient long * factor / short */
         if (height <= width) {
-            w = (double)(width * factor) / (double)height;
+            w = trunc((double)(width * factor) / (double)height);
             h = f;
         } else {
-            h = (double)(height * factor) / (double)width;
+            h = trunc((double)(height * factor) / (double)width);
             w = f;
         }
     } else {

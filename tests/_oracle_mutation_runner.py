@@ -28,7 +28,7 @@ PY_PREFIX = "pymod_"  # names of Python-package mutants
 
 PIN_FILES = [os.path.join(ROOT, "tests", f) for f in (
     "test_oracle_geometry.py", "test_oracle_layout.py", "test_oracle_pixels.py", "test_oracle_tables.py",
-    "test_oracle_video.py")]
+    "test_oracle_video.py", "test_oracle_library_pins.py")]
 
 
 def run_pins() -> int:

@@ -27,8 +27,8 @@ MUTANTS = [
     ("max_branch_ceil", "h_bar = floor(h / beta / f) * f;", "h_bar = ceil(h / beta / f) * f;"),
     ("min_branch_floor", "w_bar = ceil(w * beta / f) * f;", "w_bar = floor(w * beta / f) * f;"),
     ("no_upscale_branch", "if (height < factor || width < factor) {", "if (0) {"),
-    ("upscale_long_side_rounded", "w = (double)(width * factor) / (double)height;",
-     "w = floor((double)(width * factor) / (double)height);"),
+    ("upscale_long_side_unrounded", "w = trunc((double)(width * factor) / (double)height);",
+     "w = (double)(width * factor) / (double)height;"),
     ("max_branch_on_original_size", "double beta = sqrt((h * w) / (double)max_pixels);",
      "double beta = sqrt((h_bar * w_bar) / (double)max_pixels);"),
     # RGBA onto white
@@ -128,10 +128,7 @@ PY_CONTROL = "pymod_control"
 
 # Readings that no pin fixes ("parity unpinned"): their mutants are expected to pass every pin. Strict, so
 # that a new pin which catches one shows up here.
-UNPINNED = {
-    "upscale_long_side_rounded": "the pages leave open whether the long side scaled in the sub-factor "
-                                 "upscale branch is rounded; every pinned case scales to an integer",
-}
+UNPINNED: dict[str, str] = {}
 
 
 @pytest.fixture(scope="module")

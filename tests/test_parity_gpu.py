@@ -191,6 +191,22 @@ def test_extreme_shapes():
     check_against_oracle(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
 
 
+def test_sub_factor_shapes_with_truncated_long_side():
+    # sub-factor shapes whose upscaled long side is not an integer: the truncating reading of smart_resize
+    # gives other grids here than keeping the fraction would (e.g. 7x8 -> 96x96, not 96x128)
+    rng = workloads.rng_for(8)
+    shapes = [(7, 8), (13, 41), (7, 22), (31, 3984), (3984, 31), (13, 15), (17, 77), (21, 95), (8, 7), (41, 13),
+              (31, 140), (5, 1234)]
+    imgs = [workloads.uniform_image(rng, h, w, 3) if i % 2 == 0 else workloads.rgba_image(rng, h, w)
+            for i, (h, w) in enumerate(shapes)]
+    check_against_oracle(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    pv, grid, _ = gpu_run(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD, dtype=torch.bfloat16)
+    ref, rgrid, _ = oracle.preprocess(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    assert np.array_equal(grid, rgrid)
+    assert [tuple(g) for g in grid[:2].tolist()] == [(1, 6, 6), (1, 4, 10)]
+    assert_bf16_close(pv, ref, "sub-factor bf16")
+
+
 def test_more_images_than_one_launch():
     # more than 512 images: the host cuts the batch into several launches
     rng = workloads.rng_for(7)

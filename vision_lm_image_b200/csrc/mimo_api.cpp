@@ -47,6 +47,9 @@ double round_ties_even(double v) {
 // smart_resize of the processing page: sub-factor upscale first (no aspect
 // guard in that branch), else the HF aspect guard; round to the factor; then
 // the max_pixels shrink (floor, zero side rejected) or min_pixels growth (ceil).
+// In the upscale branch the long side becomes the integer part of
+// long * factor / short, as the MiMo processor lineage the page names (sglang
+// MiMoProcessor semantics) computes it; the later steps use those integer sizes.
 int smart_resize_impl(int64_t height, int64_t width, int64_t factor, int64_t min_px, int64_t max_px,
                       int64_t *oh, int64_t *ow) {
     if (height <= 0 || width <= 0 || factor <= 0 || min_px < 0 || max_px <= 0 || !oh || !ow) return MIMO_EINVAL;
@@ -58,13 +61,15 @@ int smart_resize_impl(int64_t height, int64_t width, int64_t factor, int64_t min
     double h, w;
     const int64_t short_side = std::min(height, width);
     if (short_side < factor) {
-        // both sides scaled by factor/short: the short side lands exactly on the factor
+        // both sides scaled by factor/short: the short side lands exactly on the
+        // factor, the long side on the floor of the exact quotient (both operands
+        // are positive and below 2^31, so the product is exact in 64 bits)
         if (height == short_side) {
             h = f;
-            w = static_cast<double>(width * factor) / static_cast<double>(height);
+            w = static_cast<double>((width * factor) / height);
         } else {
             w = f;
-            h = static_cast<double>(height * factor) / static_cast<double>(width);
+            h = static_cast<double>((height * factor) / width);
         }
     } else {
         const double ratio = static_cast<double>(std::max(height, width)) / static_cast<double>(short_side);
