@@ -25,7 +25,10 @@ Also reported on the same JSON line:
   cpu_baseline the CPU oracle timed on a bounded sample of the same workload
                on this host's cores (rank 0, N=1 only);
   clocks       SM clock and throttle reasons sampled through NVML during the
-               timed region.
+               timed region;
+  also         (default c5 fp32 line, one GPU) the two other configurations held
+               to the bandwidth target, c5 with bf16 rows and c3 with fp32 rows,
+               each timed the same way in this process with its own roofline.
 
 --impl reference times the CPU oracle alone (rank 0; other ranks exit).
 """
@@ -63,6 +66,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-also", action="store_true",
+                    help="c5 default line: skip the c3 fp32 and c5 bf16 measurements added under 'also'")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step from a CUDA graph (the launch without the host-side call overhead)")
     return ap.parse_args()
@@ -182,6 +187,17 @@ def l2_note(input_bytes: int, output_bytes: int) -> str:
             "L2-resident; outputs %.1f MB" % (input_bytes / 1e6, output_bytes / 1e6))
 
 
+def workload_config(args, w, world: int, n_img: int, out_dtype: str, column_perm: bool, total_rows: int,
+                    input_bytes: int) -> dict:
+    """The line's config: the same keys and values on both arms (the reference arm computes the rows
+    with the oracle's geometry, this arm with the library's; the tests hold the two equal)."""
+    out_bytes = int(total_rows) * 1536 * (2 if out_dtype == "bf16" else 4) + (4 * int(total_rows) if column_perm else 0)
+    return {"workload": args.workload, "description": w["description"], "images_per_gpu": n_img,
+            "out_dtype": out_dtype, "column_perm": column_perm, "rows_per_gpu": int(total_rows),
+            "row_order": args.order, "launch": "cuda_graph" if args.graph else "api_call",
+            "l2": l2_note(input_bytes, out_bytes), "parallelism": f"dp{world}"}
+
+
 def algorithmic_bytes(packed, total_rows, dtype_bytes, perm: bool) -> dict:
     read = int(sum(int(h) * int(w) * int(c) for h, w, c in zip(packed.heights, packed.widths, packed.channels)))
     write_rows = int(total_rows) * 1536 * dtype_bytes
@@ -289,6 +305,13 @@ def run_reference(args, rank, world):
     w = workloads.workload(args.workload, n_images=args.images)
     if args.dtype:
         w["dtype"] = args.dtype
+    import oracle
+
+    oracle.build()
+    total_rows = sum(oracle.get_number_of_image_patches(im.shape[0], im.shape[1]) for im in w["images"])
+    input_bytes = sum(int(im.size) for im in w["images"])
+    config = workload_config(args, w, world, len(w["images"]), w["dtype"], bool(w["column_perm"]), total_rows,
+                             input_bytes)
     cores = host_cores()
     per_step = max(1, min(len(w["images"]), 2 * cores, 16))
     sample = f"{per_step} of the workload's {len(w['images'])} images per step, oracle on {cores} threads"
@@ -304,8 +327,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "description": w["description"], "images": len(w["images"]),
-                   "out_dtype": w["dtype"], "column_perm": w["column_perm"]},
+        "config": config,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -359,13 +381,13 @@ def run_video(args, rank, world, local_rank):
         print(json.dumps({
             "metric": METRIC + " (video frames)", "value": world * n * K / (ms * 1e-3), "unit": "frames/s",
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": out_dtype, "data": "synthetic",
             "config": {"workload": args.workload, "description": w["description"], "frames": int(n),
                        "grid_thw": [int(v) for v in grid], "out_dtype": out_dtype, "row_order": args.order,
                        "l2": l2_note(read, written)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_kind": peak_kind, "traffic": None, "algorithmic_bytes_per_launch": read + written,
-                         "kernel": "preprocess_kernel", "avg_launch_ms": ms / K},
+                         "kernel": dominant_kernel([grid], [H], [W], out_dtype), "avg_launch_ms": ms / K},
             "gpu_launches": K, "clocks": clocks.summary(), "e2e": None, "cpu_baseline": None,
         }), flush=True)
 
@@ -485,6 +507,54 @@ def run_patch_embed(args, rank, world, local_rank):
         }), flush=True)
 
 
+def also_config(args, mimo, workloads, name: str, out_dtype: str, dev, stream, scratch) -> dict:
+    """One more configuration timed like the main line (W warm-up launches, then K launches between CUDA
+    events on the launching stream), its rows written into `scratch` (the main line's output buffer,
+    reinterpreted), with its own roofline."""
+    import torch
+
+    w = workloads.workload(name)
+    tdtype = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+    dbytes = 2 if out_dtype == "bf16" else 4
+    params = mimo.make_params(w["mean"], w["std"])
+    host = mimo.pack_images(w["images"], device="cpu", pin_memory=True)
+    packed = host.to(dev)
+    grid, offs = mimo.plan_batch(host.heights, host.widths, params)
+    total = int(offs[-1])
+    flat = scratch.view(torch.uint8).view(-1)
+    need = total * 1536 * dbytes + (4 * total if w["column_perm"] else 0)
+    assert need <= flat.numel(), "scratch too small"
+    out = flat[:total * 1536 * dbytes].view(tdtype).view(total, 1536)
+    perm = flat[total * 1536 * dbytes:need].view(torch.int32) if w["column_perm"] else None
+    launches = (host.n + 511) // 512
+    for _ in range(max(args.warmup, 0)):
+        mimo.preprocess_batch_ex(params, packed, out, perm, order=args.order, stream=stream)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with ClockSampler(dev.index) as clocks:
+        ev[0].record(stream)
+        for _ in range(args.steps):
+            mimo.preprocess_batch_ex(params, packed, out, perm, order=args.order, stream=stream)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / args.steps
+    nbytes = algorithmic_bytes(host, total, dbytes, perm is not None)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = nbytes["total"] / (ms / launches * 1e-3) / 1e9
+    del packed
+    return {"workload": name, "description": w["description"], "images": host.n, "out_dtype": out_dtype,
+            "column_perm": perm is not None, "rows": total, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "value": host.n / (ms * 1e-3), "unit": UNIT,
+            "l2": l2_note(nbytes["read"], nbytes["write_rows"] + nbytes["write_perm"]),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "traffic": ncu_traffic(name, out_dtype),
+                         "algorithmic_bytes_per_launch": nbytes["total"] // launches,
+                         "kernel": dominant_kernel(grid, host.heights, host.widths, out_dtype),
+                         "avg_launch_ms": ms / launches},
+            "gpu_launches": args.steps * launches, "clocks": clocks.summary()}
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -597,6 +667,13 @@ def run_ours(args, rank, world, local_rank):
                "timing": "host wall clock around the synchronous host-to-host call"}
         del out_h, perm_h, host_e
 
+    # the other configurations held to the bandwidth target, timed in this process on one GPU
+    also = None
+    if world == 1 and args.workload == "c5" and args.dtype is None and args.images is None and not args.no_also:
+        del packed
+        also = {"c5_bf16": also_config(args, mimo, workloads, "c5", "bf16", dev, stream, out),
+                "c3_f32": also_config(args, mimo, workloads, "c3", "f32", dev, stream, out)}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = image_cpu_baseline(w, n_img, host_cores())
@@ -607,12 +684,8 @@ def run_ours(args, rank, world, local_rank):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic",
-            "config": {"workload": args.workload, "description": w["description"], "images_per_gpu": n_img,
-                       "out_dtype": out_dtype, "column_perm": perm is not None, "rows_per_gpu": total,
-                       "row_order": args.order, "launch": "cuda_graph" if args.graph else "api_call",
-                       "l2": l2_note(nbytes["read"], nbytes["write_rows"] + nbytes["write_perm"]),
-                       "parallelism": f"dp{world}"},
+            "dtype": out_dtype, "data": "synthetic",
+            "config": workload_config(args, w, world, n_img, out_dtype, perm is not None, total, nbytes["read"]),
             "output_gbs": out_gbs,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
@@ -625,6 +698,8 @@ def run_ours(args, rank, world, local_rank):
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
+        if also:
+            line["also"] = also
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

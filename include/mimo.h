@@ -241,8 +241,11 @@ int mimo_preprocess_batch_host(const mimo_params *p, int32_t n,
  *     with MIMO_ELIMIT before anything is copied or launched. With fp32 rows
  *     (24 bytes per resized pixel) an image of about 2.4 million resized
  *     pixels fits; a 1080x1920 RGBA image resized to 1088x1920 does.
- *   - The first call on a device looks the area's device address up
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call looks the area's device address up in the current
+ *     device's context (cudaGetSymbolAddress), so a device reset or a new
+ *     primary context never leaves a stale address behind. The first call on
+ *     a device may load the library's device code there; make it before any
+ *     stream capture.
  *   - Every call shares the one area and it keeps the last call's contents.
  *     Nothing in it needs to start at zero: each call writes every staged
  *     byte it reads. Calls that overlap on the GPU (from several host

@@ -82,3 +82,26 @@ def test_dominant_kernel_follows_the_dispatch_rule():
     assert kernel("c5", "bf16") == "direct_kernel"      # widths kept, bf16 rows
     assert kernel("c2", "f32") == "direct_kernel"       # identity resize
     assert kernel("c3", "f32") == "preprocess_kernel"   # widths resized
+
+
+def test_reference_arm_config_equals_the_main_arm_config():
+    # both arms print the same config for the same arguments: the reference arm computes the rows with
+    # the oracle's geometry, the main arm with the library's plan
+    import argparse
+
+    import oracle
+    import workloads
+    from vision_lm_image_b200 import mimo
+
+    for name in ("c1", "c3"):
+        args = argparse.Namespace(workload=name, order="merge", graph=False)
+        w = workloads.workload(name)
+        host = mimo.pack_images(w["images"], device="cpu")
+        _, offs = mimo.plan_batch(host.heights, host.widths, mimo.make_params(w["mean"], w["std"]))
+        read = bench.algorithmic_bytes(host, int(offs[-1]), 4, bool(w["column_perm"]))["read"]
+        ours = bench.workload_config(args, w, 1, host.n, w["dtype"], bool(w["column_perm"]), int(offs[-1]), read)
+        rows = sum(oracle.get_number_of_image_patches(im.shape[0], im.shape[1]) for im in w["images"])
+        ref = bench.workload_config(args, w, 1, len(w["images"]), w["dtype"], bool(w["column_perm"]), rows,
+                                    sum(int(im.size) for im in w["images"]))
+        assert ours == ref
+        assert set(ours) >= {"workload", "images_per_gpu", "rows_per_gpu", "row_order", "out_dtype", "l2"}

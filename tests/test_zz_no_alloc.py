@@ -6,8 +6,10 @@ fixed device array compiled into the library instead of caller-provided buffers.
 it through the C ABI and compare its rows and permutation with those of
 mimo_preprocess_batch_host, within the fp32 parity tolerance (1e-4; equality is expected, because
 both run the same kernel). There are two calls in a row: the second, smaller batch finds the first
-call's bytes still in the shared array. The file sorts last so that a run stopping at the first
-failure has already run every other test; it also passes when run alone.
+call's bytes still in the shared array, and its rows are also checked against the CPU oracle (1e-4 for
+fp32, one bf16 ulp of the rounded oracle value for bf16) and its permutation bit for bit. The file
+sorts last so that a run stopping at the first failure has already run every other test; it also
+passes when run alone.
 """
 import ctypes
 
@@ -15,17 +17,32 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
 from vision_lm_image_b200 import build, mimo
 
 pytestmark = pytest.mark.gpu
 
 FP32_ATOL = 1e-4
+BF16_ULP_FLOOR = 2.0 ** -19  # the GPU parity tests' floor on the bf16 ulp
 
 
 @pytest.fixture(scope="module", autouse=True)
 def built():
     build.build()
+    oracle.build()
+
+
+def _assert_matches_oracle(images, mean, std, got_out, got_perm, dtype):
+    ref, _, rperm = oracle.preprocess(images, mean, std, column_perm=True, threads=8)
+    assert np.array_equal(got_perm.numpy(), rperm)
+    if dtype == torch.float32:
+        assert float(np.abs(got_out.numpy().astype(np.float64) - ref).max()) <= FP32_ATOL
+    else:
+        r = oracle.bf16_bits_to_f32(oracle.round_to_bf16(ref)).astype(np.float64)
+        a = np.abs(r)
+        ulp = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(a, 1e-30))) - 7), BF16_ULP_FLOOR)
+        assert (np.abs(got_out.float().numpy().astype(np.float64) - r) <= ulp).all()
 
 
 def _host_batch(images):
@@ -68,7 +85,7 @@ def _batches():
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_noalloc_matches_host_entry_point_twice(dtype):
-    for images, mean, std in _batches():
+    for k, (images, mean, std) in enumerate(_batches()):
         params = mimo.make_params(mean, std)
         host = _host_batch(images)
         _, offs = mimo.plan_batch(host.heights, host.widths, params)
@@ -78,6 +95,8 @@ def test_noalloc_matches_host_entry_point_twice(dtype):
         assert torch.equal(got_perm, ref_perm)
         diff = (got_out.float() - ref_out.float()).abs().max().item()
         assert diff <= FP32_ATOL, diff
+        if k == 1:
+            _assert_matches_oracle(images, mean, std, got_out, got_perm, dtype)
 
 
 def test_noalloc_rejects_an_image_beyond_the_staging_size():

@@ -10,8 +10,6 @@
 // library holds MIMO_NOALLOC_STAGING_BYTES of it until the process exits.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "mimo.h"
 #include "mimo_internal.h"
 
@@ -20,25 +18,18 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_stage[MIMO_NOALLOC_STAGING_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void *g_stage_ptr[kMaxDevices] = {};
-
 }  // namespace
 
-// Device address of the staging array on the current device. In host code
-// the array's name is only a host-side handle, so the address is looked up
-// once per device, with that device current, and kept for later calls.
+// Device address of the staging array in the current device's context. In
+// host code the array's name is only a host-side handle, so the address is
+// looked up with the device current. It is looked up on every call rather
+// than cached: a cudaDeviceReset or a new primary context loads the module
+// again, and the array can then sit at another address. The lookup is a
+// runtime table query, small beside the copies of a call.
 int noalloc_staging(void **dev_ptr, size_t *bytes) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MIMO_ECUDA;
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_stage_ptr[dev] == nullptr) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_stage) != cudaSuccess || p == nullptr) return MIMO_ECUDA;
-        g_stage_ptr[dev] = p;
-    }
-    *dev_ptr = g_stage_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_stage) != cudaSuccess || p == nullptr) return MIMO_ECUDA;
+    *dev_ptr = p;
     *bytes = MIMO_NOALLOC_STAGING_BYTES;
     return MIMO_OK;
 }
