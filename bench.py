@@ -66,6 +66,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", action="store_true",
+                    help="every rank takes the same batch and runs its own merge-unit window of it "
+                         "(mimo_preprocess_units): strong scaling of one batch, images split across ranks")
     ap.add_argument("--no-also", action="store_true",
                     help="c5 default line: skip the c3 fp32 and c5 bf16 measurements added under 'also'")
     ap.add_argument("--graph", action="store_true",
@@ -195,7 +198,8 @@ def workload_config(args, w, world: int, n_img: int, out_dtype: str, column_perm
     return {"workload": args.workload, "description": w["description"], "images_per_gpu": n_img,
             "out_dtype": out_dtype, "column_perm": column_perm, "rows_per_gpu": int(total_rows),
             "row_order": args.order, "launch": "cuda_graph" if args.graph else "api_call",
-            "l2": l2_note(input_bytes, out_bytes), "parallelism": f"dp{world}"}
+            "l2": l2_note(input_bytes, out_bytes),
+            "parallelism": f"dp{world}" + (" merge-unit windows of one batch" if getattr(args, "shard", False) else "")}
 
 
 def algorithmic_bytes(packed, total_rows, dtype_bytes, perm: bool) -> dict:
@@ -577,7 +581,8 @@ def run_ours(args, rank, world, local_rank):
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    w = workloads.workload(args.workload, seed_offset=7919 * rank, n_images=args.images)
+    # weak scaling: each rank its own batch; --shard: one batch, a merge-unit window per rank
+    w = workloads.workload(args.workload, seed_offset=0 if args.shard else 7919 * rank, n_images=args.images)
     out_dtype = args.dtype or w["dtype"]
     tdtype = torch.bfloat16 if out_dtype == "bf16" else torch.float32
     dbytes = 2 if out_dtype == "bf16" else 4
@@ -586,14 +591,28 @@ def run_ours(args, rank, world, local_rank):
     packed = host.to(dev)
     grid, offs = mimo.plan_batch(host.heights, host.widths, params)
     total = int(offs[-1])
-    out = torch.empty((total, 1536), dtype=tdtype, device=dev)
+    window = None
+    if args.shard:
+        from vision_lm_image_b200 import shard
+
+        if args.order != "merge":
+            raise SystemExit("--shard runs merge order only")
+        window = shard.unit_windows(total // 4, world)[rank]
+    out_rows = 4 * window[1] if window else total
+    out = torch.empty((out_rows, 1536), dtype=tdtype, device=dev)
     perm = torch.empty(total, dtype=torch.int32, device=dev) if w["column_perm"] else None
     n_img = host.n
     launches_per_step = (n_img + 511) // 512
     stream = torch.cuda.current_stream(dev)
 
+    def launch(on=None):
+        if window:
+            mimo.preprocess_units(params, packed, window[0], window[1], out, perm, stream=on)
+        else:
+            mimo.preprocess_batch_ex(params, packed, out, perm, order=args.order, stream=on)
+
     def step():
-        mimo.preprocess_batch_ex(params, packed, out, perm, order=args.order, stream=stream)
+        launch(stream)
 
     graph = None
     if args.graph:
@@ -602,7 +621,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            mimo.preprocess_batch_ex(params, packed, out, perm, order=args.order)
+            launch()
         step = graph.replay
 
     for _ in range(max(args.warmup, 0)):
@@ -630,15 +649,29 @@ def run_ours(args, rank, world, local_rank):
     max_ms = float(t.item())
 
     nbytes = algorithmic_bytes(host, total, dbytes, perm is not None)
+    if window:
+        # this rank's share: its window's rows and permutation entries, and each touched image's bytes
+        # in proportion to the image's units inside the window
+        lo, hi = 4 * window[0], 4 * (window[0] + window[1])
+        read = 0.0
+        for i in range(n_img):
+            inside = max(0, min(hi, int(offs[i + 1])) - max(lo, int(offs[i])))
+            read += int(host.heights[i]) * int(host.widths[i]) * int(host.channels[i]) * inside / max(
+                int(offs[i + 1] - offs[i]), 1)
+        rows_w = 4 * window[1]
+        nbytes = {"read": int(read), "write_rows": rows_w * 1536 * dbytes,
+                  "write_perm": 4 * rows_w if perm is not None else 0}
+        nbytes["total"] = nbytes["read"] + nbytes["write_rows"] + nbytes["write_perm"]
     avg_launch_ms = sum(per_launch_ms) / K / launches_per_step
     peak, peak_kind = measured_hbm_peak()
     achieved = nbytes["total"] / (avg_launch_ms * 1e-3) / 1e9
-    value = world * n_img * K / (max_ms * 1e-3)
+    # whole-job images/s: every rank's own batch (weak), or the one shared batch (--shard)
+    value = (1 if window else world) * n_img * K / (max_ms * 1e-3)
     out_gbs = nbytes["write_rows"] / (max_ms / K * 1e-3) / 1e9
 
     # e2e: host images in, host rows out, through the host-buffer entry point
     e2e = None
-    if not args.no_e2e and args.e2e_steps > 0:
+    if not args.no_e2e and args.e2e_steps > 0 and not window:
         # with several ranks on one host each rank pins a 64-image prefix of its batch (the full batch
         # would pin ~15 GB of host memory per rank); images/s is per image either way
         e2e_n = n_img if world == 1 else min(n_img, 64)
@@ -669,7 +702,8 @@ def run_ours(args, rank, world, local_rank):
 
     # the other configurations held to the bandwidth target, timed in this process on one GPU
     also = None
-    if world == 1 and args.workload == "c5" and args.dtype is None and args.images is None and not args.no_also:
+    if (world == 1 and args.workload == "c5" and args.dtype is None and args.images is None and not args.no_also
+            and not args.shard):
         del packed
         also = {"c5_bf16": also_config(args, mimo, workloads, "c5", "bf16", dev, stream, out),
                 "c3_f32": also_config(args, mimo, workloads, "c3", "f32", dev, stream, out)}
@@ -683,9 +717,10 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-            "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": out_dtype, "data": "synthetic",
-            "config": workload_config(args, w, world, n_img, out_dtype, perm is not None, total, nbytes["read"]),
+            "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "strong" if window else "weak",
+            "vs_baseline": None, "dtype": out_dtype, "data": "synthetic",
+            "config": workload_config(args, w, world, n_img, out_dtype, perm is not None, total,
+                                      algorithmic_bytes(host, total, dbytes, False)["read"]),
             "output_gbs": out_gbs,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,

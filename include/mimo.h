@@ -203,6 +203,32 @@ int mimo_preprocess_batch_ex(const mimo_params *p, int32_t n,
                              const mimo_outputs *out, void *stream);
 
 /*
+ * A window of the batch's merge units, for splitting one batch (or one large
+ * image) across devices by merge-block ranges. Merge unit u of the batch is
+ * the 32x32 merge block whose 4 rows are batch rows 4u..4u+3 in merge order:
+ * units are counted over the images in batch order, and inside an image in
+ * merge-block order (block row, block col). The call runs the fused path of
+ * mimo_preprocess_batch_ex on units [first_unit, first_unit + unit_count)
+ * only, which may start and end inside an image.
+ *   - Rows: merge order only (MIMO_ORDER_COLUMN -> MIMO_EUNSUPPORTED). d_out
+ *     holds the window's rows: batch row 4u + k lands at row
+ *     4 (u - first_unit) + k of d_out; out_rows_capacity >= 4 * unit_count.
+ *     d_positions, if given, follows the rows the same way ([4 unit_count][2]).
+ *   - d_column_perm [total_rows] and d_window_index [total_rows / 4] stay
+ *     batch-global: the window writes the entries of its own units, at their
+ *     batch positions and with batch-global values, and nothing else.
+ *   - Windows that tile [0, total_rows / 4) write, between them, exactly what
+ *     one mimo_preprocess_batch_ex call over the batch writes.
+ * Errors: as mimo_preprocess_batch_ex; MIMO_EINVAL for a negative first_unit
+ * or unit_count; MIMO_ERANGE when the window reaches past the batch's units.
+ * An empty window launches nothing. Asynchronous on `stream`.
+ */
+int mimo_preprocess_units(const mimo_params *p, int32_t n,
+                          const uint8_t *d_src, size_t src_bytes, const int64_t *src_offsets,
+                          const int32_t *heights, const int32_t *widths, const int32_t *channels,
+                          int64_t first_unit, int64_t unit_count, const mimo_outputs *out, void *stream);
+
+/*
  * The same path from host memory to host memory (inputs copied in, rows and
  * permutation copied back), for callers whose images and results live on
  * the host. The caller supplies device staging buffers of at least the batch
@@ -344,6 +370,23 @@ int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int
                      const float *d_bias, int32_t out_dtype, void *d_out, int32_t *d_error, void *stream);
 
 /*
+ * Test hook for the failure path of mimo_patch_embed; no counterpart on the
+ * pages. The same launch, except that the operand loader of every CTA stops
+ * after stop_after_kblocks 64-wide K blocks of its first tile (0 ..
+ * 1536 / 64), so the tensor-core pipeline waits for operands that never
+ * arrive, and each wait gives up after wait_rounds polling rounds (> 0)
+ * instead of the default 2^20. The kernel then records a nonzero code in
+ * *d_error (1: operands, 3: accumulator; the first role to give up wins),
+ * stops every role, waits (bounded) for the copies and tensor-core work it
+ * started, frees its tensor memory and returns; d_out is left incomplete.
+ * Arguments otherwise as mimo_patch_embed (rows > 0). Asynchronous on
+ * `stream`. For tests only: no normal call reaches this path.
+ */
+int mimo_patch_embed_stall_test(const void *d_rows, int64_t rows, const void *d_weight, int32_t embed_dim,
+                                const float *d_bias, int32_t out_dtype, void *d_out, int32_t *d_error,
+                                int32_t stop_after_kblocks, uint32_t wait_rounds, void *stream);
+
+/*
  * The pixel path followed by the patch embedding, image run by image run
  * (vision page, MiMoVisionTransformer.forward: patch rows -> patch embed).
  * Images are grouped into runs whose bf16 patch rows fit half of d_scratch;
@@ -380,6 +423,19 @@ const char *mimo_status_string(int status);
 
 /* Library ABI version (major*10000 + minor*100 + patch). */
 int mimo_version(void);
+
+/*
+ * Debug builds only (compiled with -DMIMO_BOUNDS_CHECK; no counterpart on the
+ * pages): the number of accesses of the pixel kernels that failed their bounds
+ * check since the last query, and the kind of the first (1: staged source copy
+ * outside the caller's buffer, 2: direct source load outside the image, 3:
+ * shared-memory tile index, 4: output row outside the validated rows, 5:
+ * permutation / position / window entry outside its table). A failed check
+ * skips its access and never traps. The query synchronises with the device's
+ * earlier work and clears both values. Release builds return
+ * MIMO_EUNSUPPORTED.
+ */
+int mimo_bounds_check_status(int64_t *violations, int32_t *first_kind);
 
 #ifdef __cplusplus
 }

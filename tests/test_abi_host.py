@@ -361,7 +361,8 @@ def _category(c_param: str) -> str:
     if "*" in c_param:
         return "pointer"
     base = c_param.replace("const ", "").split()[0]
-    return {"int32_t": "i32", "int64_t": "i64", "size_t": "size", "double": "f64", "int": "i32"}[base]
+    return {"int32_t": "i32", "uint32_t": "u32", "int64_t": "i64", "size_t": "size", "double": "f64",
+            "int": "i32"}[base]
 
 
 def _ctypes_category(t) -> str:
@@ -373,6 +374,8 @@ def _ctypes_category(t) -> str:
         return "f64"
     if t in (ctypes.c_int32, ctypes.c_int):
         return "i32"
+    if t is ctypes.c_uint32:
+        return "u32"
     if t is ctypes.c_int64:
         return "i64"
     raise AssertionError(f"unexpected ctypes type {t}")

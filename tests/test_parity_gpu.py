@@ -608,3 +608,118 @@ def _unpack(packed):
     buf = packed.buffer.numpy()
     return [buf[o:o + h * w * c].reshape(h, w, c)
             for o, h, w, c in zip(packed.offsets, packed.heights, packed.widths, packed.channels)]
+
+
+# ---------------------------------------------------------------- merge-unit windows (multi-device split)
+def _full_and_windows(images, mean, std, dtype, windows):
+    """One mimo_preprocess_batch_ex call over the batch, and the same batch as unit windows."""
+    params = mimo.make_params(mean, std)
+    packed = mimo.pack_images(images, device="cuda")
+    _, offs = mimo.plan_batch(packed.heights, packed.widths, params)
+    total = int(offs[-1])
+    ref = torch.empty((total, 1536), dtype=dtype, device="cuda")
+    rperm = torch.empty(total, dtype=torch.int32, device="cuda")
+    rpos = torch.empty((total, 2), dtype=torch.int32, device="cuda")
+    rwin = torch.empty(total // 4, dtype=torch.int32, device="cuda")
+    mimo.preprocess_batch_ex(params, packed, ref, rperm, rpos, rwin)
+    perm = torch.full((total,), -1, dtype=torch.int32, device="cuda")
+    win = torch.full((total // 4,), -1, dtype=torch.int32, device="cuda")
+    parts, pos_parts = [], []
+    for first, count in windows:
+        out = torch.full((4 * count, 1536), float("nan"), dtype=dtype, device="cuda")
+        pos = torch.full((4 * count, 2), -1, dtype=torch.int32, device="cuda")
+        mimo.preprocess_units(params, packed, first, count, out, perm, pos, win)
+        parts.append(out)
+        pos_parts.append(pos)
+    torch.cuda.synchronize()
+    return (ref, rperm, rpos, rwin), (torch.cat(parts), perm, torch.cat(pos_parts), win), total
+
+
+@pytest.mark.parametrize("split", ["halves", "ragged"])
+def test_unit_windows_reproduce_one_large_image(split):
+    # c4: one 4096x4096 image (8100 merge units) cut by merge-block ranges, staged kernel
+    w = workloads.workload("c4")
+    windows = [(0, 4050), (4050, 4050)] if split == "halves" else [(0, 1), (1, 89), (90, 3911), (4001, 4099)]
+    (ref, rperm, rpos, rwin), (got, perm, pos, win), total = _full_and_windows(
+        w["images"], w["mean"], w["std"], torch.float32, windows)
+    assert total == 32400
+    assert torch.equal(got, ref)
+    assert torch.equal(perm, rperm) and torch.equal(pos, rpos) and torch.equal(win, rwin)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_unit_windows_random_batches_both_kernels(dtype):
+    rng = np.random.Generator(np.random.PCG64(61))
+    # resized batch (staged kernel) and a kept-width batch (unstaged kernel in bf16)
+    batches = [workloads.random_small_batch(62, 11, max_side=300, min_side=1), _kept_width_batch(
+        [(96, 128, 3), (200, 64, 4), (130, 96, 3), (64, 160, 4)], 63)]
+    for images in batches:
+        params = mimo.make_params(workloads.CLIP_MEAN, workloads.CLIP_STD)
+        hs = [im.shape[0] for im in images]
+        ws = [im.shape[1] for im in images]
+        units = int(mimo.plan_batch(hs, ws, params)[1][-1]) // 4
+        cuts = sorted(set(int(c) for c in rng.integers(1, units, size=4)))
+        bounds = [0] + cuts + [units]
+        windows = [(bounds[k], bounds[k + 1] - bounds[k]) for k in range(len(bounds) - 1)]
+        (ref, rperm, rpos, rwin), (got, perm, pos, win), _ = _full_and_windows(
+            images, workloads.CLIP_MEAN, workloads.CLIP_STD, dtype, windows)
+        assert torch.equal(got, ref)
+        assert torch.equal(perm, rperm) and torch.equal(pos, rpos) and torch.equal(win, rwin)
+    # the last batch's rows against the oracle too (one bf16 ulp / 1e-4)
+    oref, _, operm = oracle.preprocess(images, workloads.CLIP_MEAN, workloads.CLIP_STD, column_perm=True)
+    assert np.array_equal(perm.cpu().numpy(), operm)
+    if dtype == torch.float32:
+        assert_fp32_close(got.cpu().numpy(), oref, "windows")
+    else:
+        assert_bf16_close(got, oref, "windows")
+
+
+def test_unit_windows_errors():
+    w = workloads.workload("c1")
+    params = mimo.make_params(w["mean"], w["std"])
+    packed = mimo.pack_images(w["images"], device="cuda")
+    out = torch.empty((48, 1536), dtype=torch.float32, device="cuda")
+    with pytest.raises(mimo.MimoError) as e:   # the image has 12 units
+        mimo.preprocess_units(params, packed, 10, 3, out)
+    assert e.value.status == 10
+    with pytest.raises(mimo.MimoError) as e:   # 8 rows of room for 3 units
+        mimo.preprocess_units(params, packed, 0, 3, out[:8])
+    assert e.value.status == 7
+    o = mimo.MimoOutputs()
+    o.out_dtype, o.row_order, o.d_out, o.out_rows_capacity = mimo.F32, mimo.ORDER_COLUMN, out.data_ptr(), 48
+    buf = packed.buffer
+    st = mimo.lib().mimo_preprocess_units(ctypes.byref(params), packed.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
+                                          *packed.ptrs, 0, 12, ctypes.byref(o), None)
+    assert st == 5  # column order is not offered for windows
+    mimo.preprocess_units(params, packed, 3, 0, out)  # an empty window launches nothing
+
+
+# ---------------------------------------------------------------- failure path of the tensor-core kernel
+def test_patch_embed_wait_runs_out_and_the_next_launch_is_correct():
+    """The operand loader stops after 3 of the 24 K blocks and every wait gives up after 2^14 polling
+    rounds: the kernel must return with a nonzero status word (operands or accumulator never came), not
+    hang; a normal launch right after must be correct, so the failed launch gave its tensor memory back."""
+    M, N = 1024, 512
+    g = torch.Generator(device="cpu").manual_seed(91)
+    rows = torch.randn((M, 1536), generator=g).to(torch.bfloat16).cuda()
+    w = (torch.randn((N, 1536), generator=g) * 0.02).to(torch.bfloat16).cuda()
+    out = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    st = mimo.lib().mimo_patch_embed_stall_test(
+        ctypes.c_void_p(rows.data_ptr()), M, ctypes.c_void_p(w.data_ptr()), N, None, mimo.BF16,
+        ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(err.data_ptr()), 3, 1 << 14,
+        ctypes.c_void_p(stream.cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    assert int(err.item()) in (1, 3), int(err.item())
+    # bad hook arguments are rejected on the host
+    for stop, rounds in ((-1, 100), (25, 100), (3, 0)):
+        assert mimo.lib().mimo_patch_embed_stall_test(
+            ctypes.c_void_p(rows.data_ptr()), M, ctypes.c_void_p(w.data_ptr()), N, None, mimo.BF16,
+            ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(err.data_ptr()), stop, rounds, None) == 1
+    # the next normal launches on the same device are complete and correct
+    for out_dtype in (torch.bfloat16, torch.float32):
+        emb = mimo.patch_embed(rows, w, out_dtype=out_dtype)
+        ref, scale = _embed_ref(rows, w, None)
+        _assert_embed_close(emb, ref, scale, "after a stalled launch")

@@ -78,3 +78,66 @@ def test_lpt_properties():
     assert shard.lpt_assign([], 4) == [[], [], [], []]
     with pytest.raises(ValueError):
         shard.lpt_assign([1], 0)
+
+
+def _window_worker(rank, world, port, sizes, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        windows, grid, offs = shard.window_plan([h for h, _ in sizes], [w for _, w in sizes], world)
+        first, count = windows[rank]
+        gathered = [None] * world
+        dist.all_gather_object(gathered, (rank, first, count, offs.tolist(),
+                                          shard.window_images(offs, first, count)))
+        q.put(gathered if rank == 0 else None)
+    finally:
+        dist.destroy_process_group()
+
+
+def _run_ranks(target, world, sizes):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=target, args=(r, world, port, sizes, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = None
+    for _ in range(world):
+        item = q.get(timeout=120)
+        if item is not None:
+            res = item
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return res
+
+
+@pytest.mark.parametrize("sizes", [[(4096, 4096)], [(1080, 1920), (4096, 4096), (16, 192), (640, 480)]])
+def test_unit_windows_two_ranks_gloo(sizes):
+    # one huge image (or a batch dominated by one): the two ranks split it by merge-block ranges
+    build.build()
+    world = 2
+    res = _run_ranks(_window_worker, world, sizes)
+    assert res is not None and res[0][3] == res[1][3]
+    units = res[0][3][-1] // 4
+    covered = np.zeros(units, np.int64)
+    for _, first, count, _, _ in res:
+        covered[first:first + count] += 1
+    assert (covered == 1).all()  # every merge unit exactly once
+    counts = [c for _, _, c, _, _ in res]
+    assert max(counts) - min(counts) <= 1  # balanced within one merge unit
+    # the largest image is shared between the ranks
+    offs = np.array(res[0][3])
+    big = int(np.argmax(np.diff(offs)))
+    assert all(big in imgs for *_, imgs in res)
+
+
+def test_unit_windows_properties():
+    for total in (0, 1, 7, 8100, 522240):
+        for world in (1, 2, 3, 8):
+            w = shard.unit_windows(total, world)
+            assert w[0][0] == 0 and sum(c for _, c in w) == total
+            assert all(w[r][0] + w[r][1] == w[r + 1][0] for r in range(world - 1))
+            assert max(c for _, c in w) - min(c for _, c in w) <= 1
+    with pytest.raises(ValueError):
+        shard.unit_windows(5, 0)

@@ -231,25 +231,50 @@ struct Tables {
     int32_t *win = nullptr;
 };
 
+// A window of merge units: units [lo, hi) of the batch, counted over the images
+// in batch order and in merge order inside each image (unit u holds batch rows
+// 4u..4u+3 in merge order). Emitted rows (and their rotary positions) land
+// `row_shift` rows before their batch row; the permutation and the window
+// index stay batch-global.
+struct UnitWindow {
+    int64_t lo = 0, hi = std::numeric_limits<int64_t>::max();
+    int64_t row_shift = 0;
+};
+
 int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_t last, const uint8_t *d_src,
                  size_t src_bytes, const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
                  const int32_t *channels, int32_t out_dtype, void *d_out, int32_t *d_perm, void *stream,
-                 const Tables &tables = Tables(), int64_t row_base = 0) {
+                 const Tables &tables = Tables(), int64_t row_base = 0, const UnitWindow &win = UnitWindow()) {
     static thread_local mimo::LaunchParams lp;  // 31 KB: kept off the stack
+    // units of image i inside the window: [lo_i, hi_i) of its own units
+    auto unit_span = [&](int32_t i, int64_t *lo_i, int64_t *hi_i) {
+        const int64_t u0 = v.plan.row0[i] / 4;
+        *lo_i = std::max<int64_t>(win.lo - u0, 0);
+        *hi_i = std::min<int64_t>(win.hi - u0, v.plan.img[i].blocks);
+        return *hi_i > *lo_i;
+    };
+    // emitted rows land row_shift rows early: shift the row and position bases (addresses only; every
+    // row the window writes lies at or after row_shift)
+    const uintptr_t out_base = reinterpret_cast<uintptr_t>(d_out) -
+                               static_cast<uintptr_t>(win.row_shift) * mimo::kRowWidth * (out_dtype == MIMO_BF16 ? 2u : 4u);
+    const uintptr_t pos_base = reinterpret_cast<uintptr_t>(tables.pos) -
+                               static_cast<uintptr_t>(win.row_shift) * 2u * sizeof(int32_t);
     int32_t i = first;
+    int64_t lo_i = 0, hi_i = 0;
+    while (i < last && !unit_span(i, &lo_i, &hi_i)) ++i;
     while (i < last) {
         std::memset(&lp, 0, sizeof(lp));
         lp.src = d_src;
-        lp.out = d_out;
+        lp.out = reinterpret_cast<void *>(out_base);
         lp.perm = d_perm;
-        lp.pos = tables.pos;
+        lp.pos = tables.pos ? reinterpret_cast<int32_t *>(pos_base) : nullptr;
         lp.win = tables.win;
         lp.order = tables.order;
+        lp.unit0 = static_cast<int32_t>(lo_i);  // the launch's first image may start inside it
         fold_normalisation(p, &lp);
         int64_t blocks = 0;
         int32_t tr = 1, tc = 1, k = 0;
-        while (i < last && k < mimo::kMaxImagesPerLaunch &&
-               blocks + v.plan.img[i].blocks <= static_cast<int64_t>(INT32_MAX)) {
+        while (i < last && k < mimo::kMaxImagesPerLaunch && blocks + (hi_i - lo_i) <= static_cast<int64_t>(INT32_MAX)) {
             const ImagePlan &ip = v.plan.img[i];
             mimo::ImageDesc &d = lp.img[k];
             d.src_off = src_offsets[i];
@@ -265,11 +290,15 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
             // the image; they read nothing past the end of the caller's buffer
             d.limit = static_cast<int64_t>(src_bytes) - src_offsets[i];
             lp.block_start[k] = static_cast<int32_t>(blocks);
-            blocks += ip.blocks;
+            blocks += hi_i - lo_i;
             tr = std::max(tr, ip.tile_rows);
             tc = std::max(tc, ip.tile_cols);
             ++k;
-            ++i;
+            // the next image with units in the window; only the window's first image starts inside
+            // itself, so later images of a launch begin at their unit 0
+            do {
+                ++i;
+            } while (i < last && !unit_span(i, &lo_i, &hi_i));
         }
         lp.block_start[k] = static_cast<int32_t>(blocks);
         lp.n = k;
@@ -284,6 +313,13 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
         const size_t raw_floats = static_cast<size_t>(tr) * static_cast<size_t>(lp.raw_stride) / 4u;
         lp.raw = static_cast<int32_t>(tile_floats);  // tile | raw staging rows
         const size_t smem = sizeof(float) * (tile_floats + raw_floats);
+#if defined(MIMO_BOUNDS_CHECK)
+        // rows this call may emit (kernel numbering: batch row - row_base), inside the window
+        lp.chk_row_lo = std::max<int64_t>(v.plan.row0[first], 4 * win.lo) - row_base;
+        lp.chk_row_hi = std::min<int64_t>(v.plan.row0[last], win.hi > INT64_MAX / 4 ? INT64_MAX : 4 * win.hi) - row_base;
+        lp.chk_table_rows = v.plan.row0[last] - row_base;
+        lp.chk_smem_floats = static_cast<int32_t>(tile_floats + raw_floats);
+#endif
         const int st = mimo::launch_preprocess(lp, blocks, out_dtype, smem, stream);
         if (st != MIMO_OK) return st;
     }
@@ -367,6 +403,40 @@ int mimo_preprocess_batch_ex(const mimo_params *p, int32_t n, const uint8_t *d_s
     tables.win = out->d_window_index;
     return launch_range(p, v, 0, n, d_src, src_bytes, src_offsets, heights, widths, channels, out->out_dtype,
                         out->d_out, out->d_column_perm, stream, tables);
+}
+
+int mimo_preprocess_units(const mimo_params *p, int32_t n, const uint8_t *d_src, size_t src_bytes,
+                          const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
+                          const int32_t *channels, int64_t first_unit, int64_t unit_count, const mimo_outputs *out,
+                          void *stream) {
+    if (!out) return MIMO_EINVAL;
+    if (out->row_order == MIMO_ORDER_COLUMN) return MIMO_EUNSUPPORTED;
+    if (out->row_order != MIMO_ORDER_MERGE) return MIMO_EINVAL;
+    if (first_unit < 0 || unit_count < 0) return MIMO_EINVAL;
+    Validated v;
+    // rows are checked against the window below, not against the whole batch
+    int st = validate_batch(p, n, d_src, src_bytes, src_offsets, heights, widths, channels, out->out_dtype,
+                            out->d_out, std::numeric_limits<int64_t>::max(), out->d_column_perm, &v);
+    if (st != MIMO_OK) return st;
+    const int64_t total_units = v.total_rows / 4;
+    if (unit_count > total_units || first_unit > total_units - unit_count) return MIMO_ERANGE;
+    if (unit_count == 0) return MIMO_OK;
+    if (4 * unit_count > out->out_rows_capacity) return MIMO_ECAPACITY;
+    for (const void *t : {static_cast<const void *>(out->d_positions), static_cast<const void *>(out->d_window_index)}) {
+        if (!t) continue;
+        if (!aligned16(t)) return MIMO_EALIGN;
+        if (v.total_rows > INT32_MAX) return MIMO_EOVERFLOW;
+    }
+    Tables tables;
+    tables.order = MIMO_ORDER_MERGE;
+    tables.pos = out->d_positions;
+    tables.win = out->d_window_index;
+    UnitWindow win;
+    win.lo = first_unit;
+    win.hi = first_unit + unit_count;
+    win.row_shift = 4 * first_unit;  // rows and positions of the window start at d_out / d_positions
+    return launch_range(p, v, 0, n, d_src, src_bytes, src_offsets, heights, widths, channels, out->out_dtype,
+                        out->d_out, out->d_column_perm, stream, tables, 0, win);
 }
 
 int mimo_preprocess_batch(const mimo_params *p, int32_t n, const uint8_t *d_src, size_t src_bytes,
@@ -585,6 +655,21 @@ int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int
                                     d_error, stream);
 }
 
+int mimo_patch_embed_stall_test(const void *d_rows, int64_t rows, const void *d_weight, int32_t embed_dim,
+                                const float *d_bias, int32_t out_dtype, void *d_out, int32_t *d_error,
+                                int32_t stop_after_kblocks, uint32_t wait_rounds, void *stream) {
+    if (rows <= 0 || embed_dim <= 0 || (embed_dim % 256) != 0) return MIMO_EINVAL;
+    if (out_dtype != MIMO_F32 && out_dtype != MIMO_BF16) return MIMO_EINVAL;
+    if (stop_after_kblocks < 0 || stop_after_kblocks > mimo::kRowWidth / 64 || wait_rounds == 0) return MIMO_EINVAL;
+    if (!d_rows || !d_weight || !d_out || !d_error) return MIMO_EINVAL;
+    if (!aligned16(d_rows) || !aligned16(d_weight) || !aligned16(d_out) || (d_bias && !aligned16(d_bias)) ||
+        (reinterpret_cast<uintptr_t>(d_error) & 3u) != 0)
+        return MIMO_EALIGN;
+    if (rows > (int64_t(1) << 31) - 1) return MIMO_EOVERFLOW;
+    return mimo::launch_patch_embed(d_rows, rows, mimo::kRowWidth, d_weight, embed_dim, d_bias, out_dtype, d_out,
+                                    d_error, stream, wait_rounds, stop_after_kblocks);
+}
+
 int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src, size_t src_bytes,
                           const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
                           const int32_t *channels, int32_t row_order, const void *d_weight, int32_t embed_dim,
@@ -687,6 +772,11 @@ const char *mimo_status_string(int status) {
         case MIMO_ELIMIT: return "an image does not fit the fixed staging area of the no-allocation entry point";
         default: return "unknown status";
     }
+}
+
+int mimo_bounds_check_status(int64_t *violations, int32_t *first_kind) {
+    if (!violations || !first_kind) return MIMO_EINVAL;
+    return mimo::bounds_check_status(violations, first_kind);
 }
 
 int mimo_version(void) { return 10000; }
@@ -833,6 +923,12 @@ int mimo_preprocess_video(const mimo_params *p, int32_t n_frames, const uint8_t 
     lp.raw_stride = ((32 + 4 * vp.ip.tile_cols) + 15) & ~15;
     const size_t raw_floats = static_cast<size_t>(lp.tile_rows) * static_cast<size_t>(lp.raw_stride) / 4u;
     lp.raw = static_cast<int32_t>(tile_floats);
+#if defined(MIMO_BOUNDS_CHECK)
+    lp.chk_row_lo = 0;
+    lp.chk_row_hi = vp.rows;
+    lp.chk_table_rows = vp.rows;
+    lp.chk_smem_floats = static_cast<int32_t>(tile_floats + raw_floats);
+#endif
     return mimo::launch_preprocess(lp, blocks, out->out_dtype, sizeof(float) * (tile_floats + raw_floats), stream);
 }
 

@@ -47,6 +47,25 @@ struct ImageDesc {
 };
 static_assert(sizeof(ImageDesc) == 56, "descriptor layout");
 
+// Debug builds compiled with -DMIMO_BOUNDS_CHECK check every global load and
+// store of the pixel kernels (and their shared-memory tile indices) against the
+// extents they must stay in: the image's bytes and the caller's source buffer,
+// the output rows and tables the host validated. A failed check skips the
+// access and counts it in a device status word (mimo_bounds_check_status); it
+// never traps. Release builds compile the checks away.
+#if defined(MIMO_BOUNDS_CHECK)
+#define MIMO_CHECK(cond, kind) (::mimo::bounds_ok((cond), (kind)))
+#else
+#define MIMO_CHECK(cond, kind) true
+#endif
+enum : int32_t {
+    kChkSrcCopy = 1,     // staged source copy outside the caller's buffer
+    kChkSrcLoad = 2,     // direct source load outside the image
+    kChkSmem = 3,        // shared-memory tile or staging index outside its region
+    kChkRowStore = 4,    // output row outside the validated rows
+    kChkTableStore = 5,  // permutation / position / window entry outside its table
+};
+
 // Everything one launch needs travels by value as the kernel's parameter
 // block (__grid_constant__), so a launch needs no device-side table and no
 // host-to-device copy. The block is sized for kCap images: the driver copies
@@ -59,13 +78,19 @@ struct LaunchParamsT {
     int32_t *pos;        // may be null: (patch row, patch column) per emitted row
     int32_t *win;        // may be null: merge-order unit of each column-major unit
     int32_t order;       // 0: merge-block order, 1: column order
-    int32_t pad0;
+    int32_t unit0;       // first merge unit of img[0] in this launch (a launch may start inside an image)
     float k[3], b[3];    // normalisation folded: v = x*k[c] + b[c]
     int32_t n;           // images in this launch
     int32_t tile_rows;   // rows of the shared-memory tile (max over images)
     int32_t tile_stride; // row stride (floats, multiple of 4) of the tile
     int32_t raw;         // float offset of the raw staging rows
     int32_t raw_stride;  // bytes per raw staging row (multiple of 16)
+#if defined(MIMO_BOUNDS_CHECK)
+    int64_t chk_row_lo, chk_row_hi;  // rows the kernel may emit (its own row numbering)
+    int64_t chk_table_rows;          // rows the permutation covers (window index: a quarter)
+    int32_t chk_smem_floats;         // floats of dynamic shared memory (tile + raw)
+    int32_t chk_pad;
+#endif
     int32_t block_start[kCap + 1];  // prefix sum of blocks (video blocks are halves)
     ImageDesc img[kCap];
 };
@@ -107,9 +132,19 @@ MIMO_HD int64_t block_span(int64_t b, int64_t in, int64_t out) {
 
 int launch_preprocess(const LaunchParams &lp, int64_t blocks, int out_dtype, size_t smem_bytes, void *stream);
 
-// Patch embedding GEMM on the tensor cores (mimo_patch_embed.cu).
+#if defined(MIMO_BOUNDS_CHECK) && defined(__CUDACC__)
+__device__ bool bounds_ok(bool ok, int kind);
+#endif
+// Failed bounds checks since the last query, and the kind of the first
+// (MIMO_EUNSUPPORTED unless built with -DMIMO_BOUNDS_CHECK); clears both.
+int bounds_check_status(int64_t *violations, int32_t *first_kind);
+
+// Patch embedding GEMM on the tensor cores (mimo_patch_embed.cu). wait_rounds
+// = 0 keeps the default wait limit; stop_after >= 0 (tests of the failure path
+// only) stops each CTA's operand loader after that many 64-wide K blocks.
 int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_weight, int32_t N, const float *d_bias,
-                       int32_t out_dtype, void *d_out, int32_t *d_err, void *stream);
+                       int32_t out_dtype, void *d_out, int32_t *d_err, void *stream, uint32_t wait_rounds = 0,
+                       int32_t stop_after = -1);
 
 // Device address and size of the library's fixed staging area on the
 // current device (mimo_noalloc.cu).

@@ -56,7 +56,7 @@ constexpr int kEpiWarps = 4;
 constexpr int kStagePitch = 128 + 16;       // epilogue staging row: one 128-byte output line + pad (no bank conflicts)
 constexpr int kEpiStageBytes = 32 * kStagePitch;  // per epilogue warp: 32 rows
 constexpr uint16_t kPairMask = 0x3;         // both CTAs of the cluster
-constexpr uint32_t kWaitLimit = 1u << 20;   // try_wait rounds before a wait is declared stuck
+constexpr uint32_t kWaitLimit = 1u << 20;   // try_wait rounds before a wait is declared stuck (default)
 
 enum : int { kErrNone = 0, kErrFullWait = 1, kErrEmptyWait = 2, kErrAccumWait = 3, kErrAccumFreeWait = 4,
              kErrDrainWait = 5 };
@@ -106,12 +106,12 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
-// Bounded wait for the phase with the given parity to complete; false if the
-// limit ran out (the caller records the error and stops). Cluster scope: some
-// of the arrivals come from the other CTA of the pair.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Bounded wait for the phase with the given parity to complete; false if
+// `limit` try_wait rounds ran out (the caller records the error and stops).
+// Cluster scope: some of the arrivals come from the other CTA of the pair.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit) {
     const uint32_t a = smem_u32(bar);
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    for (uint32_t i = 0; i < limit; ++i) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -218,7 +218,7 @@ template <bool kOutBF16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     patch_embed_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                        const float *__restrict__ bias, void *__restrict__ out, int64_t M, int32_t N, int32_t K,
-                       int32_t *__restrict__ err) {
+                       int32_t *__restrict__ err, uint32_t wait_limit, int32_t stop_after) {
     extern __shared__ __align__(1024) uint8_t gemm_smem_raw[];
     // 1024-byte aligned tiles (the swizzle pattern repeats every 1024 bytes); the
     // offset is the same in both CTAs, as the pair MMA requires
@@ -266,8 +266,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int a_row = static_cast<int>((t / n_tiles) * kPairM) + static_cast<int>(rank) * kBM;
                 const int b_row = static_cast<int>(t % n_tiles) * kBN + static_cast<int>(rank) * kBNHalf;
                 for (int kb = 0; kb < kblocks; ++kb, ++g) {
+                    // test hook: a loader that stops after `stop_after` k blocks (never in normal launches)
+                    if (stop_after >= 0 && g >= static_cast<uint32_t>(stop_after)) break;
                     const uint32_t s = g % kStages, use = g / kStages;
-                    if (use > 0 && !mbar_wait(&S.empty[s], (use - 1) & 1)) {
+                    if (use > 0 && !mbar_wait(&S.empty[s], (use - 1) & 1, wait_limit)) {
                         fail(S, err, kErrEmptyWait);
                         break;
                     }
@@ -283,7 +285,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // CTA's barrier counts the peer's copies as well)
             if (leader)
                 for (uint32_t q = (g > kStages ? g - kStages : 0); q < g; ++q)
-                    mbar_wait(&S.full[q % kStages], (q / kStages) & 1);
+                    mbar_wait(&S.full[q % kStages], (q / kStages) & 1, wait_limit);
         }
     } else if (warp == 1) {
         // ---- MMA issuer: one lane of the even CTA drives the tensor cores of both SMs
@@ -291,7 +293,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t g = 0, i = 0;
             for (int64_t t = pair; t < total_tiles && !stopped(S); t += pairs, ++i) {
                 const uint32_t b = i & 1, use_b = i >> 1;
-                if (use_b > 0 && !mbar_wait(&S.acc_free[b], (use_b - 1) & 1)) {
+                if (use_b > 0 && !mbar_wait(&S.acc_free[b], (use_b - 1) & 1, wait_limit)) {
                     fail(S, err, kErrAccumFreeWait);
                     break;
                 }
@@ -300,7 +302,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 bool ok = true;
                 for (int kb = 0; kb < kblocks; ++kb, ++g) {
                     const uint32_t s = g % kStages;
-                    if (!mbar_wait(&S.full[s], (g / kStages) & 1)) {
+                    if (!mbar_wait(&S.full[s], (g / kStages) & 1, wait_limit)) {
                         fail(S, err, kErrFullWait);
                         ok = false;
                         break;
@@ -328,7 +330,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             // every MMA issued has finished before TMEM can be freed (bounded)
             umma_commit_local(&S.drain);
-            if (!mbar_wait(&S.drain, 0)) fail(S, err, kErrDrainWait);
+            if (!mbar_wait(&S.drain, 0, wait_limit)) fail(S, err, kErrDrainWait);
         }
     } else {
         // ---- epilogue (both CTAs): warp w reads TMEM lanes 32*(w % 4) .. +31 (its accessible quarter)
@@ -338,7 +340,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int64_t t = pair; t < total_tiles; t += pairs, ++i) {
             const uint32_t b = i & 1;
             // uniform across the warp: tcgen05.ld below is a warp-wide instruction
-            const bool ready = __all_sync(0xffffffffu, !stopped(S) && mbar_wait(&S.acc_full[b], (i >> 1) & 1));
+            const bool ready =
+                __all_sync(0xffffffffu, !stopped(S) && mbar_wait(&S.acc_full[b], (i >> 1) & 1, wait_limit));
             if (!ready) {
                 if (lane == 0) fail(S, err, kErrAccumWait);
                 break;
@@ -426,7 +429,9 @@ bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, in
 }  // namespace
 
 int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_weight, int32_t N, const float *d_bias,
-                       int32_t out_dtype, void *d_out, int32_t *d_err, void *stream) {
+                       int32_t out_dtype, void *d_out, int32_t *d_err, void *stream, uint32_t wait_rounds,
+                       int32_t stop_after) {
+    const uint32_t wait_limit = wait_rounds ? wait_rounds : kWaitLimit;
     CUtensorMap ma, mb;
     if (!make_map(&ma, d_rows, M, K, kBM) || !make_map(&mb, d_weight, N, K, kBNHalf)) return MIMO_ECUDA;
     const int64_t tiles = ((M + kPairM - 1) / kPairM) * (N / kBN);
@@ -455,7 +460,9 @@ int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_w
     if (cudaOccupancyMaxActiveClusters(&max_pairs, kernel, &cfg) != cudaSuccess || max_pairs < 1) return MIMO_ECUDA;
     const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
-    if (cudaLaunchKernelEx(&cfg, kernel, ma, mb, d_bias, d_out, M, N, K, d_err) != cudaSuccess) return MIMO_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, kernel, ma, mb, d_bias, d_out, M, N, K, d_err, wait_limit, stop_after) !=
+        cudaSuccess)
+        return MIMO_ECUDA;
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
 }
 

@@ -33,6 +33,22 @@
 #include "mimo_internal.h"
 
 namespace mimo {
+
+#if defined(MIMO_BOUNDS_CHECK)
+// Debug builds: accesses that failed their bounds check (skipped, not made),
+// and the kind of the first one.
+__device__ unsigned long long g_bounds_violations;
+__device__ int g_bounds_first_kind;
+
+__device__ __noinline__ bool bounds_ok(bool ok, int kind) {
+    if (!ok) {
+        atomicAdd(&g_bounds_violations, 1ull);
+        atomicCAS(&g_bounds_first_kind, 0, kind);
+    }
+    return ok;
+}
+#endif
+
 namespace {
 
 constexpr float kTwo23 = 8388608.0f;
@@ -79,7 +95,7 @@ __device__ __forceinline__ int find_image(const Params &P, int blk) {
 // Taps, staging geometry and output addresses of one merge block (double-
 // buffered in shared memory: the pipeline holds the current block and the
 // next one). Every later phase reads the block's constants from here.
-struct TapSet {
+struct alignas(16) TapSet {  // 16-byte aligned: the fused RGB path reads tap quads as int4 / float4
     int32_t ty[2][kBlock];   // tile row of each output row's two taps
     int32_t tx[2][kBlock];   // tile column of each output column's two taps
     float ly[kBlock];        // weight of the second row tap
@@ -148,7 +164,8 @@ __device__ __forceinline__ void compute_taps(const Params &P, TapSet &T, const T
     } else {
         ii = find_image(P, blk);
         const ImageDesc &Dc = P.img[ii];
-        int local = blk - P.block_start[ii];
+        // the launch's first image may start at merge unit unit0 (image launches only)
+        int local = blk - P.block_start[ii] + (ii == 0 ? P.unit0 : 0);
         const bool vid = (Dc.flags & kVideo) != 0;
         tt = vid ? (local & 1) : 0;
         if (vid) local >>= 1;
@@ -343,16 +360,34 @@ __device__ __forceinline__ void issue_stage(const Params &P, const TapSet &T, ui
             if (cs < rs + L) {
                 const int64_t left = limit - cs;
                 const int nb = left < 16 ? static_cast<int>(left) : 16;
-                cp_async16(raw + j * P.raw_stride + 16 * c, img + cs, nb);
+                if (MIMO_CHECK(cs >= 0 && nb > 0 && cs + nb <= limit, kChkSrcCopy) &&
+                    MIMO_CHECK(j < P.tile_rows && 16 * c + 16 <= P.raw_stride, kChkSmem))
+                    cp_async16(raw + j * P.raw_stride + 16 * c, img + cs, nb);
             }
         }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
+// The RGB pixel at byte offset o of a staged row, its bytes in bytes 0..2 of
+// the result: two aligned 32-bit shared loads and a funnel shift.
+__device__ __forceinline__ uint32_t rgb_at(const uint8_t *row, uint32_t o) {
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(row + (o & ~3u));
+    return __funnelshift_r(w[0], w[1], (o & 3u) * 8u);
+}
+
+// Whether block T's staged rows are converted and interpolated along W in one
+// step (RGB, resized width, contiguously staged columns); emit_block then
+// skips its horizontal pass.
+__device__ __forceinline__ bool fused_hpass(const TapSet &T) {
+    return T.C == 3 && (T.flags & (kIdentityCols | kGatherCols)) == 0;
+}
+
 // Converts block T's staged bytes to planar fp32 in the tile (RGBA
 // composited onto white): a job = 4 consecutive pixels of one tile row.
-// Gathered columns are loaded here directly from global memory.
+// For RGB with a resized width a job is instead one quad of output columns of
+// a tile row, interpolated along W on the way (fused_hpass). Gathered columns
+// are loaded here directly from global memory.
 template <class Params>
 __device__ __forceinline__ void finish_stage(const Params &P, const TapSet &T, const uint8_t *raw, float *tile,
                                              int TS, int plane, int tid) {
@@ -360,7 +395,54 @@ __device__ __forceinline__ void finish_stage(const Params &P, const TapSet &T, c
     const int nrows = T.nrows;
     const int C = T.C;
     const float2 m23 = f2(-kTwo23, -kTwo23);
-    if ((flags & kGatherCols) == 0) {
+    if (fused_hpass(T)) {
+        // job = (tile row j, output quad q): the two taps of each of the quad's 4 output columns come
+        // straight from the staged bytes, and (1 - lx) a + lx b = fma(lx, b - a, a) lands over columns
+        // 4q..4q+3 of the tile row. b - a is formed exactly from the 2^23 bit patterns, so the values
+        // equal those of converting the row and then interpolating it.
+        const int W = T.W, y_first = T.y_first, x_first = T.x_first;
+        const bool grow = (flags & kGatherRows) != 0;
+        const int jobs = nrows * 8;
+        const int t0 = (jobs <= 2 * (kThreads - 64)) ? 64 : 0;
+        const int step = kThreads - t0;
+        const float2 neg1 = f2(-1.0f, -1.0f);
+        for (int job = tid - t0; job < jobs; job += step) {
+            if (job < 0) break;
+            const int j = job >> 3, q = job & 7;
+            const int sy = grow ? T.srow[j] : y_first + j;
+            const uint32_t mis = ((static_cast<uint32_t>(sy) * static_cast<uint32_t>(W) + x_first) * 3u) & 15u;
+            const uint8_t *row = raw + j * P.raw_stride;
+            const int4 ta = *reinterpret_cast<const int4 *>(&T.tx[0][4 * q]);
+            const int4 tb = *reinterpret_cast<const int4 *>(&T.tx[1][4 * q]);
+            const float4 l = *reinterpret_cast<const float4 *>(&T.lx[4 * q]);
+            // every tap read stays inside the staged row, every write inside the tile
+            if (!MIMO_CHECK(j < P.tile_rows && 4 * q + 4 <= TS &&
+                                min(min(min(ta.x, ta.y), min(ta.z, ta.w)), min(min(tb.x, tb.y), min(tb.z, tb.w))) >= 0 &&
+                                ((mis + 3u * static_cast<uint32_t>(max(max(max(ta.x, ta.y), max(ta.z, ta.w)),
+                                                                        max(max(tb.x, tb.y), max(tb.z, tb.w))))) &
+                                 ~3u) + 8u <= static_cast<uint32_t>(P.raw_stride),
+                            kChkSmem))
+                continue;
+            const uint32_t a0 = rgb_at(row, mis + 3u * ta.x), a1 = rgb_at(row, mis + 3u * ta.y);
+            const uint32_t a2 = rgb_at(row, mis + 3u * ta.z), a3 = rgb_at(row, mis + 3u * ta.w);
+            const uint32_t b0 = rgb_at(row, mis + 3u * tb.x), b1 = rgb_at(row, mis + 3u * tb.y);
+            const uint32_t b2 = rgb_at(row, mis + 3u * tb.z), b3 = rgb_at(row, mis + 3u * tb.w);
+            const float2 l01 = f2(l.x, l.y), l23 = f2(l.z, l.w);
+            float *t = tile + j * TS + 4 * q;
+#define MIMO_FUSED_CHANNEL(c)                                                                     \
+    {                                                                                             \
+        const float2 A01 = f2(byte_bits<c>(a0), byte_bits<c>(a1));                                \
+        const float2 A23 = f2(byte_bits<c>(a2), byte_bits<c>(a3));                                \
+        const float2 v01 = fma2(l01, fma2(A01, neg1, f2(byte_bits<c>(b0), byte_bits<c>(b1))), add2(A01, m23)); \
+        const float2 v23 = fma2(l23, fma2(A23, neg1, f2(byte_bits<c>(b2), byte_bits<c>(b3))), add2(A23, m23)); \
+        *reinterpret_cast<float4 *>(t + (c) * plane) = make_float4(v01.x, v01.y, v23.x, v23.y);  \
+    }
+            MIMO_FUSED_CHANNEL(0)
+            MIMO_FUSED_CHANNEL(1)
+            MIMO_FUSED_CHANNEL(2)
+#undef MIMO_FUSED_CHANNEL
+        }
+    } else if ((flags & kGatherCols) == 0) {
         const int W = T.W, y_first = T.y_first, x_first = T.x_first;
         const bool grow = (flags & kGatherRows) != 0;
         const int Q = T.Q;
@@ -379,6 +461,9 @@ __device__ __forceinline__ void finish_stage(const Params &P, const TapSet &T, c
             const uint32_t mis = ((static_cast<uint32_t>(sy) * static_cast<uint32_t>(W) + x_first) *
                                   static_cast<uint32_t>(C)) & 15u;
             const uint32_t o = mis + static_cast<uint32_t>(C * px0);
+            if (!MIMO_CHECK(j < P.tile_rows && px0 + 4 <= TS && (o & ~3u) + 16u <= static_cast<uint32_t>(P.raw_stride),
+                            kChkSmem))
+                continue;
             const uint32_t *rw = reinterpret_cast<const uint32_t *>(raw + j * P.raw_stride) + (o >> 2);
             const uint32_t w0 = rw[0], w1 = rw[1], w2 = rw[2], w3 = rw[3];
             float2 R0, R1, G0, G1, B0, B1;
@@ -423,6 +508,7 @@ __device__ __forceinline__ void finish_stage(const Params &P, const TapSet &T, c
             const int i = e & (kMaxTile - 1);
             const int sy = grow ? T.srow[j] : T.y_first + j;
             const int64_t pix = static_cast<int64_t>(sy) * W + T.scol[i];
+            if (!MIMO_CHECK(pix >= 0 && (pix + 1) * C <= T.limit && j < P.tile_rows && i < TS, kChkSrcLoad)) continue;
             float r, g, b;
             if (C == 4) {
                 const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(img) + pix);
@@ -453,6 +539,7 @@ __device__ __forceinline__ void finish_stage(const Params &P, const TapSet &T, c
 template <bool kBF16, class Params>
 __device__ __forceinline__ void store_quad(const Params &P, int64_t row, int c, int col, int slot0, bool both,
                                            float2 v01, float2 v23) {
+    if (!MIMO_CHECK(row >= P.chk_row_lo && row < P.chk_row_hi, kChkRowStore)) return;
     const float2 k2 = f2(P.k[c], P.k[c]), b2 = f2(P.b[c], P.b[c]);
     const float2 n01 = fma2(v01, k2, b2);
     const float2 n23 = fma2(v23, k2, b2);
@@ -485,16 +572,20 @@ __device__ __forceinline__ void write_unit_tables(const Params &P, int tid, int6
     const int64_t dst_unit = t_units + static_cast<int64_t>(bw) * gh2 + bh;  // column order
     if (tid == 0 && P.perm != nullptr) {
         const int32_t s0 = static_cast<int32_t>(row0 + 4 * src_unit);
-        __stcs(reinterpret_cast<int4 *>(P.perm + row0 + 4 * dst_unit), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
+        if (MIMO_CHECK(row0 + 4 * dst_unit >= 0 && row0 + 4 * dst_unit + 4 <= P.chk_table_rows, kChkTableStore))
+            __stcs(reinterpret_cast<int4 *>(P.perm + row0 + 4 * dst_unit), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
     } else if (tid == 1 && P.pos != nullptr) {
         // rows (mh, mw) = (0,0), (0,1), (1,0), (1,1) of the unit
         const int32_t h = 2 * bh, w = 2 * bw;
         int4 *d = reinterpret_cast<int4 *>(P.pos + 2 * row_base);
-        __stcs(d, make_int4(h, w, h, w + 1));
-        __stcs(d + 1, make_int4(h + 1, w, h + 1, w + 1));
+        if (MIMO_CHECK(row_base >= P.chk_row_lo && row_base + 4 <= P.chk_row_hi, kChkTableStore)) {
+            __stcs(d, make_int4(h, w, h, w + 1));
+            __stcs(d + 1, make_int4(h + 1, w, h + 1, w + 1));
+        }
     } else if (tid == 2 && P.win != nullptr) {
         const int64_t u0 = row0 / 4;
-        P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
+        if (MIMO_CHECK(u0 + dst_unit >= 0 && 4 * (u0 + dst_unit) + 4 <= P.chk_table_rows, kChkTableStore))
+            P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
     }
 }
 
@@ -508,22 +599,26 @@ __device__ __forceinline__ void emit_block(const Params &P, const TapSet &T, flo
     // horizontal pass (resized widths only), in place: the warp owning tile
     // row j reads every lane's two taps, then writes the 32 interpolated
     // values over columns 0..31 of the same row
-    const bool hpass = (flags & kIdentityCols) == 0;
+    const bool hpass = (flags & kIdentityCols) == 0 && !fused_hpass(T);
     if (hpass) {
         const int x0 = T.tx[0][lane], x1 = T.tx[1][lane];
         const float lx = T.lx[lane];
         for (int j = warp; j < nrows; j += kThreads / 32) {
             float *t = tile + j * TS;
             float h[3];
+            // a lane whose check fails skips its accesses, never the __syncwarp
+            const bool ok = MIMO_CHECK(j < P.tile_rows && x0 >= 0 && x1 >= 0 && x0 < TS && x1 < TS, kChkSmem);
 #pragma unroll
             for (int c = 0; c < 3; ++c) {
-                const float a = t[c * plane + x0];
-                const float b = t[c * plane + x1];
+                const float a = ok ? t[c * plane + x0] : 0.0f;
+                const float b = ok ? t[c * plane + x1] : 0.0f;
                 h[c] = fmaf(lx, b - a, a);
             }
             __syncwarp();
+            if (ok) {
 #pragma unroll
-            for (int c = 0; c < 3; ++c) t[c * plane + lane] = h[c];
+                for (int c = 0; c < 3; ++c) t[c * plane + lane] = h[c];
+            }
         }
         __syncthreads();
     }
@@ -539,6 +634,10 @@ __device__ __forceinline__ void emit_block(const Params &P, const TapSet &T, flo
     const int dy = (mh << 4) | py;
     const int dx0 = (mw << 4) | (q << 2);
     const bool yident = (flags & kIdentityRows) != 0;
+    if (!MIMO_CHECK(T.ty[0][dy] >= 0 && T.ty[1][dy] >= 0 && T.ty[0][dy] < P.tile_rows && T.ty[1][dy] < P.tile_rows &&
+                        dx0 + 4 <= TS,
+                    kChkSmem))
+        return;
     const float *a_row = tile + T.ty[0][dy] * TS + dx0;
     const float *b_row = tile + T.ty[1][dy] * TS + dx0;
     // (1 - ly) a + ly b as two FMAs: a - ly a, then + ly b
@@ -706,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, kVideoLaunch ? 5 : 6) direct_kernel(
     {
         const ImageDesc &D = P.img[ii];
         const int g = D.Wr / kBlock;
-        int local = begin - P.block_start[ii];
+        int local = begin - P.block_start[ii] + (ii == 0 ? P.unit0 : 0);
         const bool vid = (D.flags & kVideo) != 0;
         tt = vid ? (local & 1) : 0;
         if (vid) local >>= 1;
@@ -755,11 +854,20 @@ __global__ void __launch_bounds__(kThreads, kVideoLaunch ? 5 : 6) direct_kernel(
         const int64_t f = video ? min(2 * t + tt, D.frames - 1) : 0;
         const uint8_t *img = P.src + D.src_off + f * D.frame_stride;
         const int64_t x = static_cast<int64_t>(bw) * kBlock + dx0;
-        uint32_t wa[4], wb[4];
+        uint32_t wa[4] = {0u, 0u, 0u, 0u}, wb[4] = {0u, 0u, 0u, 0u};
         float4 va[3], vb[3];
-        load_quad(img + (static_cast<int64_t>(sy0) * W + x) * C, C, wa);
+        // the quad's bytes lie inside the frame and the caller's buffer (skipped otherwise)
+        const int64_t frame_bytes = static_cast<int64_t>(H) * W * C;
+        const int64_t qa = (static_cast<int64_t>(sy0) * W + x) * C, qb = (static_cast<int64_t>(sy1) * W + x) * C;
+        if (MIMO_CHECK(qa >= 0 && qa + (C == 4 ? 16 : 12) <= frame_bytes &&
+                           f * D.frame_stride + qa + (C == 4 ? 16 : 12) <= D.limit,
+                       kChkSrcLoad))
+            load_quad(img + qa, C, wa);
         if (!yident) {
-            load_quad(img + (static_cast<int64_t>(sy1) * W + x) * C, C, wb);
+            if (MIMO_CHECK(qb >= 0 && qb + (C == 4 ? 16 : 12) <= frame_bytes &&
+                               f * D.frame_stride + qb + (C == 4 ? 16 : 12) <= D.limit,
+                           kChkSrcLoad))
+                load_quad(img + qb, C, wb);
             convert4(wb, C, vb);
         }
         convert4(wa, C, va);
@@ -790,15 +898,22 @@ __global__ void __launch_bounds__(kThreads, kVideoLaunch ? 5 : 6) direct_kernel(
             const int64_t dst_unit = t_units + static_cast<int64_t>(bw) * gh2 + bh;  // column order
             if (tid == 0 && P.perm != nullptr) {
                 const int32_t s0 = static_cast<int32_t>(D.row0 + 4 * src_unit);
-                __stcs(reinterpret_cast<int4 *>(P.perm + D.row0 + 4 * dst_unit), make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
+                if (MIMO_CHECK(D.row0 + 4 * dst_unit >= 0 && D.row0 + 4 * dst_unit + 4 <= P.chk_table_rows,
+                               kChkTableStore))
+                    __stcs(reinterpret_cast<int4 *>(P.perm + D.row0 + 4 * dst_unit),
+                           make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
             } else if (tid == 1 && P.pos != nullptr) {
                 const int32_t h = 2 * bh, w = 2 * bw;
                 int4 *d = reinterpret_cast<int4 *>(P.pos + 2 * (D.row0 + 4 * unit));
-                __stcs(d, make_int4(h, w, h, w + 1));
-                __stcs(d + 1, make_int4(h + 1, w, h + 1, w + 1));
+                if (MIMO_CHECK(D.row0 + 4 * unit >= P.chk_row_lo && D.row0 + 4 * unit + 4 <= P.chk_row_hi,
+                               kChkTableStore)) {
+                    __stcs(d, make_int4(h, w, h, w + 1));
+                    __stcs(d + 1, make_int4(h + 1, w, h + 1, w + 1));
+                }
             } else if (tid == 2 && P.win != nullptr) {
                 const int64_t u0 = D.row0 / 4;
-                P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
+                if (MIMO_CHECK(u0 + dst_unit >= 0 && 4 * (u0 + dst_unit) + 4 <= P.chk_table_rows, kChkTableStore))
+                    P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
             }
         }
         if constexpr (kVideoLaunch) {
@@ -917,6 +1032,28 @@ int launch_kernels(const Params &lp, int64_t blocks, int out_dtype, size_t smem_
 }
 
 }  // namespace
+
+int bounds_check_status(int64_t *violations, int32_t *first_kind) {
+#if defined(MIMO_BOUNDS_CHECK)
+    unsigned long long v = 0;
+    int k = 0;
+    if (cudaMemcpyFromSymbol(&v, g_bounds_violations, sizeof(v)) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&k, g_bounds_first_kind, sizeof(k)) != cudaSuccess)
+        return MIMO_ECUDA;
+    const unsigned long long zero = 0;
+    const int zk = 0;
+    if (cudaMemcpyToSymbol(g_bounds_violations, &zero, sizeof(zero)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_bounds_first_kind, &zk, sizeof(zk)) != cudaSuccess)
+        return MIMO_ECUDA;
+    *violations = static_cast<int64_t>(v);
+    *first_kind = k;
+    return MIMO_OK;
+#else
+    (void)violations;
+    (void)first_kind;
+    return MIMO_EUNSUPPORTED;
+#endif
+}
 
 int launch_preprocess(const LaunchParams &lp, int64_t blocks, int out_dtype, size_t smem_bytes, void *stream) {
     if (blocks <= 0) return MIMO_OK;

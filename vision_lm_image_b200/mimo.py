@@ -36,11 +36,11 @@ STATUS_NAMES = {
     10: "MIMO_ERANGE", 11: "MIMO_ELIMIT",
 }
 EXPORTED = ("mimo_params_default", "mimo_smart_resize", "mimo_num_patches", "mimo_plan_batch",
-            "mimo_preprocess_batch", "mimo_preprocess_batch_ex", "mimo_preprocess_batch_host",
+            "mimo_preprocess_batch", "mimo_preprocess_batch_ex", "mimo_preprocess_units", "mimo_preprocess_batch_host",
             "mimo_preprocess_batch_host_noalloc", "mimo_expand_prompt_ids", "mimo_video_max_pixels",
             "mimo_smart_nframes", "mimo_sample_frames", "mimo_plan_video", "mimo_preprocess_video",
-            "mimo_patch_embed", "mimo_preprocess_embed",
-            "mimo_status_string", "mimo_version")
+            "mimo_patch_embed", "mimo_patch_embed_stall_test", "mimo_preprocess_embed",
+            "mimo_status_string", "mimo_version", "mimo_bounds_check_status")
 NOALLOC_STAGING_BYTES = 64 << 20
 
 
@@ -89,6 +89,62 @@ def library_path() -> str:
     return _build.LIB_PATH
 
 
+def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
+    """Argument and result types of every exported function."""
+    L.mimo_params_default.argtypes = [ctypes.POINTER(MimoParams)]
+    L.mimo_params_default.restype = None
+    L.mimo_smart_resize.argtypes = [_i64, _i64, _i64, _i64, _i64, ctypes.POINTER(_i64), ctypes.POINTER(_i64)]
+    L.mimo_smart_resize.restype = ctypes.c_int
+    L.mimo_num_patches.argtypes = [_i64, _i64, ctypes.POINTER(MimoParams), ctypes.POINTER(_i64)]
+    L.mimo_num_patches.restype = ctypes.c_int
+    L.mimo_plan_batch.argtypes = [_i32, _p, _p, ctypes.POINTER(MimoParams), _p, _p]
+    L.mimo_plan_batch.restype = ctypes.c_int
+    L.mimo_preprocess_batch.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p, _i32,
+                                        _p, _i64, _p, _p]
+    L.mimo_preprocess_batch.restype = ctypes.c_int
+    L.mimo_preprocess_batch_ex.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p,
+                                           ctypes.POINTER(MimoOutputs), _p]
+    L.mimo_preprocess_batch_ex.restype = ctypes.c_int
+    L.mimo_preprocess_units.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p, _i64,
+                                        _i64, ctypes.POINTER(MimoOutputs), _p]
+    L.mimo_preprocess_units.restype = ctypes.c_int
+    L.mimo_preprocess_batch_host.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p,
+                                             _i32, _p, _i64, _p, _p, _sz, _p, _i64, _p, _p]
+    L.mimo_preprocess_batch_host.restype = ctypes.c_int
+    L.mimo_preprocess_batch_host_noalloc.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p,
+                                                     _p, _i32, _p, _i64, _p, _p]
+    L.mimo_preprocess_batch_host_noalloc.restype = ctypes.c_int
+    L.mimo_expand_prompt_ids.argtypes = [_p, _i64, _i32, _p, _i64, _p, _i64, ctypes.POINTER(_i64)]
+    L.mimo_expand_prompt_ids.restype = ctypes.c_int
+    L.mimo_video_max_pixels.argtypes = [_i64, _i64, ctypes.POINTER(MimoParams), ctypes.POINTER(_i64)]
+    L.mimo_video_max_pixels.restype = ctypes.c_int
+    L.mimo_smart_nframes.argtypes = [_i64, ctypes.c_double, ctypes.c_double, _i64, _i64,
+                                     ctypes.POINTER(_i64)]
+    L.mimo_smart_nframes.restype = ctypes.c_int
+    L.mimo_sample_frames.argtypes = [_i64, _i64, ctypes.c_double, _p, _p, ctypes.POINTER(_i64)]
+    L.mimo_sample_frames.restype = ctypes.c_int
+    L.mimo_plan_video.argtypes = [_i32, _i32, _i32, _i64, ctypes.POINTER(MimoParams), _p,
+                                  ctypes.POINTER(_i64)]
+    L.mimo_plan_video.restype = ctypes.c_int
+    L.mimo_preprocess_video.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _i64, _i32, _i32, _i32,
+                                        _i64, ctypes.POINTER(MimoOutputs), _p]
+    L.mimo_preprocess_video.restype = ctypes.c_int
+    L.mimo_patch_embed.argtypes = [_p, _i64, _p, _i32, _p, _i32, _p, _p, _p]
+    L.mimo_patch_embed.restype = ctypes.c_int
+    L.mimo_patch_embed_stall_test.argtypes = [_p, _i64, _p, _i32, _p, _i32, _p, _p, _i32, ctypes.c_uint32, _p]
+    L.mimo_patch_embed_stall_test.restype = ctypes.c_int
+    L.mimo_preprocess_embed.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, ctypes.c_size_t, _p, _p, _p, _p,
+                                        _i32, _p, _i32, _p, _i32, _p, _i64, _p, ctypes.c_size_t, _p, _p]
+    L.mimo_preprocess_embed.restype = ctypes.c_int
+    L.mimo_status_string.argtypes = [ctypes.c_int]
+    L.mimo_status_string.restype = ctypes.c_char_p
+    L.mimo_version.argtypes = []
+    L.mimo_version.restype = ctypes.c_int
+    L.mimo_bounds_check_status.argtypes = [ctypes.POINTER(_i64), ctypes.POINTER(_i32)]
+    L.mimo_bounds_check_status.restype = ctypes.c_int
+    return L
+
+
 def lib() -> ctypes.CDLL:
     """The loaded CUDA library; raises if it has not been built."""
     global _lib
@@ -99,53 +155,30 @@ def lib() -> ctypes.CDLL:
                 raise MimoLibraryMissing(
                     f"{path} is missing: build it with `python -m vision_lm_image_b200.build` "
                     "(or __graft_entry__.build()); there is no fallback path")
-            L = ctypes.CDLL(path)
-            L.mimo_params_default.argtypes = [ctypes.POINTER(MimoParams)]
-            L.mimo_params_default.restype = None
-            L.mimo_smart_resize.argtypes = [_i64, _i64, _i64, _i64, _i64, ctypes.POINTER(_i64), ctypes.POINTER(_i64)]
-            L.mimo_smart_resize.restype = ctypes.c_int
-            L.mimo_num_patches.argtypes = [_i64, _i64, ctypes.POINTER(MimoParams), ctypes.POINTER(_i64)]
-            L.mimo_num_patches.restype = ctypes.c_int
-            L.mimo_plan_batch.argtypes = [_i32, _p, _p, ctypes.POINTER(MimoParams), _p, _p]
-            L.mimo_plan_batch.restype = ctypes.c_int
-            L.mimo_preprocess_batch.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p, _i32,
-                                                _p, _i64, _p, _p]
-            L.mimo_preprocess_batch.restype = ctypes.c_int
-            L.mimo_preprocess_batch_ex.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p,
-                                                   ctypes.POINTER(MimoOutputs), _p]
-            L.mimo_preprocess_batch_ex.restype = ctypes.c_int
-            L.mimo_preprocess_batch_host.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p, _p,
-                                                     _i32, _p, _i64, _p, _p, _sz, _p, _i64, _p, _p]
-            L.mimo_preprocess_batch_host.restype = ctypes.c_int
-            L.mimo_preprocess_batch_host_noalloc.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _p, _p, _p,
-                                                             _p, _i32, _p, _i64, _p, _p]
-            L.mimo_preprocess_batch_host_noalloc.restype = ctypes.c_int
-            L.mimo_expand_prompt_ids.argtypes = [_p, _i64, _i32, _p, _i64, _p, _i64, ctypes.POINTER(_i64)]
-            L.mimo_expand_prompt_ids.restype = ctypes.c_int
-            L.mimo_video_max_pixels.argtypes = [_i64, _i64, ctypes.POINTER(MimoParams), ctypes.POINTER(_i64)]
-            L.mimo_video_max_pixels.restype = ctypes.c_int
-            L.mimo_smart_nframes.argtypes = [_i64, ctypes.c_double, ctypes.c_double, _i64, _i64,
-                                             ctypes.POINTER(_i64)]
-            L.mimo_smart_nframes.restype = ctypes.c_int
-            L.mimo_sample_frames.argtypes = [_i64, _i64, ctypes.c_double, _p, _p, ctypes.POINTER(_i64)]
-            L.mimo_sample_frames.restype = ctypes.c_int
-            L.mimo_plan_video.argtypes = [_i32, _i32, _i32, _i64, ctypes.POINTER(MimoParams), _p,
-                                          ctypes.POINTER(_i64)]
-            L.mimo_plan_video.restype = ctypes.c_int
-            L.mimo_preprocess_video.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, _sz, _i64, _i32, _i32, _i32,
-                                                _i64, ctypes.POINTER(MimoOutputs), _p]
-            L.mimo_preprocess_video.restype = ctypes.c_int
-            L.mimo_patch_embed.argtypes = [_p, _i64, _p, _i32, _p, _i32, _p, _p, _p]
-            L.mimo_patch_embed.restype = ctypes.c_int
-            L.mimo_preprocess_embed.argtypes = [ctypes.POINTER(MimoParams), _i32, _p, ctypes.c_size_t, _p, _p, _p, _p,
-                                                _i32, _p, _i32, _p, _i32, _p, _i64, _p, ctypes.c_size_t, _p, _p]
-            L.mimo_preprocess_embed.restype = ctypes.c_int
-            L.mimo_status_string.argtypes = [ctypes.c_int]
-            L.mimo_status_string.restype = ctypes.c_char_p
-            L.mimo_version.argtypes = []
-            L.mimo_version.restype = ctypes.c_int
-            _lib = L
+            _lib = _declare(ctypes.CDLL(path))
     return _lib
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Runs the calls of this module inside the block through another build of the library (for example
+    the bounds-checked debug build), then restores the default one."""
+    global _lib
+    other = _declare(ctypes.CDLL(path))
+    with _lock:
+        saved, _lib = _lib, other
+    try:
+        yield other
+    finally:
+        with _lock:
+            _lib = saved
+
+
+def bounds_check_status() -> tuple[int, int]:
+    """(failed checks since the last query, kind of the first) of a bounds-checked build; clears both."""
+    v, k = _i64(), _i32()
+    _check(lib().mimo_bounds_check_status(ctypes.byref(v), ctypes.byref(k)), "bounds_check_status")
+    return v.value, k.value
 
 
 def _lib_status_string(status: int) -> str:
@@ -417,6 +450,38 @@ def preprocess_batch_ex(params: MimoParams, packed: PackedBatch, out, perm=None,
         ctypes.byref(params), packed.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(),
         *packed.ptrs, ctypes.byref(o), _stream_handle(stream, buf.device))
     _check(st, "preprocess_batch_ex")
+
+
+def preprocess_units(params: MimoParams, packed: PackedBatch, first_unit: int, unit_count: int, out, perm=None,
+                     positions=None, window=None, stream=None) -> None:
+    """Raw ABI call of mimo_preprocess_units: merge units [first_unit, first_unit + unit_count) of the batch.
+
+    ``out`` (and ``positions``) hold the window's rows only, merge order; ``perm`` [total_rows] and
+    ``window`` [total_rows / 4] are batch-global and receive the window's entries."""
+    buf = _packed_buffer(packed)
+    _, offs = plan_batch(packed.heights, packed.widths, params)
+    total = int(offs[-1])
+    f32, bf16, i32, _ = _DTYPES or _dtypes()
+    if perm is not None:
+        _tensor(perm, "perm", buf.device, i32)
+        if perm.numel() < total:
+            raise ValueError(f"perm holds {perm.numel()} entries; the batch has {total} rows")
+    if window is not None:
+        _tensor(window, "window", buf.device, i32)
+        if window.numel() < total // 4:
+            raise ValueError(f"window holds {window.numel()} entries; the batch has {total // 4} merge units")
+    o = MimoOutputs()
+    o.out_dtype = _dtype_code(out.dtype)
+    o.row_order = ORDER_MERGE
+    o.d_out = out.data_ptr()
+    o.out_rows_capacity = _row_capacity(out, "out", buf.device, positions=positions)
+    o.d_column_perm = perm.data_ptr() if perm is not None else None
+    o.d_positions = positions.data_ptr() if positions is not None else None
+    o.d_window_index = window.data_ptr() if window is not None else None
+    st = lib().mimo_preprocess_units(
+        ctypes.byref(params), packed.n, ctypes.c_void_p(buf.data_ptr()), buf.numel(), *packed.ptrs,
+        int(first_unit), int(unit_count), ctypes.byref(o), _stream_handle(stream, buf.device))
+    _check(st, "preprocess_units")
 
 
 def preprocess(images, mean=None, std=None, min_pixels: int | None = None, max_pixels: int | None = None,

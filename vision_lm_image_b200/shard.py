@@ -11,6 +11,12 @@ the same assignment from the same sizes without communicating.
 The batch plan (image_grid_thw, row offsets) stays global: a rank's rows for
 image i are rows [row_offsets[i], row_offsets[i+1]) of the batch, so shards
 can be reassembled, or consumed in place, without renumbering.
+
+Whole images bound the balance of that assignment by the largest image. The
+second plan cuts the batch's merge units instead (unit u = batch rows
+4u..4u+3 in merge order) into one contiguous window per rank, equal up to a
+single unit: an image larger than a rank's share is split by merge-block
+ranges, and each rank runs one mimo_preprocess_units call on its window.
 """
 from __future__ import annotations
 
@@ -52,3 +58,26 @@ def rank_images(images, rank: int, world: int, params=None):
     assign, grid, offs = shard_plan(heights, widths, world, params)
     mine = assign[rank]
     return [images[i] for i in mine], mine, grid, offs
+
+
+def unit_windows(total_units: int, world: int) -> list[tuple[int, int]]:
+    """Contiguous merge-unit windows (first_unit, unit_count), one per rank, tiling [0, total_units) with
+    counts that differ by at most one."""
+    if world <= 0:
+        raise ValueError("world must be positive")
+    if total_units < 0:
+        raise ValueError("total_units must be non-negative")
+    bounds = [r * total_units // world for r in range(world + 1)]
+    return [(bounds[r], bounds[r + 1] - bounds[r]) for r in range(world)]
+
+
+def window_plan(heights: Sequence[int], widths: Sequence[int], world: int, params=None):
+    """Returns (windows per rank, grid_thw [n, 3], row_offsets [n + 1]) for a batch cut by merge units."""
+    grid, offs = mimo.plan_batch(heights, widths, params)
+    return unit_windows(int(offs[-1]) // 4, world), grid, offs
+
+
+def window_images(offs, first_unit: int, unit_count: int) -> list[int]:
+    """Batch indices of the images a window touches (whole or in part)."""
+    lo, hi = 4 * first_unit, 4 * (first_unit + unit_count)
+    return [i for i in range(len(offs) - 1) if offs[i] < hi and offs[i + 1] > lo]
