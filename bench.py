@@ -60,6 +60,9 @@ def parse():
                     help="pe: the patch embedding GEMM on the bf16 rows of c5 (--images sets the image count)")
     ap.add_argument("--embed-dim", type=int, default=1280, help="pe: output width of the patch embedding")
     ap.add_argument("--gemm-only", action="store_true", help="pe: time the GEMM alone (no cuBLAS, no pixel chain)")
+    ap.add_argument("--chain-only", action="store_true",
+                    help="pe: time only mimo_preprocess_embed (uint8 pixels -> embeddings through a scratch)")
+    ap.add_argument("--scratch-mb", type=int, default=192, help="pe: scratch of the chained pixels-to-embeddings call")
     ap.add_argument("--dtype", default=None, choices=["f32", "bf16"])
     ap.add_argument("--images", type=int, default=None, help="override the workload's image count")
     ap.add_argument("--order", default="merge", choices=["merge", "column"], help="row order of the output")
@@ -100,11 +103,14 @@ def kernel_source_digest(kernel: str = "preprocess") -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str, dtype: str, kernel: str = "preprocess", rows: int | None = None):
+def ncu_traffic(workload: str, dtype: str, kernel: str = "preprocess", rows: int | None = None,
+                images: int | None = None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source.
 
-    An entry captured on a smaller case than the launch timed here (``full_rows``
-    differs from ``rows``) is scaled by rows."""
+    An entry with a per-image slope and a fixed offset (two captures of different
+    sizes) is evaluated at ``images``; an entry captured on a smaller case than
+    the launch timed here (``full_rows`` differs from ``rows``) is scaled by rows;
+    an entry captured on the whole workload applies only to that workload."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -115,6 +121,12 @@ def ncu_traffic(workload: str, dtype: str, kernel: str = "preprocess", rows: int
     if not entry or entry.get("kernel_digest") != kernel_source_digest(kernel):
         return None
     traffic = entry.get("dram_bytes_per_launch")
+    if "per_image" in entry:
+        if images is not None:
+            traffic = int(round(entry["per_image"] * images + entry["offset"]))
+        return traffic
+    if "full_rows" not in entry and images is not None and entry.get("full_images", images) != images:
+        return None
     if rows is not None and entry.get("full_rows") and entry["full_rows"] != rows:
         traffic = int(round(traffic * rows / entry["full_rows"]))
     return traffic
@@ -408,7 +420,7 @@ def compare_patch_embed(args, mimo, w, dev, rows, weight, bias, out, err, stream
     # the whole chain from uint8 pixels: two calls over the batch vs the chunked entry point
     params = mimo.make_params(w["mean"], w["std"])
     packed = mimo.pack_images(w["images"], device=dev)
-    scratch = torch.empty(192 << 20, dtype=torch.uint8, device=dev)
+    scratch = torch.empty(args.scratch_mb << 20, dtype=torch.uint8, device=dev)
     two = lambda: (mimo.preprocess_batch_ex(params, packed, rows, None, stream=stream),
                    mimo.patch_embed(rows, weight, bias, out=out, error=err, stream=stream, check=False))
     chain = lambda: mimo.preprocess_embed(packed, weight, bias, w["mean"], w["std"], scratch=scratch, stream=stream,
@@ -419,6 +431,52 @@ def compare_patch_embed(args, mimo, w, dev, rows, weight, bias, out, err, stream
     two_ms = timed(two, args.steps)
     chain_ms = timed(chain, args.steps)
     return lib_ms, two_ms, chain_ms
+
+
+def run_chain_only(args, mimo, w, dev, rank, world):
+    """Images/s of mimo_preprocess_embed alone: uint8 pixels resident in HBM to bf16 embeddings, the bf16
+    rows passing through a scratch of --scratch-mb (what an ncu capture of this command sees is exactly
+    the chained call's kernels)."""
+    import torch
+
+    params = mimo.make_params(w["mean"], w["std"])
+    packed = mimo.pack_images(w["images"], device=dev)
+    N = args.embed_dim
+    g = torch.Generator(device="cpu").manual_seed(17 + rank)
+    weight = (torch.randn((N, 1536), generator=g) * 0.02).to(torch.bfloat16).to(dev)
+    bias = torch.randn(N, generator=g).to(dev)
+    scratch = torch.empty(args.scratch_mb << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    _, offs = mimo.plan_batch(packed.heights, packed.widths, params)
+    M = int(offs[-1])
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    chain = lambda: mimo.preprocess_embed(packed, weight, bias, w["mean"], w["std"], scratch=scratch, stream=stream,
+                                          out=out, error=err, check=False)
+    for _ in range(max(args.warmup, 0)):
+        chain()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        e0.record(stream)
+        for _ in range(args.steps):
+            chain()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if int(err.item()):
+        raise SystemExit(f"patch_embed reported pipeline error {int(err.item())}")
+    ms = e0.elapsed_time(e1) / max(args.steps, 1)
+    n_img = len(w["images"])
+    flops = 2.0 * M * N * 1536
+    if rank == 0:
+        print(json.dumps({
+            "metric": "pixels-to-embeddings images/s (mimo_preprocess_embed)", "value": world * n_img / (ms * 1e-3),
+            "unit": "images/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "pe_chain", "images": n_img, "rows": M, "embed_dim": N,
+                       "scratch_mb": args.scratch_mb},
+            "tflops": flops / (ms * 1e-3) / 1e12, "clocks": clocks.summary(), "e2e": None, "cpu_baseline": None,
+        }), flush=True)
 
 
 def run_patch_embed(args, rank, world, local_rank):
@@ -432,6 +490,9 @@ def run_patch_embed(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = workloads.workload("c5", seed_offset=7919 * rank, n_images=args.images)
+    if args.chain_only:
+        run_chain_only(args, mimo, w, dev, rank, world)
+        return
     rows, _, _ = mimo.preprocess(w["images"], w["mean"], w["std"], dtype=torch.bfloat16, device=dev)
     M, K, N = rows.shape[0], rows.shape[1], args.embed_dim
     g = torch.Generator(device="cpu").manual_seed(17 + rank)
@@ -506,7 +567,7 @@ def run_patch_embed(args, rank, world, local_rank):
                 "impl": "torch.addmm (cuBLAS)", "ms": lib_ms, "tflops": flops / (lib_ms * 1e-3) / 1e12},
             "pixels_to_embeddings": None if args.gemm_only else {"images": n_img, "two_calls_ms": two_ms, "chained_ms": chain_ms,
                                      "two_calls_images_per_s": n_img / (two_ms * 1e-3),
-                                     "chained_images_per_s": n_img / (chain_ms * 1e-3), "scratch_mb": 192},
+                                     "chained_images_per_s": n_img / (chain_ms * 1e-3), "scratch_mb": args.scratch_mb},
             "gpu_launches": args.steps, "clocks": clocks.summary(), "e2e": None, "cpu_baseline": cpu,
         }), flush=True)
 
@@ -552,7 +613,7 @@ def also_config(args, mimo, workloads, name: str, out_dtype: str, dev, stream, s
             "l2": l2_note(nbytes["read"], nbytes["write_rows"] + nbytes["write_perm"]),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
-                         "traffic": ncu_traffic(name, out_dtype),
+                         "traffic": ncu_traffic(name, out_dtype, images=host.n),
                          "algorithmic_bytes_per_launch": nbytes["total"] // launches,
                          "kernel": dominant_kernel(grid, host.heights, host.widths, out_dtype),
                          "avg_launch_ms": ms / launches},
@@ -724,7 +785,7 @@ def run_ours(args, rank, world, local_rank):
             "output_gbs": out_gbs,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
-                         "traffic": ncu_traffic(args.workload, out_dtype),
+                         "traffic": ncu_traffic(args.workload, out_dtype, images=n_img) if window is None else None,
                          "algorithmic_bytes_per_launch": nbytes["total"] // launches_per_step,
                          "kernel": dominant_kernel(grid, host.heights, host.widths, out_dtype),
                          "avg_launch_ms": avg_launch_ms},

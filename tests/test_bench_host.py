@@ -33,10 +33,29 @@ def test_committed_traffic_table_is_consistent():
     # entries name the kernel sources they were captured on (bench.py reports null for any other source)
     with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
         table = json.load(f)
-    for key in ("c5_f32", "c5_bf16", "pe_bf16"):
+    for key in ("c2_f32", "c3_f32", "c4_f32", "c5_f32", "c5_bf16", "pe_bf16"):
         e = table[key]
         assert len(e["kernel_digest"]) == 16 and int(e["kernel_digest"], 16) >= 0
-        assert e["dram_bytes_per_launch"] == e["read"] + e["write"]
+        if "per_image" in e:
+            # two captures: the slope and offset reproduce both, and the full launch is their extrapolation
+            for n, c in e["captures"].items():
+                assert abs(e["per_image"] * int(n) + e["offset"] - (c["read"] + c["write"])) < 2
+            assert e["dram_bytes_per_launch"] == round(e["per_image"] * e["full_images"] + e["offset"])
+        else:
+            assert e["dram_bytes_per_launch"] == e["read"] + e["write"]
+
+
+def test_traffic_fit_is_evaluated_at_the_image_count(tmp_path, monkeypatch):
+    table = {"c5_f32": {"kernel_digest": "x", "dram_bytes_per_launch": 2560, "per_image": 10.0, "offset": -5.0,
+                        "full_images": 256},
+             "c3_f32": {"kernel_digest": "x", "dram_bytes_per_launch": 77, "full_images": 68}}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(table))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_digest", lambda kernel="preprocess": "x")
+    assert bench.ncu_traffic("c5", "f32", images=16) == 155
+    assert bench.ncu_traffic("c3", "f32", images=68) == 77
+    assert bench.ncu_traffic("c3", "f32", images=12) is None  # a whole-workload capture applies to that workload
 
 
 def test_algorithmic_bytes_of_c5():

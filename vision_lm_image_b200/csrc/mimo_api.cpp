@@ -5,6 +5,7 @@
 #include "mimo.h"
 
 #include <cuda_runtime_api.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cfenv>
@@ -18,6 +19,16 @@
 namespace {
 
 constexpr int64_t kFactor = mimo::kBlock;  // patch 16 x merge 2
+
+// NVTX range around a host step (plan, upload, kernel launch, download, wait), so
+// that a timeline profiler shows where a call spends its host time. Without an
+// attached tool a push/pop is a check of one function pointer.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 bool supported_knobs(const mimo_params *p) {
     return p->patch_size == 16 && p->temporal_patch_size == 2 && p->merge_size == 2 && p->reserved == 0;
@@ -158,6 +169,7 @@ struct BatchPlan {
 };
 
 int plan_all(int32_t n, const int32_t *heights, const int32_t *widths, const mimo_params *p, BatchPlan *bp) {
+    NvtxRange range("mimo plan");
     bp->img.resize(static_cast<size_t>(n));
     bp->row0.assign(static_cast<size_t>(n) + 1, 0);
     for (int32_t i = 0; i < n; ++i) {
@@ -245,6 +257,7 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
                  size_t src_bytes, const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
                  const int32_t *channels, int32_t out_dtype, void *d_out, int32_t *d_perm, void *stream,
                  const Tables &tables = Tables(), int64_t row_base = 0, const UnitWindow &win = UnitWindow()) {
+    NvtxRange range("mimo launch");
     static thread_local mimo::LaunchParams lp;  // 31 KB: kept off the stack
     // units of image i inside the window: [lo_i, hi_i) of its own units
     auto unit_span = [&](int32_t i, int64_t *lo_i, int64_t *hi_i) {
@@ -503,13 +516,17 @@ int mimo_preprocess_batch_host(const mimo_params *p, int32_t n, const uint8_t *h
             }
             cudaStream_t s = ss[chunk & 1];
             const int64_t r0 = v.plan.row0[first];
-            if (fail(cudaMemcpyAsync(d_src_stage + lo, h_src + lo, hi - lo, cudaMemcpyHostToDevice, s))) break;
+            {
+                NvtxRange range("mimo upload");
+                if (fail(cudaMemcpyAsync(d_src_stage + lo, h_src + lo, hi - lo, cudaMemcpyHostToDevice, s))) break;
+            }
             const int lst = launch_range(p, v, first, i, d_src_stage, src_bytes, src_offsets, heights, widths, channels,
                                          out_dtype, d_out_stage, h_column_perm ? d_perm_stage : nullptr, s);
             if (lst != MIMO_OK) {
                 result = lst;
                 break;
             }
+            NvtxRange download("mimo download");
             if (fail(cudaMemcpyAsync(static_cast<char *>(h_out) + static_cast<size_t>(r0) * row_bytes,
                                      static_cast<char *>(d_out_stage) + static_cast<size_t>(r0) * row_bytes,
                                      static_cast<size_t>(rows) * row_bytes, cudaMemcpyDeviceToHost, s)))
@@ -521,6 +538,7 @@ int mimo_preprocess_batch_host(const mimo_params *p, int32_t n, const uint8_t *h
             ++chunk;
         }
     }
+    NvtxRange wait("mimo wait");
     for (cudaStream_t s : ss) {
         if (s) {
             fail(cudaStreamSynchronize(s));

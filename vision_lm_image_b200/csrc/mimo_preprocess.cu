@@ -369,18 +369,26 @@ __device__ __forceinline__ void issue_stage(const Params &P, const TapSet &T, ui
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-// The RGB pixel at byte offset o of a staged row, its bytes in bytes 0..2 of
-// the result: two aligned 32-bit shared loads and a funnel shift.
-__device__ __forceinline__ uint32_t rgb_at(const uint8_t *row, uint32_t o) {
+// The two taps of one output column in a contiguously staged RGB row: the
+// pixel at byte offset o in bytes 0..2 of `a`, and in bytes 0..2 of `b` the
+// next pixel, or the same one again at the clamped right edge (`next` false).
+// Three aligned 32-bit shared loads and funnel shifts.
+__device__ __forceinline__ void rgb_pair(const uint8_t *row, uint32_t o, bool next, uint32_t &a, uint32_t &b) {
     const uint32_t *w = reinterpret_cast<const uint32_t *>(row + (o & ~3u));
-    return __funnelshift_r(w[0], w[1], (o & 3u) * 8u);
+    const uint32_t sh = (o & 3u) * 8u;
+    const uint32_t w0 = w[0], w1 = w[1], w2 = w[2];
+    a = __funnelshift_r(w0, w1, sh);
+    const uint32_t hi = __funnelshift_r(w1, w2, sh);
+    b = next ? __funnelshift_r(a, hi, 24) : a;
 }
 
 // Whether block T's staged rows are converted and interpolated along W in one
 // step (RGB, resized width, contiguously staged columns); emit_block then
-// skips its horizontal pass.
+// skips its horizontal pass. Kernels instantiated without the fused step
+// (kFused false: launches with no such image) never take it.
+template <bool kFused>
 __device__ __forceinline__ bool fused_hpass(const TapSet &T) {
-    return T.C == 3 && (T.flags & (kIdentityCols | kGatherCols)) == 0;
+    return kFused && T.C == 3 && (T.flags & (kIdentityCols | kGatherCols)) == 0;
 }
 
 // Converts block T's staged bytes to planar fp32 in the tile (RGBA
@@ -388,14 +396,14 @@ __device__ __forceinline__ bool fused_hpass(const TapSet &T) {
 // For RGB with a resized width a job is instead one quad of output columns of
 // a tile row, interpolated along W on the way (fused_hpass). Gathered columns
 // are loaded here directly from global memory.
-template <class Params>
+template <bool kFused, class Params>
 __device__ __forceinline__ void finish_stage(const Params &P, const TapSet &T, const uint8_t *raw, float *tile,
                                              int TS, int plane, int tid) {
     const int flags = T.flags;
     const int nrows = T.nrows;
     const int C = T.C;
     const float2 m23 = f2(-kTwo23, -kTwo23);
-    if (fused_hpass(T)) {
+    if (fused_hpass<kFused>(T)) {
         // job = (tile row j, output quad q): the two taps of each of the quad's 4 output columns come
         // straight from the staged bytes, and (1 - lx) a + lx b = fma(lx, b - a, a) lands over columns
         // 4q..4q+3 of the tile row. b - a is formed exactly from the 2^23 bit patterns, so the values
@@ -415,18 +423,20 @@ __device__ __forceinline__ void finish_stage(const Params &P, const TapSet &T, c
             const int4 ta = *reinterpret_cast<const int4 *>(&T.tx[0][4 * q]);
             const int4 tb = *reinterpret_cast<const int4 *>(&T.tx[1][4 * q]);
             const float4 l = *reinterpret_cast<const float4 *>(&T.lx[4 * q]);
-            // every tap read stays inside the staged row, every write inside the tile
-            if (!MIMO_CHECK(j < P.tile_rows && 4 * q + 4 <= TS &&
-                                min(min(min(ta.x, ta.y), min(ta.z, ta.w)), min(min(tb.x, tb.y), min(tb.z, tb.w))) >= 0 &&
-                                ((mis + 3u * static_cast<uint32_t>(max(max(max(ta.x, ta.y), max(ta.z, ta.w)),
-                                                                        max(max(tb.x, tb.y), max(tb.z, tb.w))))) &
-                                 ~3u) + 8u <= static_cast<uint32_t>(P.raw_stride),
+            // every tap read (three words from the first tap) stays inside the staged row, every write
+            // inside the tile, and the second tap is the first one or the pixel after it
+            if (!MIMO_CHECK(j < P.tile_rows && 4 * q + 4 <= TS && min(min(ta.x, ta.y), min(ta.z, ta.w)) >= 0 &&
+                                static_cast<unsigned>(tb.x - ta.x) <= 1u && static_cast<unsigned>(tb.y - ta.y) <= 1u &&
+                                static_cast<unsigned>(tb.z - ta.z) <= 1u && static_cast<unsigned>(tb.w - ta.w) <= 1u &&
+                                ((mis + 3u * static_cast<uint32_t>(max(max(ta.x, ta.y), max(ta.z, ta.w)))) & ~3u) +
+                                        12u <= static_cast<uint32_t>(P.raw_stride),
                             kChkSmem))
                 continue;
-            const uint32_t a0 = rgb_at(row, mis + 3u * ta.x), a1 = rgb_at(row, mis + 3u * ta.y);
-            const uint32_t a2 = rgb_at(row, mis + 3u * ta.z), a3 = rgb_at(row, mis + 3u * ta.w);
-            const uint32_t b0 = rgb_at(row, mis + 3u * tb.x), b1 = rgb_at(row, mis + 3u * tb.y);
-            const uint32_t b2 = rgb_at(row, mis + 3u * tb.z), b3 = rgb_at(row, mis + 3u * tb.w);
+            uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+            rgb_pair(row, mis + 3u * ta.x, tb.x != ta.x, a0, b0);
+            rgb_pair(row, mis + 3u * ta.y, tb.y != ta.y, a1, b1);
+            rgb_pair(row, mis + 3u * ta.z, tb.z != ta.z, a2, b2);
+            rgb_pair(row, mis + 3u * ta.w, tb.w != ta.w, a3, b3);
             const float2 l01 = f2(l.x, l.y), l23 = f2(l.z, l.w);
             float *t = tile + j * TS + 4 * q;
 #define MIMO_FUSED_CHANNEL(c)                                                                     \
@@ -590,7 +600,7 @@ __device__ __forceinline__ void write_unit_tables(const Params &P, int tid, int6
 }
 
 // Interpolation, normalisation and stores of one staged block.
-template <bool kBF16, class Params>
+template <bool kBF16, bool kFused, class Params>
 __device__ __forceinline__ void emit_block(const Params &P, const TapSet &T, float *tile, int TS, int plane,
                                            int tid, int warp, int lane) {
     const int flags = T.flags;
@@ -599,7 +609,7 @@ __device__ __forceinline__ void emit_block(const Params &P, const TapSet &T, flo
     // horizontal pass (resized widths only), in place: the warp owning tile
     // row j reads every lane's two taps, then writes the 32 interpolated
     // values over columns 0..31 of the same row
-    const bool hpass = (flags & kIdentityCols) == 0 && !fused_hpass(T);
+    const bool hpass = (flags & kIdentityCols) == 0 && !fused_hpass<kFused>(T);
     if (hpass) {
         const int x0 = T.tx[0][lane], x1 = T.tx[1][lane];
         const float lx = T.lx[lane];
@@ -672,7 +682,7 @@ __device__ __forceinline__ void emit_block(const Params &P, const TapSet &T, flo
 // interpolated and stored, the source bytes of block k+1 are already in
 // shared memory and those of block k+2 are in flight (cp.async), and warps
 // 0-1 compute the taps of the block after.
-template <bool kBF16, class Params>
+template <bool kBF16, bool kFused, class Params>
 __global__ void __launch_bounds__(kThreads, 5) preprocess_kernel(const __grid_constant__ Params P) {
     extern __shared__ float4 smem4[];
     float *const tile = reinterpret_cast<float *>(smem4);  // [3][rows][stride] | raw bytes
@@ -699,16 +709,16 @@ __global__ void __launch_bounds__(kThreads, 5) preprocess_kernel(const __grid_co
     issue_stage(P, S[0], raw, tid);
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    finish_stage(P, S[0], raw, tile, TS, plane, tid);
+    finish_stage<kFused>(P, S[0], raw, tile, TS, plane, tid);
     __syncthreads();
     if (begin + 1 < end) issue_stage(P, S[1], raw, tid);
 
     int slot = 0;
     for (int blk = begin; blk < end; ++blk) {
-        emit_block<kBF16>(P, S[slot], tile, TS, plane, tid, warp, lane);
+        emit_block<kBF16, kFused>(P, S[slot], tile, TS, plane, tid, warp, lane);
         asm volatile("cp.async.wait_all;" ::: "memory");
         __syncthreads();  // tile and S[slot] free; raw holds block blk+1
-        if (blk + 1 < end) finish_stage(P, S[slot ^ 1], raw, tile, TS, plane, tid);
+        if (blk + 1 < end) finish_stage<kFused>(P, S[slot ^ 1], raw, tile, TS, plane, tid);
         if (warp < 2 && blk + 2 < end) compute_taps(P, S[slot], S[slot ^ 1], blk + 2, cur, warp, lane);
         __syncthreads();  // tile holds block blk+1, S[slot] the taps of blk+2, raw is free
         if (blk + 2 < end) issue_stage(P, S[slot], raw, tid);
@@ -954,9 +964,9 @@ struct LaunchSetup {
     int per_sm = 0;
 };
 
-template <bool kBF16, class Params>
+template <bool kBF16, bool kFused, class Params>
 int launch_typed(const Params &lp, int64_t blocks, size_t smem_bytes, cudaStream_t stream) {
-    auto kern = preprocess_kernel<kBF16, Params>;
+    auto kern = preprocess_kernel<kBF16, kFused, Params>;
     static thread_local LaunchSetup setup;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ECUDA;
@@ -1013,11 +1023,14 @@ int launch_direct(const Params &lp, int64_t blocks, cudaStream_t stream) {
 // heights (there the staged kernel's burst reads keep the write stream faster).
 template <class Params>
 int launch_kernels(const Params &lp, int64_t blocks, int out_dtype, size_t smem_bytes, cudaStream_t s) {
-    bool widths_kept = true, heights_kept = true, video = false;
+    bool widths_kept = true, heights_kept = true, video = false, fused = false;
     for (int i = 0; i < lp.n; ++i) {
-        widths_kept = widths_kept && (lp.img[i].flags & kIdentityCols) != 0;
-        heights_kept = heights_kept && (lp.img[i].flags & kIdentityRows) != 0;
-        video = video || (lp.img[i].flags & kVideo) != 0;
+        const int32_t f = lp.img[i].flags;
+        widths_kept = widths_kept && (f & kIdentityCols) != 0;
+        heights_kept = heights_kept && (f & kIdentityRows) != 0;
+        video = video || (f & kVideo) != 0;
+        // an RGB image with a resized, contiguously staged width takes the fused conversion step
+        fused = fused || (((f >> kChannelShift) & 0xFF) == 3 && (f & (kIdentityCols | kGatherCols)) == 0);
     }
     // a video launch carries exactly one clip
     if (widths_kept && (out_dtype == MIMO_BF16 || heights_kept) && (!video || lp.n == 1)) {
@@ -1027,8 +1040,13 @@ int launch_kernels(const Params &lp, int64_t blocks, int out_dtype, size_t smem_
         return out_dtype == MIMO_BF16 ? launch_direct<true, false>(lp, blocks, s)
                                       : launch_direct<false, false>(lp, blocks, s);
     }
-    return out_dtype == MIMO_BF16 ? launch_typed<true>(lp, blocks, smem_bytes, s)
-                                  : launch_typed<false>(lp, blocks, smem_bytes, s);
+    // the staged kernel with the fused RGB step only where a launch needs it: it costs registers
+    // (and measurably some time) in launches that never take it
+    if (fused)
+        return out_dtype == MIMO_BF16 ? launch_typed<true, true>(lp, blocks, smem_bytes, s)
+                                      : launch_typed<false, true>(lp, blocks, smem_bytes, s);
+    return out_dtype == MIMO_BF16 ? launch_typed<true, false>(lp, blocks, smem_bytes, s)
+                                  : launch_typed<false, false>(lp, blocks, smem_bytes, s);
 }
 
 }  // namespace

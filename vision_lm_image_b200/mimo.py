@@ -654,8 +654,11 @@ def patch_embed(rows, weight, bias=None, out_dtype=None, out=None, error=None, s
 
 def preprocess_embed(images, weight, bias=None, mean=None, std=None, min_pixels: int | None = None,
                      max_pixels: int | None = None, out_dtype=None, order: str = "merge",
-                     scratch_bytes: int = 192 << 20, scratch=None, device="cuda", stream=None, check: bool = True):
-    """Pixel path + patch embedding chunk by chunk: returns (embeddings [rows, embed_dim], image_grid_thw)."""
+                     scratch_bytes: int = 192 << 20, scratch=None, device="cuda", stream=None, check: bool = True,
+                     out=None, error=None):
+    """Pixel path + patch embedding chunk by chunk: returns (embeddings [rows, embed_dim], image_grid_thw).
+
+    ``out`` ([rows, embed_dim]) and ``error`` (one int32) may be passed in to be reused across calls."""
     import torch
 
     out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
@@ -676,17 +679,23 @@ def preprocess_embed(images, weight, bias=None, mean=None, std=None, min_pixels:
         _packed_buffer(packed, dev)
         grid, offs = plan_batch(packed.heights, packed.widths, params)
         total = int(offs[-1])
-        out = torch.empty((total, N), dtype=out_dtype, device=dev)
+        if out is None:
+            out = torch.empty((total, N), dtype=out_dtype, device=dev)
+        _tensor(out, "out", dev, cols=N)
+        if int(out.shape[0]) < total:
+            raise ValueError(f"out must hold {total} rows, got {out.shape[0]}")
+        out_dtype = out.dtype
         if scratch is None:
             scratch = torch.empty(scratch_bytes, dtype=torch.uint8, device=dev)
         _tensor(scratch, "scratch", dev, torch.uint8)
-        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev) if error is None else error
+        _tensor(err, "error", dev, torch.int32)
         order_code = {"merge": ORDER_MERGE, "column": ORDER_COLUMN}[order]
         st = lib().mimo_preprocess_embed(
             ctypes.byref(params), packed.n, ctypes.c_void_p(packed.buffer.data_ptr()), packed.buffer.numel(),
             *packed.ptrs, order_code, ctypes.c_void_p(weight.data_ptr()), N,
             ctypes.c_void_p(bias.data_ptr() if bias is not None else 0), _dtype_code(out_dtype),
-            ctypes.c_void_p(out.data_ptr()), total, ctypes.c_void_p(scratch.data_ptr()), scratch.numel(),
+            ctypes.c_void_p(out.data_ptr()), int(out.shape[0]), ctypes.c_void_p(scratch.data_ptr()), scratch.numel(),
             ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, dev))
         _check(st, "preprocess_embed")
     if check:
