@@ -406,7 +406,13 @@ int mimo_patch_embed_stall_test(const void *d_rows, int64_t rows, const void *d_
  *   d_scratch:  device buffer of scratch_bytes, 16-byte aligned, owned by the
  *               caller; half of it must hold one image's rows (rows x 3072
  *               bytes), MIMO_ECAPACITY otherwise. About 2 x 96 MB or more
- *               keeps the GEMMs' last waves full.
+ *               keeps the GEMMs' last waves full. The rows are stored with an
+ *               L2 evict-last policy and, once a GEMM has read a half, its
+ *               lines are dropped from L2 without a write-back (when d_scratch
+ *               is 128-byte aligned): its contents are undefined after the
+ *               call. With halves of one image's rows (a 1080p image: 2 x 26 MB)
+ *               the rows never reach HBM; larger halves trade that for fuller
+ *               GEMM waves.
  * No permutation or index tables (mimo_preprocess_batch_ex writes those).
  * Asynchronous on `stream`. Argument errors return before anything is
  * queued; a CUDA error part-way waits for the second stream's queued GEMMs

@@ -256,7 +256,8 @@ struct UnitWindow {
 int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_t last, const uint8_t *d_src,
                  size_t src_bytes, const int64_t *src_offsets, const int32_t *heights, const int32_t *widths,
                  const int32_t *channels, int32_t out_dtype, void *d_out, int32_t *d_perm, void *stream,
-                 const Tables &tables = Tables(), int64_t row_base = 0, const UnitWindow &win = UnitWindow()) {
+                 const Tables &tables = Tables(), int64_t row_base = 0, const UnitWindow &win = UnitWindow(),
+                 bool keep_rows = false) {
     NvtxRange range("mimo launch");
     static thread_local mimo::LaunchParams lp;  // 31 KB: kept off the stack
     // units of image i inside the window: [lo_i, hi_i) of its own units
@@ -284,6 +285,7 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
         lp.win = tables.win;
         lp.order = tables.order;
         lp.unit0 = static_cast<int32_t>(lo_i);  // the launch's first image may start inside it
+        lp.keep_rows = keep_rows ? 1 : 0;
         fold_normalisation(p, &lp);
         int64_t blocks = 0;
         int32_t tr = 1, tc = 1, k = 0;
@@ -756,7 +758,7 @@ int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src,
         const int64_t rows = v.plan.row0[i1] - row_base;
         if (run >= 2 && cudaStreamWaitEvent(main_s, aux.rows_read[h], 0) != cudaSuccess) return bail(MIMO_ECUDA);
         st = launch_range(p, v, i0, i1, d_src, src_bytes, src_offsets, heights, widths, channels, MIMO_BF16,
-                          halves[h], nullptr, stream, tables, row_base);
+                          halves[h], nullptr, stream, tables, row_base, UnitWindow(), true);
         if (st != MIMO_OK) return bail(st);
         if (cudaEventRecord(aux.rows_ready[h], main_s) != cudaSuccess ||
             cudaStreamWaitEvent(aux.s, aux.rows_ready[h], 0) != cudaSuccess)
@@ -765,6 +767,10 @@ int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src,
                                       static_cast<uint8_t *>(d_out) + static_cast<size_t>(row_base) * embed_dim * esz,
                                       d_error, aux.s);
         if (st != MIMO_OK) return bail(st);
+        // the half has been read: drop its rows from L2 without writing them back to HBM (a scratch that
+        // is not 128-byte aligned keeps them; they are then written back as usual)
+        st = mimo::launch_discard_l2(halves[h], rows * row_bytes, aux.s);
+        if (st != MIMO_OK && st != MIMO_EALIGN) return bail(st);
         if (cudaEventRecord(aux.rows_read[h], aux.s) != cudaSuccess) return bail(MIMO_ECUDA);
         i0 = i1;
     }

@@ -85,6 +85,8 @@ struct LaunchParamsT {
     int32_t tile_stride; // row stride (floats, multiple of 4) of the tile
     int32_t raw;         // float offset of the raw staging rows
     int32_t raw_stride;  // bytes per raw staging row (multiple of 16)
+    int32_t keep_rows;   // bf16 rows read again right away (chained patch embedding): stored with L2 evict-last
+    int32_t pad1;
 #if defined(MIMO_BOUNDS_CHECK)
     int64_t chk_row_lo, chk_row_hi;  // rows the kernel may emit (its own row numbering)
     int64_t chk_table_rows;          // rows the permutation covers (window index: a quarter)
@@ -131,6 +133,10 @@ MIMO_HD int64_t block_span(int64_t b, int64_t in, int64_t out) {
 }
 
 int launch_preprocess(const LaunchParams &lp, int64_t blocks, int out_dtype, size_t smem_bytes, void *stream);
+
+// Drops `bytes` from `p` (128-byte aligned) out of L2 without writing them back
+// (their contents become undefined), on `stream`.
+int launch_discard_l2(void *p, int64_t bytes, void *stream);
 
 #if defined(MIMO_BOUNDS_CHECK) && defined(__CUDACC__)
 __device__ bool bounds_ok(bool ok, int kind);

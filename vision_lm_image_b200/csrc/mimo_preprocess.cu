@@ -565,8 +565,21 @@ __device__ __forceinline__ void store_quad(const Params &P, int64_t row, int c, 
         uint2 u;
         u.x = *reinterpret_cast<const uint32_t *>(&lo2);
         u.y = *reinterpret_cast<const uint32_t *>(&hi2);
-        __stcs(reinterpret_cast<uint2 *>(o), u);
-        if (both) __stcs(reinterpret_cast<uint2 *>(o + 256), u);
+        if (P.keep_rows) {
+            // rows that the patch embedding reads right after this launch (mimo_preprocess_embed): stored
+            // with an L2 evict-last policy so that they are read back from L2, not from HBM
+            uint64_t pol;
+            asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+            asm volatile("st.global.L2::cache_hint.v2.b32 [%0], {%1, %2}, %3;" ::"l"(o), "r"(u.x), "r"(u.y), "l"(pol)
+                         : "memory");
+            if (both)
+                asm volatile("st.global.L2::cache_hint.v2.b32 [%0], {%1, %2}, %3;" ::"l"(o + 256), "r"(u.x), "r"(u.y),
+                             "l"(pol)
+                             : "memory");
+        } else {
+            __stcs(reinterpret_cast<uint2 *>(o), u);
+            if (both) __stcs(reinterpret_cast<uint2 *>(o + 256), u);
+        }
     }
 }
 
@@ -1050,6 +1063,27 @@ int launch_kernels(const Params &lp, int64_t blocks, int out_dtype, size_t smem_
 }
 
 }  // namespace
+
+namespace {
+// Drops 128-byte lines from L2 without writing them back to HBM. The chained
+// pixels-to-embeddings call runs it over a scratch half once the GEMM has read
+// it: those rows are dead, and writing them back would cost HBM bandwidth.
+__global__ void discard_l2_kernel(uint8_t *p, int64_t lines) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < lines;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        asm volatile("discard.global.L2 [%0], 128;" ::"l"(p + 128 * i) : "memory");
+}
+}  // namespace
+
+int launch_discard_l2(void *p, int64_t bytes, void *stream) {
+    if ((reinterpret_cast<uintptr_t>(p) & 127u) != 0) return MIMO_EALIGN;
+    const int64_t lines = bytes / 128;
+    if (lines <= 0) return MIMO_OK;
+    const int64_t blocks = std::min<int64_t>((lines + 255) / 256, 148 * 8);
+    discard_l2_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint8_t *>(p), lines);
+    return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
+}
 
 int bounds_check_status(int64_t *violations, int32_t *first_kind) {
 #if defined(MIMO_BOUNDS_CHECK)
