@@ -96,10 +96,18 @@ KERNEL_SOURCES = {
 
 
 def kernel_source_digest(kernel: str = "preprocess") -> str:
+    """Digest of a kernel's source code, comments and blank lines left out (a comment edit does not
+    make a capture of the same code stale)."""
+    import re
+
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(code.encode())
     return h.hexdigest()[:16]
 
 

@@ -10,7 +10,9 @@
 //     with 16-byte cp.async, then converts them to planar fp32 on the 0..255
 //     scale, compositing RGBA onto white on the way (function _to_rgb);
 //   - interpolates along W for every staged row, in place (skipped when the
-//     width is not resized), then along H with packed f32x2 arithmetic, applies
+//     width is not resized; for RGB images this step and the conversion are
+//     one: each job reads its output columns' two taps straight from the
+//     staged bytes), then along H with packed f32x2 arithmetic, applies
 //     (x - 255*mean)/(255*std) folded to x*k + b (module docstring), and
 //     writes each 16-pixel row segment twice, once per temporal frame, laid
 //     out (c, tt, py, px) in merge-block row order (cortiq page, conventions);
@@ -18,8 +20,10 @@
 //     page, column_permutation).
 // CTAs are persistent: each takes a contiguous range of blocks and overlaps
 // the source copies of the next blocks with the stores of the current one.
-// Launches whose images or frames all keep their width go to a second,
-// unstaged kernel (direct_kernel below) when that measured faster.
+// The staged kernel is instantiated with and without the fused RGB step; a
+// launch takes the fused one only when one of its images needs it. Launches
+// whose images or frames all keep their width go to a second, unstaged kernel
+// (direct_kernel below) when that measured faster.
 // There is no inter-CTA communication, no atomics and no global wait; every
 // output element has exactly one writer.
 #include <cuda_bf16.h>
