@@ -124,3 +124,18 @@ def test_reference_arm_config_equals_the_main_arm_config():
                                     sum(int(im.size) for im in w["images"]))
         assert ours == ref
         assert set(ours) >= {"workload", "images_per_gpu", "rows_per_gpu", "row_order", "out_dtype", "l2"}
+
+
+def test_kernel_digest_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    src = tmp_path / "vision_lm_image_b200" / "csrc"
+    src.mkdir(parents=True)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", {"k": ("vision_lm_image_b200/csrc/a.cu",)})
+
+    def digest(text):
+        (src / "a.cu").write_text(text)
+        return bench.kernel_source_digest("k")
+
+    base = digest("int f(int x) {\n    return x + 1;\n}\n")
+    assert digest("// a note\nint f(int x) {  /* the sum */\n\n    return x + 1;  // one more\n}\n") == base
+    assert digest("int f(int x) {\n    return x + 2;\n}\n") != base
