@@ -141,3 +141,28 @@ def test_unit_windows_properties():
             assert max(c for _, c in w) - min(c for _, c in w) <= 1
     with pytest.raises(ValueError):
         shard.unit_windows(5, 0)
+
+
+def _gather_worker(rank, world, port, units, q):
+    import torch
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        windows = shard.unit_windows(units, world)
+        first, count = windows[rank]
+        # stand-in rows: row r of the batch holds r in every column
+        rows = torch.arange(4 * first, 4 * (first + count), dtype=torch.float32).repeat_interleave(6).view(-1, 6)
+        out = shard.gather_windows(rows, windows, dst=0)
+        q.put(None if out is None else out.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,units", [(2, 8100), (3, 7)])
+def test_gather_windows_reassembles_the_batch_gloo(world, units):
+    res = _run_ranks(_gather_worker, world, units)
+    # _run_ranks keeps the one result that is not None: rank 0's gathered rows
+    assert res is not None and res.shape == (4 * units, 6)
+    assert np.array_equal(res[:, 0], np.arange(4 * units, dtype=np.float32))
+    assert (res == res[:, :1]).all()

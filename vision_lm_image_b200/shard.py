@@ -81,3 +81,40 @@ def window_images(offs, first_unit: int, unit_count: int) -> list[int]:
     """Batch indices of the images a window touches (whole or in part)."""
     lo, hi = 4 * first_unit, 4 * (first_unit + unit_count)
     return [i for i in range(len(offs) - 1) if offs[i] < hi and offs[i + 1] > lo]
+
+
+def gather_windows(local_rows, windows: Sequence[tuple[int, int]], dst: int = 0, group=None, out=None):
+    """Collects every rank's window rows on rank ``dst`` in batch row order.
+
+    Each rank passes the rows of its own merge-unit window (``local_rows``: [4 * count, cols], as written by
+    mimo_preprocess_units) and the shared window plan. Rank ``dst`` receives the other windows with one
+    grouped batch of point-to-point transfers (NCCL send/recv over NVLink for CUDA tensors) straight into
+    the matching row ranges of ``out`` ([total_rows, cols], allocated when not given) and returns it; the
+    other ranks send theirs and return None. No collective touches the data path before this call."""
+    import torch
+    import torch.distributed as dist
+
+    rank = dist.get_rank(group)
+    world = dist.get_world_size(group)
+    if len(windows) != world:
+        raise ValueError("one window per rank")
+    first, count = windows[rank]
+    if local_rows.shape[0] != 4 * count:
+        raise ValueError(f"rank {rank} holds {local_rows.shape[0]} rows for a window of {count} merge units")
+    total = 4 * (windows[-1][0] + windows[-1][1])
+    if rank != dst:
+        if count:
+            dist.send(local_rows.contiguous(), dst=dist.get_global_rank(group, dst) if group else dst, group=group)
+        return None
+    if out is None:
+        out = torch.empty((total,) + tuple(local_rows.shape[1:]), dtype=local_rows.dtype, device=local_rows.device)
+    out[4 * first:4 * (first + count)].copy_(local_rows)
+    ops = []
+    for r, (f, c) in enumerate(windows):
+        if r == dst or c == 0:
+            continue
+        src = dist.get_global_rank(group, r) if group else r
+        ops.append(dist.P2POp(dist.irecv, out[4 * f:4 * (f + c)], src, group))
+    for w in dist.batch_isend_irecv(ops) if ops else []:
+        w.wait()
+    return out
