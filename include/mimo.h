@@ -371,9 +371,9 @@ int mimo_patch_embed(const void *d_rows, int64_t rows, const void *d_weight, int
 
 /*
  * Test hook for the failure path of mimo_patch_embed; no counterpart on the
- * pages. The same launch, except that the operand loader of every CTA stops
- * after stop_after_kblocks 64-wide K blocks of its first tile (0 ..
- * 1536 / 64), so the tensor-core pipeline waits for operands that never
+ * pages. The same launch, except that the operand loaders of every CTA stop
+ * after stop_after_kblocks 128-wide K blocks of its first tile (0 ..
+ * 1536 / 128), so the tensor-core pipeline waits for operands that never
  * arrive, and each wait gives up after wait_rounds polling rounds (> 0)
  * instead of the default 2^20. The kernel then records a nonzero code in
  * *d_error (1: operands, 3: accumulator; the first role to give up wins),

@@ -680,7 +680,7 @@ int mimo_patch_embed_stall_test(const void *d_rows, int64_t rows, const void *d_
                                 int32_t stop_after_kblocks, uint32_t wait_rounds, void *stream) {
     if (rows <= 0 || embed_dim <= 0 || (embed_dim % 256) != 0) return MIMO_EINVAL;
     if (out_dtype != MIMO_F32 && out_dtype != MIMO_BF16) return MIMO_EINVAL;
-    if (stop_after_kblocks < 0 || stop_after_kblocks > mimo::kRowWidth / 64 || wait_rounds == 0) return MIMO_EINVAL;
+    if (stop_after_kblocks < 0 || stop_after_kblocks > mimo::kRowWidth / 128 || wait_rounds == 0) return MIMO_EINVAL;
     if (!d_rows || !d_weight || !d_out || !d_error) return MIMO_EINVAL;
     if (!aligned16(d_rows) || !aligned16(d_weight) || !aligned16(d_out) || (d_bias && !aligned16(d_bias)) ||
         (reinterpret_cast<uintptr_t>(d_error) & 3u) != 0)

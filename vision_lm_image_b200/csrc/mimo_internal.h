@@ -147,7 +147,7 @@ int bounds_check_status(int64_t *violations, int32_t *first_kind);
 
 // Patch embedding GEMM on the tensor cores (mimo_patch_embed.cu). wait_rounds
 // = 0 keeps the default wait limit; stop_after >= 0 (tests of the failure path
-// only) stops each CTA's operand loader after that many 64-wide K blocks.
+// only) stops each CTA's operand loaders after that many 128-wide K blocks.
 int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_weight, int32_t N, const float *d_bias,
                        int32_t out_dtype, void *d_out, int32_t *d_err, void *stream, uint32_t wait_rounds = 0,
                        int32_t stop_after = -1);

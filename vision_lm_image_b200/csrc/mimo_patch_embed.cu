@@ -12,11 +12,15 @@
 // tiles of C in m-major order (the embed_dim / 256 tiles that share rows run
 // side by side, so each row block is read from HBM once). Each CTA of a pair
 // holds half of A (128 rows) and half of B (128 of the 256 weight rows) per
-// 64-wide K block; warp 0 of each CTA streams them with TMA (128-byte swizzle)
-// into a 6-stage ring and both halves signal the even CTA's barrier. One lane
-// of the even CTA issues tcgen05.mma.cta_group::2 (M256 N256 K16: the tensor
-// cores of both SMs, each reading its own half of A and both halves of B) and
-// frees each stage in both CTAs with a multicast tcgen05.commit. Warps 2-5 of
+// 128-wide K block, as two 64-wide halves in the 128-byte swizzle; warp 0 of
+// each CTA streams its A with TMA and warp 6 its B, into a 3-stage ring, and
+// all of it signals the even CTA's barrier. One lane of the even CTA issues
+// tcgen05.mma.cta_group::2 (M256 N256 K16: the tensor cores of both SMs, each
+// reading its own half of A and both halves of B), eight per stage, and frees
+// each stage in both CTAs with a multicast tcgen05.commit. A stage of 128 K
+// (1024 tensor-core cycles per SM) rather than 64 is what lets one thread keep
+// the tensor pipe fed: each barrier wait, copy issue and commit costs that
+// thread a few hundred cycles, and one tcgen05.mma about 80. Warps 2-5 of
 // each CTA drain their 128 accumulator rows with tcgen05.ld, add the bias,
 // convert and store. TMEM holds two accumulators (2 x 256 columns) per CTA, so
 // the epilogue of one tile runs under the MMAs of the next. Splitting the tile
@@ -43,13 +47,16 @@ constexpr int kPairM = 256;                // rows of C per tile (128 per CTA of
 constexpr int kBM = 128;                    // rows of A per CTA
 constexpr int kBN = 256;                    // columns of C per tile
 constexpr int kBNHalf = kBN / 2;            // weight rows per CTA
-constexpr int kBK = 64;                     // kBK * 2 B = one 128-byte swizzle row
-constexpr int kStages = 6;
+constexpr int kBK = 128;                    // K per stage
+constexpr int kAtomK = 64;                  // kAtomK * 2 B = one 128-byte swizzle row (one TMA box)
+constexpr int kStages = 3;
 constexpr int kUmmaK = 16;
-constexpr int kATileBytes = kBM * kBK * 2;      // 16 KB
-constexpr int kBTileBytes = kBNHalf * kBK * 2;  // 16 KB
+constexpr int kAAtomBytes = kBM * kAtomK * 2;      // 16 KB: 128 rows of one 64-wide half
+constexpr int kBAtomBytes = kBNHalf * kAtomK * 2;  // 16 KB
+constexpr int kATileBytes = kBM * kBK * 2;         // 32 KB
+constexpr int kBTileBytes = kBNHalf * kBK * 2;     // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
-constexpr int kGemmThreads = 192;           // 6 warps
+constexpr int kGemmThreads = 224;           // 7 warps: A loader, MMA, 4 epilogue, B loader
 constexpr int kAccCols = kBN;               // one fp32 accumulator: 128 lanes x 256 columns per CTA
 constexpr int kTmemCols = 2 * kAccCols;     // double-buffered
 constexpr int kEpiWarps = 4;
@@ -258,8 +265,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = S.tmem_base;
 
-    if (warp == 0) {
-        // ---- producer (both CTAs): this CTA's halves of A and B, k-block counter g runs across tiles
+    if (warp == 0 || warp == 6) {
+        // ---- producers (both CTAs): warp 0 this CTA's half of A, warp 6 its half of B; the
+        // k-block counter g runs across tiles
+        const bool loads_a = warp == 0;
         if (lane == 0) {
             uint32_t g = 0;
             for (int64_t t = pair; t < total_tiles && !stopped(S); t += pairs) {
@@ -275,15 +284,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     if (stopped(S)) break;
                     uint8_t *a = tiles + s * kStageBytes;
-                    if (leader) mbar_expect_tx(&S.full[s], 2 * kStageBytes);  // both CTAs' halves
                     const uint32_t full_bar = cluster_addr(&S.full[s], 0);
-                    tma_load_2d_pair(a, &map_a, full_bar, kb * kBK, a_row);
-                    tma_load_2d_pair(a + kATileBytes, &map_b, full_bar, kb * kBK, b_row);
+                    // The B bytes may land before the expectation is posted: the transaction count of
+                    // the phase goes negative for a while, and the phase cannot complete before the
+                    // single arrival below.
+                    if (loads_a) {
+                        if (leader) mbar_expect_tx(&S.full[s], 2 * kStageBytes);  // both CTAs, A and B
+                        tma_load_2d_pair(a, &map_a, full_bar, kb * kBK, a_row);
+                        tma_load_2d_pair(a + kAAtomBytes, &map_a, full_bar, kb * kBK + kAtomK, a_row);
+                    } else {
+                        uint8_t *b = a + kATileBytes;
+                        tma_load_2d_pair(b, &map_b, full_bar, kb * kBK, b_row);
+                        tma_load_2d_pair(b + kBAtomBytes, &map_b, full_bar, kb * kBK + kAtomK, b_row);
+                    }
                 }
             }
             // copies still in flight land before the CTA can leave (bounded; the even
-            // CTA's barrier counts the peer's copies as well)
-            if (leader)
+            // CTA's barrier counts the B loader's and the peer's copies as well)
+            if (leader && loads_a)
                 for (uint32_t q = (g > kStages ? g - kStages : 0); q < g; ++q)
                     mbar_wait(&S.full[q % kStages], (q / kStages) & 1, wait_limit);
         }
@@ -312,9 +330,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t bb = a + kATileBytes;
 #pragma unroll
                     for (int k = 0; k < kBK / kUmmaK; ++k) {
-                        // advancing 16 bf16 (32 bytes) inside the swizzled 128-byte row
-                        const uint64_t da = kmajor_sw128_desc(a + k * kUmmaK * 2);
-                        const uint64_t db = kmajor_sw128_desc(bb + k * kUmmaK * 2);
+                        // 64-wide half k / 4, then 16 bf16 (32 bytes) at a time inside its swizzled 128-byte rows
+                        const int h = k / (kAtomK / kUmmaK), kk = k % (kAtomK / kUmmaK);
+                        const uint64_t da = kmajor_sw128_desc(a + h * kAAtomBytes + kk * kUmmaK * 2);
+                        const uint64_t db = kmajor_sw128_desc(bb + h * kBAtomBytes + kk * kUmmaK * 2);
                         const uint32_t accumulate = (kb > 0 || k > 0) ? 1u : 0u;
                         asm volatile(
                             "{\n\t.reg .pred p;\n\t"
@@ -332,7 +351,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             umma_commit_local(&S.drain);
             if (!mbar_wait(&S.drain, 0, wait_limit)) fail(S, err, kErrDrainWait);
         }
-    } else {
+    } else if (warp <= 5) {
         // ---- epilogue (both CTAs): warp w reads TMEM lanes 32*(w % 4) .. +31 (its accessible quarter)
         const int quarter = warp & 3;
         uint8_t *stage = tiles + kStages * kStageBytes + (warp - 2) * kEpiStageBytes;
@@ -419,7 +438,7 @@ bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, in
     if (!fn) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kAtomK), static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
