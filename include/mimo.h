@@ -27,7 +27,7 @@
  *   - Ownership: the caller owns every buffer. The library never allocates
  *     or frees device memory at run time. Between calls it keeps:
  *       - the fixed staging area of mimo_preprocess_batch_host_noalloc;
- *       - the second stream and events of mimo_preprocess_embed, per host
+ *       - the two streams and events of mimo_preprocess_embed, per host
  *         thread and device;
  *       - cached device attributes (SM count, occupancy, shared-memory
  *         opt-in).
@@ -392,10 +392,11 @@ int mimo_patch_embed_stall_test(const void *d_rows, int64_t rows, const void *d_
  * Images are grouped into runs whose bf16 patch rows fit half of d_scratch;
  * the runs alternate between the two halves. The pixel kernel writes a run's
  * rows on `stream`, and the patch-embedding GEMM (as mimo_patch_embed) reads
- * them on a second stream the library keeps per host thread and device, so it
- * overlaps the next run's pixel kernel. Events order each GEMM after its rows
- * and each reuse of a half after the GEMM that read it; `stream` finally waits
- * for the last GEMMs. Equal, bit for bit, to mimo_preprocess_batch_ex with
+ * them on one of two streams the library keeps per host thread and device,
+ * one per half, so it overlaps the next run's pixel kernel, and the next
+ * run's GEMM can fill the SMs its last wave leaves idle. Events order each
+ * GEMM after its rows and each reuse of a half after the GEMM that read it;
+ * `stream` finally waits for both. Equal, bit for bit, to mimo_preprocess_batch_ex with
  * MIMO_BF16 rows followed by mimo_patch_embed on them.
  *   p, n, d_src, src_bytes, src_offsets, heights, widths, channels: as in
  *       mimo_preprocess_batch.
@@ -415,7 +416,7 @@ int mimo_patch_embed_stall_test(const void *d_rows, int64_t rows, const void *d_
  *               GEMM waves.
  * No permutation or index tables (mimo_preprocess_batch_ex writes those).
  * Asynchronous on `stream`. Argument errors return before anything is
- * queued; a CUDA error part-way waits for the second stream's queued GEMMs
+ * queued; a CUDA error part-way waits for the library streams' queued GEMMs
  * before it returns, so none of them runs after the call.
  */
 int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src, size_t src_bytes,

@@ -707,18 +707,20 @@ int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src,
         return MIMO_EALIGN;
     if (v.total_rows > (int64_t(1) << 31) - 1) return MIMO_EOVERFLOW;
     // runs of whole images alternate between the two halves of the scratch. The pixel kernel of run r
-    // goes on the caller's stream, the GEMM of run r on a second stream of the library's, so that it
-    // overlaps the pixel kernel of run r + 1 (the unstaged pixel kernel holds no shared memory and fits
-    // beside the GEMM's CTAs). Events order each GEMM after its run's rows and each reuse of a half after
-    // the GEMM that read it; the caller's stream finally waits for the last GEMMs.
+    // goes on the caller's stream, the GEMM of run r on a stream of the library's that belongs to its
+    // half, so that it overlaps the pixel kernel of run r + 1 (the unstaged pixel kernel holds no shared
+    // memory and fits beside the GEMM's CTAs) and the GEMM of run r + 1 can start on the SMs that the
+    // last, partial wave of run r's tiles leaves idle. Events order each GEMM after its run's rows and
+    // each reuse of a half after the GEMM that read it; the caller's stream finally waits for both.
+    // (Four slots of one run each, rotating, measured no faster than two halves.)
     const int64_t row_bytes = static_cast<int64_t>(mimo::kRowWidth) * 2;
     const int64_t run_rows = static_cast<int64_t>(scratch_bytes / 2) / row_bytes;
     for (int32_t i = 0; i < n; ++i)
         if (v.plan.row0[i + 1] - v.plan.row0[i] > run_rows) return MIMO_ECAPACITY;  // exceeds half the scratch
-    // the second stream and its events, made once per host thread and device
+    // the two streams and their events, made once per host thread and device
     struct Aux {
         bool ready = false;
-        cudaStream_t s = nullptr;
+        cudaStream_t s[2] = {nullptr, nullptr};
         cudaEvent_t rows_ready[2] = {nullptr, nullptr}, rows_read[2] = {nullptr, nullptr};
     };
     constexpr int kMaxDevices = 64;
@@ -728,9 +730,9 @@ int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src,
     Aux &aux = aux_of[dev];
     if (!aux.ready) {
         // handles made before a failed creation are kept and reused by the next attempt
-        if (!aux.s && cudaStreamCreateWithFlags(&aux.s, cudaStreamNonBlocking) != cudaSuccess) return MIMO_ECUDA;
         for (int k = 0; k < 2; ++k)
-            if ((!aux.rows_ready[k] && cudaEventCreateWithFlags(&aux.rows_ready[k], cudaEventDisableTiming) !=
+            if ((!aux.s[k] && cudaStreamCreateWithFlags(&aux.s[k], cudaStreamNonBlocking) != cudaSuccess) ||
+                (!aux.rows_ready[k] && cudaEventCreateWithFlags(&aux.rows_ready[k], cudaEventDisableTiming) !=
                                            cudaSuccess) ||
                 (!aux.rows_read[k] &&
                  cudaEventCreateWithFlags(&aux.rows_read[k], cudaEventDisableTiming) != cudaSuccess))
@@ -738,10 +740,11 @@ int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src,
         aux.ready = true;
     }
     cudaStream_t main_s = static_cast<cudaStream_t>(stream);
-    // an error after the first enqueue waits for the second stream's work, so
+    // an error after the first enqueue waits for the library streams' work, so
     // that no GEMM still reads the scratch or writes d_out after the return
     auto bail = [&aux](int status) {
-        cudaStreamSynchronize(aux.s);
+        cudaStreamSynchronize(aux.s[0]);
+        cudaStreamSynchronize(aux.s[1]);
         return status;
     };
     uint8_t *halves[2] = {static_cast<uint8_t *>(d_scratch), static_cast<uint8_t *>(d_scratch) + run_rows * row_bytes};
@@ -761,17 +764,17 @@ int mimo_preprocess_embed(const mimo_params *p, int32_t n, const uint8_t *d_src,
                           halves[h], nullptr, stream, tables, row_base, UnitWindow(), true);
         if (st != MIMO_OK) return bail(st);
         if (cudaEventRecord(aux.rows_ready[h], main_s) != cudaSuccess ||
-            cudaStreamWaitEvent(aux.s, aux.rows_ready[h], 0) != cudaSuccess)
+            cudaStreamWaitEvent(aux.s[h], aux.rows_ready[h], 0) != cudaSuccess)
             return bail(MIMO_ECUDA);
         st = mimo::launch_patch_embed(halves[h], rows, mimo::kRowWidth, d_weight, embed_dim, d_bias, out_dtype,
                                       static_cast<uint8_t *>(d_out) + static_cast<size_t>(row_base) * embed_dim * esz,
-                                      d_error, aux.s);
+                                      d_error, aux.s[h]);
         if (st != MIMO_OK) return bail(st);
         // the half has been read: drop its rows from L2 without writing them back to HBM (a scratch that
         // is not 128-byte aligned keeps them; they are then written back as usual)
-        st = mimo::launch_discard_l2(halves[h], rows * row_bytes, aux.s);
+        st = mimo::launch_discard_l2(halves[h], rows * row_bytes, aux.s[h]);
         if (st != MIMO_OK && st != MIMO_EALIGN) return bail(st);
-        if (cudaEventRecord(aux.rows_read[h], aux.s) != cudaSuccess) return bail(MIMO_ECUDA);
+        if (cudaEventRecord(aux.rows_read[h], aux.s[h]) != cudaSuccess) return bail(MIMO_ECUDA);
         i0 = i1;
     }
     // the caller's stream sees every GEMM done

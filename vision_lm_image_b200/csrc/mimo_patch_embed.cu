@@ -455,10 +455,19 @@ int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_w
     if (!make_map(&ma, d_rows, M, K, kBM) || !make_map(&mb, d_weight, N, K, kBNHalf)) return MIMO_ECUDA;
     const int64_t tiles = ((M + kPairM - 1) / kPairM) * (N / kBN);
     const size_t smem = static_cast<size_t>(kStages) * kStageBytes + kEpiWarps * kEpiStageBytes + 1024;
-    auto kernel = out_dtype == MIMO_BF16 ? patch_embed_kernel<true> : patch_embed_kernel<false>;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-        cudaSuccess)
-        return MIMO_ECUDA;
+    const int out_bf16 = out_dtype == MIMO_BF16 ? 1 : 0;
+    auto kernel = out_bf16 ? patch_embed_kernel<true> : patch_embed_kernel<false>;
+    // per host thread and device: the shared-memory opt-in and the number of
+    // resident CTA pairs, looked up on the first launch (a chained call
+    // launches this kernel once per run of images)
+    struct Setup {
+        int max_pairs[2] = {0, 0};
+    };
+    constexpr int kMaxDevices = 64;
+    static thread_local Setup setup_of[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MIMO_ECUDA;
+    int &max_pairs = setup_of[dev].max_pairs[out_bf16];
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -471,12 +480,16 @@ int launch_patch_embed(const void *d_rows, int64_t M, int32_t K, const void *d_w
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     // persistent: as many pairs as can be resident at once (one CTA per SM)
-    int dev = 0, sms = 0, max_pairs = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2)
-        return MIMO_ECUDA;
-    cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
-    if (cudaOccupancyMaxActiveClusters(&max_pairs, kernel, &cfg) != cudaSuccess || max_pairs < 1) return MIMO_ECUDA;
+    if (max_pairs < 1) {
+        int sms = 0, found = 0;
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2)
+            return MIMO_ECUDA;
+        cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
+        if (cudaOccupancyMaxActiveClusters(&found, kernel, &cfg) != cudaSuccess || found < 1) return MIMO_ECUDA;
+        max_pairs = found;
+    }
     const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
     if (cudaLaunchKernelEx(&cfg, kernel, ma, mb, d_bias, d_out, M, N, K, d_err, wait_limit, stop_after) !=
