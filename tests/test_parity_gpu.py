@@ -541,6 +541,23 @@ def test_preprocess_embed_equals_two_step(order, out_dtype):
                        ref.view(torch.int16 if out_dtype == torch.bfloat16 else torch.int32))
 
 
+def test_preprocess_embed_one_image_runs_equal_two_step():
+    # 1080p images (8,160 rows: 160 GEMM tiles, a ragged last wave on the CTA pairs) through a scratch whose
+    # halves hold exactly one image: five runs alternate over the two halves and their two library streams,
+    # so consecutive GEMMs overlap; bit for bit the two calls on the whole batch
+    w5 = workloads.workload("c5", n_images=5)
+    g = torch.Generator(device="cpu").manual_seed(6)
+    w = (torch.randn((1280, 1536), generator=g) * 0.02).to(torch.bfloat16).cuda()
+    bias = torch.randn(1280, generator=g).cuda()
+    rows, grid, _ = mimo.preprocess(w5["images"], w5["mean"], w5["std"], dtype=torch.bfloat16)
+    ref = mimo.patch_embed(rows, w, bias)
+    for _ in range(2):  # the second call reuses the library's streams and events
+        emb, grid2 = mimo.preprocess_embed(w5["images"], w, bias, w5["mean"], w5["std"],
+                                           scratch_bytes=2 * 8160 * 3072)
+        assert torch.equal(grid, grid2)
+        assert torch.equal(emb.view(torch.int16), ref.view(torch.int16))
+
+
 def test_preprocess_embed_c5_sample_against_oracle():
     # full-size geometry (1080x1920 -> 8160 rows each, RGB and RGBA), default scratch; sampled rows vs the oracle chain
     w5 = workloads.workload("c5", n_images=4)
