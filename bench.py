@@ -28,7 +28,9 @@ Also reported on the same JSON line:
                timed region;
   also         (default c5 fp32 line, one GPU) the two other configurations held
                to the bandwidth target, c5 with bf16 rows and c3 with fp32 rows,
-               each timed the same way in this process with its own roofline.
+               each timed the same way in this process with its own roofline;
+               and the patch embedding on the c5 bf16 rows (tensor roofline,
+               cuBLAS on the same operands beside it).
 
 --impl reference times the CPU oracle alone (rank 0; other ranks exit).
 """
@@ -73,7 +75,8 @@ def parse():
                     help="every rank takes the same batch and runs its own merge-unit window of it "
                          "(mimo_preprocess_units): strong scaling of one batch, images split across ranks")
     ap.add_argument("--no-also", action="store_true",
-                    help="c5 default line: skip the c3 fp32 and c5 bf16 measurements added under 'also'")
+                    help="c5 default line: skip the c3 fp32, c5 bf16 and patch-embedding measurements added "
+                         "under 'also'")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step from a CUDA graph (the launch without the host-side call overhead)")
     return ap.parse_args()
@@ -628,6 +631,67 @@ def also_config(args, mimo, workloads, name: str, out_dtype: str, dev, stream, s
             "gpu_launches": args.steps * launches, "clocks": clocks.summary()}
 
 
+def also_patch_embed(args, mimo, w, dev, stream, scratch) -> dict:
+    """The patch embedding on the bf16 rows of the same c5 batch `w`, timed like the main line (W warm-up
+    launches, then K launches between CUDA events), with cuBLAS on the same operands in the same process
+    for context. The rows and the embeddings live in `scratch` (the main line's output buffer)."""
+    import torch
+
+    params = mimo.make_params(w["mean"], w["std"])
+    host = mimo.pack_images(w["images"], device="cpu", pin_memory=True)
+    packed = host.to(dev)
+    _, offs = mimo.plan_batch(host.heights, host.widths, params)
+    M, K, N = int(offs[-1]), 1536, args.embed_dim
+    flat = scratch.view(torch.uint8).view(-1)
+    assert (M * K + M * N) * 2 <= flat.numel(), "scratch too small"
+    rows = flat[:M * K * 2].view(torch.bfloat16).view(M, K)
+    out = flat[M * K * 2:(M * K + M * N) * 2].view(torch.bfloat16).view(M, N)
+    mimo.preprocess_batch_ex(params, packed, rows, None, stream=stream)
+    del packed
+    g = torch.Generator(device="cpu").manual_seed(17)
+    weight = (torch.randn((N, K), generator=g) * 0.02).to(torch.bfloat16).to(dev)
+    bias = torch.randn(N, generator=g).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 0)):
+            fn()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        for _ in range(args.steps):
+            fn()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        return ev[0].elapsed_time(ev[1]) / args.steps
+
+    with ClockSampler(dev.index) as clocks:
+        ms = timed(lambda: mimo.patch_embed(rows, weight, bias, out=out, error=err, stream=stream, check=False))
+    if int(err.item()):
+        raise SystemExit(f"patch_embed reported pipeline error {int(err.item())}")
+    bias16 = bias.to(torch.bfloat16)
+    lib_ms = timed(lambda: torch.addmm(bias16, rows, weight.t(), out=out))
+    flops = 2.0 * M * N * K
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        peak, kind = float(pk["bf16_tflops"]), "measured"
+    except Exception:
+        peak, kind = 1590.0, "fallback"
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"workload": "pe", "description": f"bf16 rows of c5 ({M} x {K}) x weight [{N}, {K}] + bias -> bf16 "
+            f"[{M}, {N}]", "rows": M, "embed_dim": N, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "value": M / (ms * 1e-3), "unit": "tokens/s",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_kind": kind,
+                         "traffic": ncu_traffic("pe", "bf16", "patch_embed", M),
+                         "algorithmic_flops_per_launch": flops, "kernel": "patch_embed_kernel",
+                         "avg_launch_ms": ms},
+            "library_gemm": {"impl": "torch.addmm (cuBLAS)", "ms": lib_ms,
+                             "tflops": flops / (lib_ms * 1e-3) / 1e12},
+            "gpu_launches": args.steps, "clocks": clocks.summary()}
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -775,7 +839,8 @@ def run_ours(args, rank, world, local_rank):
             and not args.shard):
         del packed
         also = {"c5_bf16": also_config(args, mimo, workloads, "c5", "bf16", dev, stream, out),
-                "c3_f32": also_config(args, mimo, workloads, "c3", "f32", dev, stream, out)}
+                "c3_f32": also_config(args, mimo, workloads, "c3", "f32", dev, stream, out),
+                "pe_bf16": also_patch_embed(args, mimo, w, dev, stream, out)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
