@@ -249,15 +249,22 @@ def cpu_baseline(w, sample_images: int, threads: int, min_seconds: float = 0.0):
             return done / dt, dt
 
 
-def dominant_kernel(grid, heights, widths, out_dtype: str) -> str:
-    """The pixel kernel an image launch runs, by the library's dispatch rule: the unstaged
-    direct_kernel when every width is kept and either the rows are bf16 or every height is kept too,
-    else the staged preprocess_kernel."""
+def dominant_kernel(grid, heights, widths, out_dtype: str, video: bool = False) -> str:
+    """The pixel kernel a launch runs, by the library's dispatch rule: for images, the warp-staged
+    warp_kernel when every height shrinks by 1.25 or more and no axis gathers its taps (a shrink of
+    about 1.94 or more gathers); else the unstaged direct_kernel when every width is kept and either
+    the rows are bf16 or every height is kept too; else the staged preprocess_kernel."""
     import numpy as np
 
     grid = np.asarray(grid)
-    widths_kept = bool(np.all(grid[:, 2] * 16 == np.asarray(widths)))
-    heights_kept = bool(np.all(grid[:, 1] * 16 == np.asarray(heights)))
+    h, w = np.asarray(heights, dtype=np.int64), np.asarray(widths, dtype=np.int64)
+    hr, wr = grid[:, 1].astype(np.int64) * 16, grid[:, 2].astype(np.int64) * 16
+    shrunk = bool(np.all(4 * h >= 5 * hr))
+    gather = bool(np.any(32 * h > 62 * hr) or np.any(32 * w > 62 * wr))
+    if shrunk and not gather and not video:
+        return "warp_kernel"
+    widths_kept = bool(np.all(wr == w))
+    heights_kept = bool(np.all(hr == h))
     return "direct_kernel" if widths_kept and (out_dtype == "bf16" or heights_kept) else "preprocess_kernel"
 
 
@@ -414,7 +421,7 @@ def run_video(args, rank, world, local_rank):
                        "l2": l2_note(read, written)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_kind": peak_kind, "traffic": None, "algorithmic_bytes_per_launch": read + written,
-                         "kernel": dominant_kernel([grid], [H], [W], out_dtype), "avg_launch_ms": ms / K},
+                         "kernel": dominant_kernel([grid], [H], [W], out_dtype, video=True), "avg_launch_ms": ms / K},
             "gpu_launches": K, "clocks": clocks.summary(), "e2e": None, "cpu_baseline": None,
         }), flush=True)
 

@@ -100,7 +100,8 @@ def test_dominant_kernel_follows_the_dispatch_rule():
     assert kernel("c5", "f32") == "preprocess_kernel"   # 1080 -> 1088 rows: heights resized
     assert kernel("c5", "bf16") == "direct_kernel"      # widths kept, bf16 rows
     assert kernel("c2", "f32") == "direct_kernel"       # identity resize
-    assert kernel("c3", "f32") == "preprocess_kernel"   # widths resized
+    assert kernel("c3", "f32") == "preprocess_kernel"   # widths resized, heights within 1.25 of kept
+    assert kernel("c4", "f32") == "warp_kernel"         # 4096 -> 2880: every height shrunk by 1.42
 
 
 def test_reference_arm_config_equals_the_main_arm_config():

@@ -13,6 +13,7 @@ import pytest
 import torch
 
 import workloads
+from _shrunk import shrunk_batch
 from vision_lm_image_b200 import build, mimo
 
 pytestmark = pytest.mark.gpu
@@ -24,18 +25,18 @@ def checked():
     return build.build_checked()
 
 
-def _all_outputs(images, mean, std, dtype, order="merge"):
+def _all_outputs(images, mean, std, dtype, order="merge", **kw):
     pv, grid, perm, pos, win = mimo.preprocess(images, mean, std, dtype=dtype, column_perm=True, order=order,
-                                               positions=True, window_index=True)
+                                               positions=True, window_index=True, **kw)
     torch.cuda.synchronize()
     return pv, perm, pos, win
 
 
-def _compare(images, mean, std, dtype, checked, order="merge"):
-    ref = _all_outputs(images, mean, std, dtype, order)
+def _compare(images, mean, std, dtype, checked, order="merge", **kw):
+    ref = _all_outputs(images, mean, std, dtype, order, **kw)
     with mimo.use_library(checked):
         assert mimo.bounds_check_status() == (0, 0)  # a fresh query starts clean
-        got = _all_outputs(images, mean, std, dtype, order)
+        got = _all_outputs(images, mean, std, dtype, order, **kw)
         status = mimo.bounds_check_status()
     assert status == (0, 0), f"{status[0]} failed bounds checks, first of kind {status[1]}"
     for a, b in zip(ref, got):
@@ -72,18 +73,35 @@ def test_kept_width_and_strong_downscale_pass_every_check(checked, dtype):
     assert torch.equal(ref[0], got[0]) and torch.equal(ref[2], got[2])
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_shrunk_batches_pass_every_check(checked, dtype):
+    # every height shrunk by 1.25 to 1.9 (warp-staged kernel), RGB and RGBA, both row orders
+    imgs = shrunk_batch(1340, 8, 40_000)
+    for order in ("merge", "column"):
+        _compare(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD, dtype, checked, order=order,
+                 max_pixels=40_000)
+
+
 @pytest.mark.parametrize("kept", [False, True])
 def test_image_ending_at_the_buffer_end_passes_every_check(checked, kept):
     # the last image's final byte is the last byte of the source buffer: staged copies of 16-byte chunks
-    # and 12/16-byte quads must stop there
+    # and 12/16-byte quads must stop there (kept: the unstaged kernel; else the staged kernel, then the
+    # same batch shrunk by max_pixels for the warp-staged kernel)
     rng = workloads.rng_for(1320)
     shape = (64, 96) if kept else (61, 95)
     imgs = [workloads.uniform_image(rng, 40, 50, 3), workloads.uniform_image(rng, *shape, 3)]
+    _buffer_end_case(imgs, shape, mimo.make_params(), checked)
+    if not kept:
+        big = (411, 397)
+        imgs = [workloads.uniform_image(rng, 300, 350, 3), workloads.uniform_image(rng, *big, 3)]
+        _buffer_end_case(imgs, big, mimo.make_params(max_pixels=60_000), checked)
+
+
+def _buffer_end_case(imgs, shape, params, checked):
     host = mimo.pack_images(imgs, device="cpu")
     end = int(host.offsets[-1]) + shape[0] * shape[1] * 3
     packed = mimo.pack_images(imgs, device="cuda")
     packed.buffer = packed.buffer[:end]  # no padding after the last image
-    params = mimo.make_params()
     _, offs = mimo.plan_batch(host.heights, host.widths, params)
     total = int(offs[-1])
     outs = []

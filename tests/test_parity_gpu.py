@@ -15,6 +15,7 @@ import torch
 
 import oracle
 import workloads
+from _shrunk import shrunk_batch
 from vision_lm_image_b200 import build, mimo
 
 pytestmark = pytest.mark.gpu
@@ -181,6 +182,55 @@ def test_gathered_taps_strong_downscale():
     imgs = [workloads.uniform_image(rng, 2000, 2000, 3), workloads.rgba_image(rng, 1500, 3000),
             workloads.uniform_image(rng, 3000, 700, 3)]
     check_against_oracle(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD, max_pixels=200_000)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_shrunk_batch_warp_staged_matches_oracle(dtype):
+    # every row, the permutation and the index tables, in both row orders, against the oracle
+    imgs = shrunk_batch(71, 9, 40_000)
+    mean, std = workloads.IMAGENET_MEAN, workloads.IMAGENET_STD
+    for order in ("merge", "column"):
+        pv, grid, perm, pos, win = mimo.preprocess(imgs, mean, std, dtype=dtype, column_perm=True, order=order,
+                                                   positions=True, window_index=True, max_pixels=40_000)
+        torch.cuda.synchronize()
+        ref, rgrid, rperm, rpos, rwin = oracle.preprocess(imgs, mean, std, column_perm=True, order=order,
+                                                          positions=True, window=True, threads=8,
+                                                          max_pixels=40_000)
+        assert np.array_equal(grid.numpy(), rgrid)
+        assert np.array_equal(perm.cpu().numpy(), rperm)
+        assert np.array_equal(pos.cpu().numpy(), rpos)
+        assert np.array_equal(win.cpu().numpy(), rwin)
+        if dtype == torch.float32:
+            assert_fp32_close(pv.cpu().numpy(), ref, order)
+        else:
+            assert_bf16_close(pv, ref, order)
+
+
+@pytest.mark.parametrize("c", [3, 4])
+def test_shrunk_image_ending_at_the_buffer_end(c):
+    # a shrunk image (warp-staged kernel) whose last row ends exactly at the end of the declared buffer:
+    # its 16-byte staging copies are cut there (zero-filled) and nothing past it is read
+    h, w, mp = 411, 397, 60_000
+    hr, wr = oracle.smart_resize(h, w, max_pixels=mp)
+    assert 4 * h >= 5 * hr and 10 * h <= 19 * hr and 10 * w <= 19 * wr
+    rng = workloads.rng_for(912)
+    img = workloads.rgba_image(rng, h, w) if c == 4 else workloads.uniform_image(rng, h, w, 3)
+    nbytes = h * w * c
+    dev_buf = torch.zeros(nbytes + 4096, dtype=torch.uint8, device="cuda")
+    dev_buf[:nbytes] = torch.from_numpy(img.reshape(-1)).cuda()
+    dev_buf[nbytes:] = 255  # bytes beyond the declared end: never used
+    params = mimo.make_params(max_pixels=mp)
+    rows = (hr // 16) * (wr // 16)
+    out = torch.empty((rows, 1536), dtype=torch.float32, device="cuda")
+    offs = np.zeros(1, np.int64)
+    hh, ww, cc = (np.array([v], np.int32) for v in (h, w, c))
+    st = mimo.lib().mimo_preprocess_batch(ctypes.byref(params), 1, ctypes.c_void_p(dev_buf.data_ptr()), nbytes,
+                                          offs.ctypes.data, hh.ctypes.data, ww.ctypes.data, cc.ctypes.data, 0,
+                                          ctypes.c_void_p(out.data_ptr()), rows, None, None)
+    assert st == 0
+    torch.cuda.synchronize()
+    ref, _ = oracle.preprocess_image(img, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD, max_pixels=mp)
+    assert_fp32_close(out.cpu().numpy(), ref, "buffer end")
 
 
 def test_extreme_shapes():
@@ -654,7 +704,7 @@ def _full_and_windows(images, mean, std, dtype, windows):
 
 @pytest.mark.parametrize("split", ["halves", "ragged"])
 def test_unit_windows_reproduce_one_large_image(split):
-    # c4: one 4096x4096 image (8100 merge units) cut by merge-block ranges, staged kernel
+    # c4: one 4096x4096 image (8100 merge units) cut by merge-block ranges, warp-staged kernel
     w = workloads.workload("c4")
     windows = [(0, 4050), (4050, 4050)] if split == "halves" else [(0, 1), (1, 89), (90, 3911), (4001, 4099)]
     (ref, rperm, rpos, rwin), (got, perm, pos, win), total = _full_and_windows(

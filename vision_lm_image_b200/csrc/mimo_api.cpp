@@ -289,6 +289,7 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
         fold_normalisation(p, &lp);
         int64_t blocks = 0;
         int32_t tr = 1, tc = 1, k = 0;
+        int64_t wr = 1, wc = 1;  // warp-staged kernel: source rows per warp, source columns per block
         while (i < last && k < mimo::kMaxImagesPerLaunch && blocks + (hi_i - lo_i) <= static_cast<int64_t>(INT32_MAX)) {
             const ImagePlan &ip = v.plan.img[i];
             mimo::ImageDesc &d = lp.img[k];
@@ -307,6 +308,10 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
             lp.block_start[k] = static_cast<int32_t>(blocks);
             blocks += hi_i - lo_i;
             tr = std::max(tr, ip.tile_rows);
+            // the taps of 4 consecutive output rows span at most floor(3 H / Hr) + 3 source rows,
+            // those of 32 consecutive columns at most floor(31 W / Wr) + 3 source columns
+            wr = std::max<int64_t>(wr, 3 * static_cast<int64_t>(heights[i]) / ip.Hr + 3);
+            wc = std::max<int64_t>(wc, 31 * static_cast<int64_t>(widths[i]) / ip.Wr + 3);
             tc = std::max(tc, ip.tile_cols);
             ++k;
             // the next image with units in the window; only the window's first image starts inside
@@ -328,6 +333,10 @@ int launch_range(const mimo_params *p, const Validated &v, int32_t first, int32_
         const size_t raw_floats = static_cast<size_t>(tr) * static_cast<size_t>(lp.raw_stride) / 4u;
         lp.raw = static_cast<int32_t>(tile_floats);  // tile | raw staging rows
         const size_t smem = sizeof(float) * (tile_floats + raw_floats);
+        // warp-staged kernel (launches that gather no axis): a row segment of up to 4 * wc bytes at any
+        // 16-byte misalignment, plus the word a 12-byte RGB read may touch past it
+        lp.warp_rows = static_cast<int32_t>(std::min<int64_t>(wr, INT32_MAX));
+        lp.warp_stride = static_cast<int32_t>(((32 + 4 * std::min<int64_t>(wc, 1 << 20)) + 15) & ~int64_t(15));
 #if defined(MIMO_BOUNDS_CHECK)
         // rows this call may emit (kernel numbering: batch row - row_base), inside the window
         lp.chk_row_lo = std::max<int64_t>(v.plan.row0[first], 4 * win.lo) - row_base;

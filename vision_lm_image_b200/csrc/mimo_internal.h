@@ -86,7 +86,8 @@ struct LaunchParamsT {
     int32_t raw;         // float offset of the raw staging rows
     int32_t raw_stride;  // bytes per raw staging row (multiple of 16)
     int32_t keep_rows;   // bf16 rows read again right away (chained patch embedding): stored with L2 evict-last
-    int32_t pad1;
+    int32_t warp_rows;   // warp-staged kernel: source rows a warp stages per block (max over images)
+    int32_t warp_stride; // warp-staged kernel: bytes per staged row (multiple of 16)
 #if defined(MIMO_BOUNDS_CHECK)
     int64_t chk_row_lo, chk_row_hi;  // rows the kernel may emit (its own row numbering)
     int64_t chk_table_rows;          // rows the permutation covers (window index: a quarter)

@@ -23,7 +23,9 @@
 // The staged kernel is instantiated with and without the fused RGB step; a
 // launch takes the fused one only when one of its images needs it. Launches
 // whose images or frames all keep their width go to a second, unstaged kernel
-// (direct_kernel below) when that measured faster.
+// (direct_kernel below) when that measured faster, and launches that shrink
+// every image's height by 1.25 or more to a third, warp-staged one
+// (warp_kernel below).
 // There is no inter-CTA communication, no atomics and no global wait; every
 // output element has exactly one writer.
 #include <cuda_bf16.h>
@@ -971,6 +973,296 @@ __global__ void __launch_bounds__(kThreads, kVideoLaunch ? 5 : 6) direct_kernel(
     }
 }
 
+// ---------------------------------------------------------------------------
+// Warp-staged kernel, for image launches whose images stage both axes' spans
+// whole (no gathered axis). Each warp owns the same 4 consecutive output rows
+// x 32 columns of every block (the direct kernel's mapping) and stages only the
+// source rows those 4 rows need, into its own two-slot slice of shared memory,
+// one block ahead with cp.async: nothing waits on more than the warp. A lane
+// reads each of its output columns' two taps straight from the staged bytes
+// (as the fused RGB step does; RGBA is composited onto white first),
+// interpolates along W in its two source rows, then along H, normalises and
+// stores as the other kernels do, with the same arithmetic: the outputs are
+// bit-identical to the staged kernel's. The taps come from the exact quotient:
+// lane l holds the taps of output column l (advanced by 32 columns from block
+// to block) and of output row l of the block row, one block ahead, and the
+// lanes exchange them with shuffles.
+// ---------------------------------------------------------------------------
+
+// Exact tap of output index d along an axis in -> out (den = 2 out), as
+// compute_taps forms it: the floor quotient q and remainder r of
+// ((2d+1) in - out) / den.
+__device__ __forceinline__ void exact_quotient(int64_t d, int32_t in, int32_t out, double inv_den, int32_t &q,
+                                               int32_t &r) {
+    const int64_t den = 2 * static_cast<int64_t>(out);
+    const int64_t num = (2 * d + 1) * in - out;
+    int64_t qq = static_cast<int64_t>(floor(static_cast<double>(num) * inv_den));
+    int64_t rr = num - qq * den;
+    while (rr < 0) {
+        --qq;
+        rr += den;
+    }
+    while (rr >= den) {
+        ++qq;
+        rr -= den;
+    }
+    q = static_cast<int32_t>(qq);
+    r = static_cast<int32_t>(rr);
+}
+
+// First tap and weight of the second from (q, r): clamped at 0 from below.
+__device__ __forceinline__ void tap_of(int32_t q, int32_t r, float inv_den_f, int32_t &i0, float &lam) {
+    const bool clamp = q < 0;
+    i0 = clamp ? 0 : q;
+    const float rf = (r < (1 << 23)) ? __uint_as_float(0x4B000000u | static_cast<uint32_t>(r)) - kTwo23
+                                     : static_cast<float>(r);
+    lam = clamp ? 0.0f : rf * inv_den_f;
+}
+
+// One block as a warp sees it: its position, the lane's column and row taps
+// (lane l: output column l, output row l of the block) and where the warp's
+// staged rows start.
+struct WarpBlock {
+    int ii, bh, bw;
+    int32_t ci0, ri0;  // first source column of output column `lane`, first source row of output row `lane`
+    float cl, rl;      // their second-tap weights
+    int32_t r_lo, c_lo;  // first staged source row (this warp) and first staged source column (the block)
+};
+
+template <bool kBF16, class Params>
+__global__ void __launch_bounds__(kThreads, 4) warp_kernel(const __grid_constant__ Params P) {
+    extern __shared__ float4 smem4[];
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int64_t B = P.block_start[P.n];
+    const int begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * B / gridDim.x);
+    const int end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * B / gridDim.x);
+    if (begin >= end) return;
+
+    // this thread's place in every block (the direct kernel's mapping)
+    const int mh = warp >> 2;
+    const int py = ((warp & 3) << 2) | (lane >> 3);
+    const int mw = (lane >> 2) & 1;
+    const int q = lane & 3;
+    const int dy = (mh << 4) | py;
+    const int dx0 = (mw << 4) | (q << 2);
+    const int col = py * 16 + q * 4;
+    const int dy_first = (mh << 4) | ((warp & 3) << 2);  // the warp's first output row in a block
+    const int wstride = P.warp_stride;
+    const int slot_bytes = P.warp_rows * wstride;
+    uint8_t *const wbuf = reinterpret_cast<uint8_t *>(smem4) + static_cast<size_t>(warp) * 2 * slot_bytes;
+
+    // axis constants of the image the cursors are for
+    int cur_img = -1;
+    int32_t den_x = 1, step_q = 0, step_r = 0, CQ = 1;
+    uint32_t cmagic = 1;
+    double inv_x = 1.0, inv_y = 1.0;
+    float inv_xf = 1.0f, inv_yf = 1.0f;
+    // column cursor of output column bw * 32 + lane, row taps of output row bh * 32 + lane
+    int32_t cq = 0, cr = 0, rq = 0, rr = 0;
+    int row_img = -1, row_bh = -1, col_img = -1, col_bh = -1, col_bw = -2;
+
+    // the taps of block (ii, bh, bw) into wb, and its staging into slot `slot`
+    auto prepare = [&](int ii, int bh, int bw, int slot, WarpBlock &wb) {
+        const ImageDesc &D = P.img[ii];
+        const int32_t H = D.H, W = D.W, Hr = D.Hr, Wr = D.Wr;
+        const int C = (D.flags >> kChannelShift) & 0xFF;
+        if (ii != cur_img) {
+            cur_img = ii;
+            den_x = 2 * Wr;
+            inv_x = 1.0 / static_cast<double>(den_x);
+            inv_xf = static_cast<float>(inv_x);
+            inv_y = 1.0 / (2.0 * static_cast<double>(Hr));
+            inv_yf = static_cast<float>(inv_y);
+            const int64_t step = 2 * static_cast<int64_t>(kBlock) * W;  // numerator change from block to block
+            step_q = static_cast<int32_t>(step / den_x);
+            step_r = static_cast<int32_t>(step - static_cast<int64_t>(step_q) * den_x);
+            // 16-byte chunks covering a staged row segment of the image at any offset
+            CQ = (30 + C * (31 * static_cast<int64_t>(W) / Wr + 3)) >> 4;
+            cmagic = (65536u + CQ - 1) / CQ;  // job / CQ as (job * cmagic) >> 16, exact for job < 64 * 18
+        }
+        if (ii == col_img && bh == col_bh && bw == col_bw + 1) {
+            cq += step_q;
+            cr += step_r;
+            if (cr >= den_x) {
+                cr -= den_x;
+                ++cq;
+            }
+        } else {
+            exact_quotient(static_cast<int64_t>(bw) * kBlock + lane, W, Wr, inv_x, cq, cr);
+        }
+        col_img = ii;
+        col_bh = bh;
+        col_bw = bw;
+        if (ii != row_img || bh != row_bh) {
+            exact_quotient(static_cast<int64_t>(bh) * kBlock + lane, H, Hr, inv_y, rq, rr);
+            row_img = ii;
+            row_bh = bh;
+        }
+        wb.ii = ii;
+        wb.bh = bh;
+        wb.bw = bw;
+        tap_of(cq, cr, inv_xf, wb.ci0, wb.cl);
+        tap_of(rq, rr, inv_yf, wb.ri0, wb.rl);
+        // the warp's source rows and the block's source columns
+        const int32_t r_lo = __shfl_sync(0xffffffffu, wb.ri0, dy_first);
+        const int32_t r_hi = min(__shfl_sync(0xffffffffu, wb.ri0, dy_first + 3) + 1, H - 1);
+        const int32_t c_lo = __shfl_sync(0xffffffffu, wb.ci0, 0);
+        const int32_t c_hi = min(__shfl_sync(0xffffffffu, wb.ci0, 31) + 1, W - 1);
+        wb.r_lo = r_lo;
+        wb.c_lo = c_lo;
+        const int nr = r_hi - r_lo + 1;
+        const int L = C * (c_hi - c_lo + 1);
+        const uint8_t *img = P.src + D.src_off;
+        uint8_t *dst = wbuf + slot * slot_bytes;
+        for (int job = lane; job < nr * CQ; job += 32) {
+            const int j = static_cast<int>((static_cast<uint32_t>(job) * cmagic) >> 16);
+            const int c = job - j * CQ;
+            const int64_t rs = (static_cast<int64_t>(r_lo + j) * W + c_lo) * C;
+            const int64_t cs = (rs & ~int64_t(15)) + 16 * c;
+            if (cs < rs + L) {
+                const int64_t left = D.limit - cs;
+                const int nb = left < 16 ? static_cast<int>(left) : 16;
+                if (MIMO_CHECK(cs >= 0 && nb > 0 && cs + nb <= D.limit, kChkSrcCopy) &&
+                    MIMO_CHECK(j < P.warp_rows && 16 * c + 16 <= wstride, kChkSmem))
+                    cp_async16(dst + j * wstride + 16 * c, img + cs, nb);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
+    // position of the first block; later blocks advance one column, then one block row, then one image
+    int ii = find_image(P, begin);
+    int bh, bw;
+    {
+        const ImageDesc &D = P.img[ii];
+        const int g = D.Wr / kBlock;
+        const int local = begin - P.block_start[ii] + (ii == 0 ? P.unit0 : 0);
+        bh = local / g;
+        bw = local - bh * g;
+    }
+    WarpBlock cur, nxt;
+    prepare(ii, bh, bw, 0, cur);
+    const float2 m23 = f2(-kTwo23, -kTwo23), neg1 = f2(-1.0f, -1.0f);
+    for (int blk = begin; blk < end; ++blk) {
+        const int slot = (blk - begin) & 1;
+        const bool more = blk + 1 < end;
+        if (more) {
+            const ImageDesc &D = P.img[ii];
+            if (++bw == D.Wr / kBlock) {
+                bw = 0;
+                if (++bh == D.Hr / kBlock) {
+                    bh = 0;
+                    ++ii;
+                }
+            }
+            prepare(ii, bh, bw, slot ^ 1, nxt);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncwarp();  // every lane's copies of this block have landed
+
+        const ImageDesc &D = P.img[cur.ii];
+        const int32_t H = D.H, W = D.W, Hr = D.Hr, Wr = D.Wr;
+        const int C = (D.flags >> kChannelShift) & 0xFF;
+        const uint8_t *base = wbuf + slot * slot_bytes;
+        // this lane's output row and columns
+        const int32_t sy0 = __shfl_sync(0xffffffffu, cur.ri0, dy);
+        const float ly = __shfl_sync(0xffffffffu, cur.rl, dy);
+        const int32_t sy1 = min(sy0 + 1, H - 1);
+        int32_t sx[4];
+        float lx[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            sx[i] = __shfl_sync(0xffffffffu, cur.ci0, dx0 + i);
+            lx[i] = __shfl_sync(0xffffffffu, cur.cl, dx0 + i);
+        }
+        const float2 l01 = f2(lx[0], lx[1]), l23 = f2(lx[2], lx[3]);
+        // the quad's values of one staged source row, interpolated along W: h[c] = columns (0,1), (2,3)
+        float2 h[2][3][2];
+#pragma unroll
+        for (int rsel = 0; rsel < 2; ++rsel) {
+            const int32_t sy = rsel ? sy1 : sy0;
+            const int j = sy - cur.r_lo;
+            // byte offset of source column c_lo in the staged row (its 16-byte misalignment)
+            const uint32_t mis = ((static_cast<uint32_t>(sy) * static_cast<uint32_t>(W) + static_cast<uint32_t>(cur.c_lo)) *
+                                  static_cast<uint32_t>(C)) & 15u;
+            const uint8_t *row = base + j * wstride;
+            uint32_t a[4], b[4];
+            bool ok = MIMO_CHECK(j >= 0 && j < P.warp_rows, kChkSmem);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const bool next = sx[i] + 1 < W;  // the second tap is the next pixel, or the pixel itself at the edge
+                const uint32_t o = mis + static_cast<uint32_t>(C * (sx[i] - cur.c_lo));
+                // RGBA reads two aligned words from o, RGB three from o rounded down to a word
+                ok = ok && MIMO_CHECK(sx[i] >= cur.c_lo && (C == 4 ? o + 8u : (o & ~3u) + 12u) <= static_cast<uint32_t>(wstride),
+                                      kChkSmem);
+                if (C == 4) {
+                    const uint32_t *w = reinterpret_cast<const uint32_t *>(row + o);
+                    a[i] = ok ? w[0] : 0u;
+                    b[i] = ok ? (next ? w[1] : a[i]) : 0u;
+                } else if (ok) {
+                    rgb_pair(row, o, next, a[i], b[i]);
+                } else {
+                    a[i] = b[i] = 0u;
+                }
+            }
+            if (C == 4) {
+                // composite both taps onto white (as the conversion does), then fma(lx, b - a, a)
+                const float2 Aa01 = add2(f2(byte_bits<3>(a[0]), byte_bits<3>(a[1])), m23);
+                const float2 Aa23 = add2(f2(byte_bits<3>(a[2]), byte_bits<3>(a[3])), m23);
+                const float2 Ab01 = add2(f2(byte_bits<3>(b[0]), byte_bits<3>(b[1])), m23);
+                const float2 Ab23 = add2(f2(byte_bits<3>(b[2]), byte_bits<3>(b[3])), m23);
+                const float2 wa01 = fma2(Aa01, f2(-255.0f, -255.0f), f2(65025.0f, 65025.0f));
+                const float2 wa23 = fma2(Aa23, f2(-255.0f, -255.0f), f2(65025.0f, 65025.0f));
+                const float2 wb01 = fma2(Ab01, f2(-255.0f, -255.0f), f2(65025.0f, 65025.0f));
+                const float2 wb23 = fma2(Ab23, f2(-255.0f, -255.0f), f2(65025.0f, 65025.0f));
+#define MIMO_WARP_RGBA(c)                                                                                       \
+    {                                                                                                           \
+        const float2 A01 = on_white2(add2(f2(byte_bits<c>(a[0]), byte_bits<c>(a[1])), m23), Aa01, wa01);        \
+        const float2 A23 = on_white2(add2(f2(byte_bits<c>(a[2]), byte_bits<c>(a[3])), m23), Aa23, wa23);        \
+        const float2 B01 = on_white2(add2(f2(byte_bits<c>(b[0]), byte_bits<c>(b[1])), m23), Ab01, wb01);        \
+        const float2 B23 = on_white2(add2(f2(byte_bits<c>(b[2]), byte_bits<c>(b[3])), m23), Ab23, wb23);        \
+        h[rsel][c][0] = fma2(l01, fma2(A01, neg1, B01), A01);                                                   \
+        h[rsel][c][1] = fma2(l23, fma2(A23, neg1, B23), A23);                                                   \
+    }
+                MIMO_WARP_RGBA(0)
+                MIMO_WARP_RGBA(1)
+                MIMO_WARP_RGBA(2)
+#undef MIMO_WARP_RGBA
+            } else {
+#define MIMO_WARP_RGB(c)                                                                                        \
+    {                                                                                                           \
+        const float2 A01 = f2(byte_bits<c>(a[0]), byte_bits<c>(a[1]));                                          \
+        const float2 A23 = f2(byte_bits<c>(a[2]), byte_bits<c>(a[3]));                                          \
+        h[rsel][c][0] = fma2(l01, fma2(A01, neg1, f2(byte_bits<c>(b[0]), byte_bits<c>(b[1]))), add2(A01, m23)); \
+        h[rsel][c][1] = fma2(l23, fma2(A23, neg1, f2(byte_bits<c>(b[2]), byte_bits<c>(b[3]))), add2(A23, m23)); \
+    }
+                MIMO_WARP_RGB(0)
+                MIMO_WARP_RGB(1)
+                MIMO_WARP_RGB(2)
+#undef MIMO_WARP_RGB
+            }
+        }
+        __syncwarp();  // the slot is read: the next block's copies may reuse it
+
+        // merge order lists units by (block row, block col), column order by (block col, block row)
+        const int gw2 = Wr / kBlock, gh2 = Hr / kBlock;
+        const int64_t unit = P.order ? static_cast<int64_t>(cur.bw) * gh2 + cur.bh : static_cast<int64_t>(cur.bh) * gw2 + cur.bw;
+        const int64_t orow = D.row0 + 4 * unit + (mh * 2 + mw);
+        const float2 ly2 = f2(ly, ly), nly2 = f2(-ly, -ly);
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+            const float2 v01 = fma2(ly2, h[1][c][0], fma2(nly2, h[0][c][0], h[0][c][0]));
+            const float2 v23 = fma2(ly2, h[1][c][1], fma2(nly2, h[0][c][1], h[0][c][1]));
+            store_quad<kBF16>(P, orow, c, col, 0, true, v01, v23);
+        }
+        if (tid < 3) write_unit_tables(P, tid, D.row0, 0, cur.bh, cur.bw, gh2, gw2, D.row0 + 4 * unit);
+        cur = nxt;
+    }
+}
+
 // Launch setup that depends only on the device and the shared-memory size,
 // kept per host thread so that small batches do not pay the driver queries on
 // every call.
@@ -1035,20 +1327,64 @@ int launch_direct(const Params &lp, int64_t blocks, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
 }
 
-// Both kernels for one parameter block type, chosen as measured: the direct
-// kernel when every width is kept, unless fp32 rows are written for resized
-// heights (there the staged kernel's burst reads keep the write stream faster).
+template <bool kBF16, class Params>
+int launch_warp(const Params &lp, int64_t blocks, cudaStream_t stream) {
+    auto kern = warp_kernel<kBF16, Params>;
+    static thread_local LaunchSetup setup;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MIMO_ECUDA;
+    if (dev != setup.dev) {
+        setup = LaunchSetup();
+        if (cudaDeviceGetAttribute(&setup.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MIMO_ECUDA;
+        setup.dev = dev;
+    }
+    // 8 warps x 2 slots x staged rows x row stride
+    const size_t smem_bytes = static_cast<size_t>(kThreads / 32) * 2u * static_cast<size_t>(lp.warp_rows) *
+                              static_cast<size_t>(lp.warp_stride);
+    if (smem_bytes > setup.attr_smem) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes)) !=
+            cudaSuccess)
+            return MIMO_ECUDA;
+        setup.attr_smem = smem_bytes;
+    }
+    if (smem_bytes != setup.occ_smem) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem_bytes) != cudaSuccess ||
+            per_sm <= 0)
+            return MIMO_ECUDA;
+        setup.per_sm = per_sm;
+        setup.occ_smem = smem_bytes;
+    }
+    const int64_t grid = std::min<int64_t>(blocks, static_cast<int64_t>(setup.sms) * setup.per_sm);
+    kern<<<static_cast<unsigned>(grid), kThreads, smem_bytes, stream>>>(lp);
+    return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ECUDA;
+}
+
+// The kernels for one parameter block type, chosen as measured:
+//  - the warp-staged kernel for image launches that shrink every image's
+//    height by 1.25 or more (and gather no axis): it recomputes both taps of
+//    each output pixel, a cost fixed per output, while the staged kernel's
+//    conversion and horizontal pass grow with the staged source rows
+//    (32 H / Hr + 2 per block); near H = Hr the staged kernel is faster;
+//  - the direct kernel when every width is kept, unless fp32 rows are written
+//    for resized heights (there the staged kernel's burst reads keep the write
+//    stream faster);
+//  - the staged kernel otherwise.
 template <class Params>
 int launch_kernels(const Params &lp, int64_t blocks, int out_dtype, size_t smem_bytes, cudaStream_t s) {
-    bool widths_kept = true, heights_kept = true, video = false, fused = false;
+    bool widths_kept = true, heights_kept = true, video = false, fused = false, gather = false, shrunk = true;
     for (int i = 0; i < lp.n; ++i) {
         const int32_t f = lp.img[i].flags;
+        gather = gather || (f & (kGatherRows | kGatherCols)) != 0;
+        shrunk = shrunk && 4 * static_cast<int64_t>(lp.img[i].H) >= 5 * static_cast<int64_t>(lp.img[i].Hr);
         widths_kept = widths_kept && (f & kIdentityCols) != 0;
         heights_kept = heights_kept && (f & kIdentityRows) != 0;
         video = video || (f & kVideo) != 0;
         // an RGB image with a resized, contiguously staged width takes the fused conversion step
         fused = fused || (((f >> kChannelShift) & 0xFF) == 3 && (f & (kIdentityCols | kGatherCols)) == 0);
     }
+    if (!video && !gather && shrunk && lp.warp_rows > 0)
+        return out_dtype == MIMO_BF16 ? launch_warp<true>(lp, blocks, s) : launch_warp<false>(lp, blocks, s);
     // a video launch carries exactly one clip
     if (widths_kept && (out_dtype == MIMO_BF16 || heights_kept) && (!video || lp.n == 1)) {
         if (video)
