@@ -22,7 +22,8 @@
  * Conventions for every entry point:
  *   - Return value: a mimo_status (0 = MIMO_OK). Every argument problem the
  *     host can see is reported before anything is launched or copied. The
- *     device code contains no traps. The pixel kernels contain no waits. The
+ *     device code contains no traps. The pixel kernels wait only for their
+ *     own CTA's or warp's copies and barriers, never on other CTAs. The
  *     patch-embedding kernel's waits are bounded and report through d_error.
  *   - Ownership: the caller owns every buffer. The library never allocates
  *     or frees device memory at run time. Between calls it keeps:
