@@ -1,12 +1,13 @@
 """The pixel kernels of the bounds-checked debug build (-DMIMO_BOUNDS_CHECK) on the parity sweeps.
 
 compute-sanitizer is not available on the GPU pool these tests run on, so the library carries its own
-check: in the debug build every global load and store of both pixel kernels, and their shared-memory tile
-indices, are checked against the extents the host validated (the image and the caller's source buffer,
-the output rows, the permutation / position / window tables). A failed check skips the access and counts
-it; it never traps. These tests run the small-batch sweeps, the kept-width (unstaged kernel) batches, an
-image ending exactly at the end of the source buffer, a video, merge-unit windows and every table
-through the debug build, and require zero failed checks and outputs bit-identical to the release build.
+check: in the debug build every global load and store of the three pixel kernels, and their shared-memory
+tile and staging indices, are checked against the extents the host validated (the image and the caller's
+source buffer, the output rows, the permutation / position / window tables). A failed check skips the
+access and counts it; it never traps. These tests run the small-batch sweeps, the kept-width (unstaged
+kernel) batches, shrunk batches (warp-staged kernel), images ending exactly at the end of the source
+buffer, a video, merge-unit windows and every table through the debug build, and require zero failed
+checks and outputs bit-identical to the release build.
 """
 import numpy as np
 import pytest
