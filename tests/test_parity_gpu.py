@@ -206,6 +206,12 @@ def test_shrunk_batch_warp_staged_matches_oracle(dtype):
             assert_bf16_close(pv, ref, order)
 
 
+def test_shrunk_batch_in_the_large_parameter_block():
+    # more than 32 images: the launch carries the 512-image parameter block (the other instantiation)
+    imgs = shrunk_batch(73, 40, 40_000, lo=250, hi=420)
+    check_against_oracle(imgs, workloads.CLIP_MEAN, workloads.CLIP_STD, max_pixels=40_000)
+
+
 @pytest.mark.parametrize("c", [3, 4])
 def test_shrunk_image_ending_at_the_buffer_end(c):
     # a shrunk image (warp-staged kernel) whose last row ends exactly at the end of the declared buffer:
