@@ -597,6 +597,22 @@ def test_preprocess_embed_equals_two_step(order, out_dtype):
                        ref.view(torch.int16 if out_dtype == torch.bfloat16 else torch.int32))
 
 
+def test_preprocess_embed_shrunk_batch_equals_two_step():
+    # images the warp-staged kernel takes, through the chained call (its bf16 rows stored L2 evict-last)
+    imgs = shrunk_batch(74, 7, 40_000)
+    mean, std = workloads.IMAGENET_MEAN, workloads.IMAGENET_STD
+    g = torch.Generator(device="cpu").manual_seed(8)
+    w = (torch.randn((512, 1536), generator=g) * 0.02).to(torch.bfloat16).cuda()
+    bias = torch.randn(512, generator=g).cuda()
+    rows, grid, _ = mimo.preprocess(imgs, mean, std, dtype=torch.bfloat16, max_pixels=40_000)
+    ref = mimo.patch_embed(rows, w, bias)
+    biggest = int((grid[:, 1] * grid[:, 2]).max())
+    emb, grid2 = mimo.preprocess_embed(imgs, w, bias, mean, std, max_pixels=40_000,
+                                       scratch_bytes=2 * (biggest + 100) * 3072)
+    assert torch.equal(grid, grid2)
+    assert torch.equal(emb.view(torch.int16), ref.view(torch.int16))
+
+
 def test_preprocess_embed_one_image_runs_equal_two_step():
     # 1080p images (8,160 rows: 160 GEMM tiles, a ragged last wave on the CTA pairs) through a scratch whose
     # halves hold exactly one image: five runs alternate over the two halves and their two library streams,
