@@ -101,7 +101,7 @@ __device__ __forceinline__ int find_image(const Params &P, int blk) {
 // Taps, staging geometry and output addresses of one merge block (double-
 // buffered in shared memory: the pipeline holds the current block and the
 // next one). Every later phase reads the block's constants from here.
-struct alignas(16) TapSet {  // 16-byte aligned: the fused RGB path reads tap quads as int4 / float4
+struct alignas(16) TapSet {  // 16-byte aligned; the fused RGB path reads tap pairs as int2 / float2
     int32_t ty[2][kBlock];   // tile row of each output row's two taps
     int32_t tx[2][kBlock];   // tile column of each output column's two taps
     float ly[kBlock];        // weight of the second row tap
@@ -134,6 +134,16 @@ struct AxisCursor {
     double inv_den = 1.0;
     float inv_den_f = 1.0f;
 };
+
+// ceil(65536 / n) for n = 1..18 (entry 0 unused): x / n = (x * entry) >> 16
+// for the job indices below (x < 64 * n), looked up instead of divided
+constexpr uint32_t ceil_65536(uint32_t n) { return (65536u + n - 1) / n; }
+__constant__ uint32_t kCeil65536[19] = {0,
+                                        ceil_65536(1),  ceil_65536(2),  ceil_65536(3),  ceil_65536(4),
+                                        ceil_65536(5),  ceil_65536(6),  ceil_65536(7),  ceil_65536(8),
+                                        ceil_65536(9),  ceil_65536(10), ceil_65536(11), ceil_65536(12),
+                                        ceil_65536(13), ceil_65536(14), ceil_65536(15), ceil_65536(16),
+                                        ceil_65536(17), ceil_65536(18)};
 
 // Warps 0 (rows) and 1 (columns): taps of block blk into T. `prev` holds the
 // taps of the block before blk in this CTA's order.
@@ -301,12 +311,13 @@ __device__ __forceinline__ void compute_taps(const Params &P, TapSet &T, const T
             if (is_col) {
                 T.x_first = gather ? 0 : first;
                 T.ncols = count;
-                const int CQ = (30 + C * count) >> 4;  // chunks covering a row segment at any 16-byte offset
-                const int Q = (count + 3) >> 2;
+                // chunks covering a row segment at any 16-byte offset: CQ <= 17 (C <= 4, count <= 64)
+                const int CQ = (30 + C * count) >> 4;
+                const int Q = (count + 3) >> 2;  // <= 16
                 T.CQ = CQ;
                 T.Q = Q;
-                T.cmagic = (65536u + CQ - 1) / CQ;  // exact for x < 64 * 18
-                T.qmagic = (65536u + Q - 1) / Q;    // exact for x < 64 * 16
+                T.cmagic = kCeil65536[CQ];  // exact for x < 64 * 18
+                T.qmagic = kCeil65536[Q];   // exact for x < 64 * 16
             } else {
                 T.y_first = gather ? 0 : first;
                 T.nrows = count;
@@ -410,48 +421,44 @@ __device__ __forceinline__ void finish_stage(const Params &P, const TapSet &T, c
     const int C = T.C;
     const float2 m23 = f2(-kTwo23, -kTwo23);
     if (fused_hpass<kFused>(T)) {
-        // job = (tile row j, output quad q): the two taps of each of the quad's 4 output columns come
-        // straight from the staged bytes, and (1 - lx) a + lx b = fma(lx, b - a, a) lands over columns
-        // 4q..4q+3 of the tile row. b - a is formed exactly from the 2^23 bit patterns, so the values
-        // equal those of converting the row and then interpolating it.
+        // job = (tile row j, output column pair q): the two taps of each of the pair's output columns
+        // come straight from the staged bytes, and (1 - lx) a + lx b = fma(lx, b - a, a) lands over
+        // columns 2q, 2q+1 of the tile row. b - a is formed exactly from the 2^23 bit patterns, so the
+        // values equal those of converting the row and then interpolating it. Pairs rather than quads:
+        // the ~34 staged rows x 16 pairs fill three rounds of warps 2-7 evenly, where quads left a
+        // second round on 80 of its 192 threads.
         const int W = T.W, y_first = T.y_first, x_first = T.x_first;
         const bool grow = (flags & kGatherRows) != 0;
-        const int jobs = nrows * 8;
-        const int t0 = (jobs <= 2 * (kThreads - 64)) ? 64 : 0;
+        const int jobs = nrows * 16;
+        const int t0 = (jobs <= 3 * (kThreads - 64)) ? 64 : 0;
         const int step = kThreads - t0;
         const float2 neg1 = f2(-1.0f, -1.0f);
         for (int job = tid - t0; job < jobs; job += step) {
             if (job < 0) break;
-            const int j = job >> 3, q = job & 7;
+            const int j = job >> 4, q = job & 15;
             const int sy = grow ? T.srow[j] : y_first + j;
             const uint32_t mis = ((static_cast<uint32_t>(sy) * static_cast<uint32_t>(W) + x_first) * 3u) & 15u;
             const uint8_t *row = raw + j * P.raw_stride;
-            const int4 ta = *reinterpret_cast<const int4 *>(&T.tx[0][4 * q]);
-            const int4 tb = *reinterpret_cast<const int4 *>(&T.tx[1][4 * q]);
-            const float4 l = *reinterpret_cast<const float4 *>(&T.lx[4 * q]);
+            const int2 ta = *reinterpret_cast<const int2 *>(&T.tx[0][2 * q]);
+            const int2 tb = *reinterpret_cast<const int2 *>(&T.tx[1][2 * q]);
+            const float2 l01 = *reinterpret_cast<const float2 *>(&T.lx[2 * q]);
             // every tap read (three words from the first tap) stays inside the staged row, every write
             // inside the tile, and the second tap is the first one or the pixel after it
-            if (!MIMO_CHECK(j < P.tile_rows && 4 * q + 4 <= TS && min(min(ta.x, ta.y), min(ta.z, ta.w)) >= 0 &&
+            if (!MIMO_CHECK(j < P.tile_rows && 2 * q + 2 <= TS && min(ta.x, ta.y) >= 0 &&
                                 static_cast<unsigned>(tb.x - ta.x) <= 1u && static_cast<unsigned>(tb.y - ta.y) <= 1u &&
-                                static_cast<unsigned>(tb.z - ta.z) <= 1u && static_cast<unsigned>(tb.w - ta.w) <= 1u &&
-                                ((mis + 3u * static_cast<uint32_t>(max(max(ta.x, ta.y), max(ta.z, ta.w)))) & ~3u) +
-                                        12u <= static_cast<uint32_t>(P.raw_stride),
+                                ((mis + 3u * static_cast<uint32_t>(max(ta.x, ta.y))) & ~3u) + 12u <=
+                                    static_cast<uint32_t>(P.raw_stride),
                             kChkSmem))
                 continue;
-            uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+            uint32_t a0, a1, b0, b1;
             rgb_pair(row, mis + 3u * ta.x, tb.x != ta.x, a0, b0);
             rgb_pair(row, mis + 3u * ta.y, tb.y != ta.y, a1, b1);
-            rgb_pair(row, mis + 3u * ta.z, tb.z != ta.z, a2, b2);
-            rgb_pair(row, mis + 3u * ta.w, tb.w != ta.w, a3, b3);
-            const float2 l01 = f2(l.x, l.y), l23 = f2(l.z, l.w);
-            float *t = tile + j * TS + 4 * q;
-#define MIMO_FUSED_CHANNEL(c)                                                                     \
-    {                                                                                             \
-        const float2 A01 = f2(byte_bits<c>(a0), byte_bits<c>(a1));                                \
-        const float2 A23 = f2(byte_bits<c>(a2), byte_bits<c>(a3));                                \
+            float *t = tile + j * TS + 2 * q;
+#define MIMO_FUSED_CHANNEL(c)                                                                                   \
+    {                                                                                                           \
+        const float2 A01 = f2(byte_bits<c>(a0), byte_bits<c>(a1));                                              \
         const float2 v01 = fma2(l01, fma2(A01, neg1, f2(byte_bits<c>(b0), byte_bits<c>(b1))), add2(A01, m23)); \
-        const float2 v23 = fma2(l23, fma2(A23, neg1, f2(byte_bits<c>(b2), byte_bits<c>(b3))), add2(A23, m23)); \
-        *reinterpret_cast<float4 *>(t + (c) * plane) = make_float4(v01.x, v01.y, v23.x, v23.y);  \
+        *reinterpret_cast<float2 *>(t + (c) * plane) = v01;                                                     \
     }
             MIMO_FUSED_CHANNEL(0)
             MIMO_FUSED_CHANNEL(1)
