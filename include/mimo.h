@@ -236,8 +236,9 @@ int mimo_preprocess_units(const mimo_params *p, int32_t n,
  * size (d_src_stage >= src_bytes; d_out_stage >= total_rows rows of
  * out_dtype; d_perm_stage >= total_rows int32 when h_column_perm is not
  * NULL), so the call allocates nothing. Host buffers should be page-locked
- * for full copy bandwidth. The batch is cut into chunks of images whose
- * upload, kernel and download overlap on two library-created streams that
+ * for full copy bandwidth. The batch is cut into chunks of whole images (a
+ * small first chunk, each later one three times larger, up to an eighth of
+ * the batch) whose upload, kernel and download overlap on two library-created streams that
  * live only for the call, ordered after the work already on the caller's
  * stream. Synchronous: returns after the last copy to h_out has completed.
  */

@@ -329,6 +329,24 @@ def test_host_buffer_entry_point_matches_device_path():
         assert torch.equal(out_h, ref.cpu()) and torch.equal(perm_h, rperm.cpu())
 
 
+def test_host_buffer_entry_point_chunks_of_several_images():
+    # 60 images of mixed sizes: the host call's chunks grow from about 1/64 of the rows to an eighth,
+    # several images each, so uploads, launches and downloads of different chunks interleave
+    imgs = workloads.random_small_batch(29, 60, max_side=400)
+    params = mimo.make_params(workloads.IMAGENET_MEAN, workloads.IMAGENET_STD)
+    ref, _, rperm = gpu_run(imgs, workloads.IMAGENET_MEAN, workloads.IMAGENET_STD, column_perm=True)
+    host = mimo.pack_images(imgs, device="cpu", pin_memory=True)
+    _, offs = mimo.plan_batch(host.heights, host.widths, params)
+    total = int(offs[-1])
+    out_h = torch.full((total, 1536), float("nan"), pin_memory=True)
+    perm_h = torch.full((total,), -1, dtype=torch.int32, pin_memory=True)
+    src_d = torch.empty_like(host.buffer, device="cuda")
+    out_d = torch.empty((total, 1536), device="cuda")
+    perm_d = torch.empty(total, dtype=torch.int32, device="cuda")
+    mimo.preprocess_batch_host(params, host, out_h, perm_h, src_d, out_d, perm_d)
+    assert torch.equal(out_h, ref.cpu()) and torch.equal(perm_h, rperm.cpu())
+
+
 def test_device_validation_errors():
     imgs = workloads.random_small_batch(16, 2, max_side=100)
     params = mimo.make_params()
