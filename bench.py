@@ -253,7 +253,8 @@ def dominant_kernel(grid, heights, widths, out_dtype: str, video: bool = False) 
     """The pixel kernel a launch runs, by the library's dispatch rule: for images, the warp-staged
     warp_kernel when every height shrinks by 1.25 or more and no axis gathers its taps (a shrink of
     about 1.94 or more gathers); else the unstaged direct_kernel when every width is kept and either
-    the rows are bf16 or every height is kept too; else the staged preprocess_kernel."""
+    the rows are bf16, or every height is kept too, or the launch is a video; else the staged
+    preprocess_kernel."""
     import numpy as np
 
     grid = np.asarray(grid)
@@ -265,7 +266,8 @@ def dominant_kernel(grid, heights, widths, out_dtype: str, video: bool = False) 
         return "warp_kernel"
     widths_kept = bool(np.all(wr == w))
     heights_kept = bool(np.all(hr == h))
-    return "direct_kernel" if widths_kept and (out_dtype == "bf16" or heights_kept) else "preprocess_kernel"
+    return ("direct_kernel" if widths_kept and (out_dtype == "bf16" or heights_kept or video)
+            else "preprocess_kernel")
 
 
 def image_cpu_baseline(w, n_img: int, cores: int, min_seconds: float = 10.0, single_seconds: float = 5.0) -> dict:

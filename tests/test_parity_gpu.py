@@ -481,11 +481,12 @@ def test_video_matches_oracle(n, shape, c):
 
 
 @pytest.mark.parametrize("dtype,shape", [(torch.bfloat16, (100, 128)), (torch.float32, (96, 128)),
-                                         (torch.bfloat16, (1080, 1920))])
+                                         (torch.float32, (100, 128)), (torch.bfloat16, (1080, 1920)),
+                                         (torch.float32, (1080, 1920))])
 @pytest.mark.parametrize("n,c", [(3, 3), (4, 4)])
 def test_video_with_kept_width_matches_oracle(dtype, shape, n, c):
-    # frames whose width is kept go to the unstaged kernel (bf16 for any height, fp32 when the
-    # height is kept too): halves pick frame 2t + tt, an odd count repeats its last frame
+    # frames whose width is kept go to the unstaged kernel, in either dtype and whether or not the
+    # height is resized: halves pick frame 2t + tt, an odd count repeats its last frame
     assert oracle.smart_resize(*shape)[1] == shape[1]
     rng = workloads.rng_for(700 + n + shape[0])
     frames = np.stack([workloads.uniform_image(rng, shape[0], shape[1], 3) if c == 3

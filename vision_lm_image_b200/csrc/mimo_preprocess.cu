@@ -1373,9 +1373,11 @@ int launch_warp(const Params &lp, int64_t blocks, cudaStream_t stream) {
 //    each output pixel, a cost fixed per output, while the staged kernel's
 //    conversion and horizontal pass grow with the staged source rows
 //    (32 H / Hr + 2 per block); near H = Hr the staged kernel is faster;
-//  - the direct kernel when every width is kept, unless fp32 rows are written
-//    for resized heights (there the staged kernel's burst reads keep the write
-//    stream faster);
+//  - the direct kernel when every width is kept, unless fp32 rows of images
+//    are written for resized heights (there the staged kernel's burst reads
+//    keep the write stream faster). A video half writes one temporal slot,
+//    half the stores per staged block, so a video takes the direct kernel in
+//    fp32 as well;
 //  - the staged kernel otherwise.
 template <class Params>
 int launch_kernels(const Params &lp, int64_t blocks, int out_dtype, size_t smem_bytes, cudaStream_t s) {
@@ -1393,7 +1395,7 @@ int launch_kernels(const Params &lp, int64_t blocks, int out_dtype, size_t smem_
     if (!video && !gather && shrunk && lp.warp_rows > 0)
         return out_dtype == MIMO_BF16 ? launch_warp<true>(lp, blocks, s) : launch_warp<false>(lp, blocks, s);
     // a video launch carries exactly one clip
-    if (widths_kept && (out_dtype == MIMO_BF16 || heights_kept) && (!video || lp.n == 1)) {
+    if (widths_kept && (out_dtype == MIMO_BF16 || heights_kept || video) && (!video || lp.n == 1)) {
         if (video)
             return out_dtype == MIMO_BF16 ? launch_direct<true, true>(lp, blocks, s)
                                           : launch_direct<false, true>(lp, blocks, s);
