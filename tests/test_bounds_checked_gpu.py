@@ -121,6 +121,21 @@ def _buffer_end_case(imgs, shape, params, checked):
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_kept_width_video_passes_every_check(checked, dtype):
+    # width 128 kept, height 100 -> 96 resized: the unstaged kernel in either dtype; each clip's last
+    # frame ends at the end of its frame buffer
+    rng = workloads.rng_for(1332)
+    for frames in (np.stack([workloads.rgba_image(rng, 100, 128) for _ in range(5)]),
+                   np.stack([workloads.uniform_image(rng, 100, 128, 3) for _ in range(4)])):
+        ref = mimo.preprocess_video(frames, dtype=dtype)
+        with mimo.use_library(checked):
+            got = mimo.preprocess_video(frames, dtype=dtype)
+            torch.cuda.synchronize()
+            assert mimo.bounds_check_status() == (0, 0)
+        assert torch.equal(ref[0], got[0])
+
+
 def test_video_and_unit_windows_pass_every_check(checked):
     rng = workloads.rng_for(1330)
     frames = np.stack([workloads.rgba_image(rng, 70, 90) for _ in range(5)])
