@@ -525,6 +525,33 @@ def test_video_budget_and_bf16_full_hd():
     assert_bf16_close(pvb, ref, "video bf16")
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_full_clip_in_the_benchmarked_launch(dtype):
+    """The 64-frame 1080p clip through the raw call and buffer layout `bench.py --workload v1` times.
+    With no video budget every temporal patch has the clip's geometry, so temporal patch t equals the
+    oracle's clip of frames 2t and 2t+1: three whole temporal patches are compared."""
+    w = workloads.video_workload("v1")
+    frames = w["frames"]
+    n, H, W, C = frames.shape
+    params = mimo.make_params(w["mean"], w["std"])
+    stride = (H * W * C + 15) // 16 * 16
+    d_frames = torch.zeros(n * stride, dtype=torch.uint8, device="cuda")
+    d_frames.view(n, stride)[:, :H * W * C].copy_(torch.from_numpy(frames.reshape(n, -1)))
+    grid, rows = mimo.plan_video(n, H, W, w["total_max_pixels"], params)
+    assert tuple(int(x) for x in grid) == (32, 68, 120) and rows == 32 * 8160
+    out = torch.empty((rows, 1536), dtype=dtype, device="cuda")
+    mimo.preprocess_video_raw(params, d_frames, n, stride, H, W, C, out, w["total_max_pixels"])
+    torch.cuda.synchronize()
+    for t in (0, 17, 31):
+        ref, g = oracle.preprocess_video(frames[2 * t:2 * t + 2], w["mean"], w["std"])
+        assert g == (1, 68, 120)
+        got = out[8160 * t:8160 * (t + 1)]
+        if dtype == torch.float32:
+            assert_fp32_close(got.cpu().numpy(), ref, f"temporal patch {t}")
+        else:
+            assert_bf16_close(got, ref, f"temporal patch {t}")
+
+
 def test_video_of_equal_frames_equals_the_image_path():
     img = workloads.random_small_batch(601, 1, max_side=300)[0]
     a, _, _ = gpu_run([img], workloads.CLIP_MEAN, workloads.CLIP_STD)
