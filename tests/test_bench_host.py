@@ -102,6 +102,14 @@ def test_dominant_kernel_follows_the_dispatch_rule():
     assert kernel("c2", "f32") == "direct_kernel"       # identity resize
     assert kernel("c3", "f32") == "preprocess_kernel"   # widths resized, heights within 1.25 of kept
     assert kernel("c4", "f32") == "warp_kernel"         # 4096 -> 2880: every height shrunk by 1.42
+    # a video clip with kept widths takes the unstaged kernel in both dtypes, resized heights or not;
+    # with resized widths, the staged one
+    import numpy as np
+
+    v_grid = np.array([[32, 68, 120]])  # 1080x1920 frames -> 1088x1920
+    for dtype in ("f32", "bf16"):
+        assert bench.dominant_kernel(v_grid, [1080], [1920], dtype, video=True) == "direct_kernel"
+        assert bench.dominant_kernel(np.array([[2, 6, 8]]), [70], [90], dtype, video=True) == "preprocess_kernel"
 
 
 def test_reference_arm_config_equals_the_main_arm_config():
