@@ -892,8 +892,9 @@ __global__ void __launch_bounds__(kThreads, kVideoLaunch ? 5 : 6) direct_kernel(
         const int64_t x = static_cast<int64_t>(bw) * kBlock + dx0;
         uint32_t wa[4] = {0u, 0u, 0u, 0u}, wb[4] = {0u, 0u, 0u, 0u};
         float4 va[3], vb[3];
-        // the quad's bytes lie inside the frame and the caller's buffer (skipped otherwise)
-        const int64_t frame_bytes = static_cast<int64_t>(H) * W * C;
+        // the quad's bytes lie inside the frame and the caller's buffer (skipped otherwise; the
+        // checks, and with them frame_bytes, exist only in the bounds-checked build)
+        [[maybe_unused]] const int64_t frame_bytes = static_cast<int64_t>(H) * W * C;
         const int64_t qa = (static_cast<int64_t>(sy0) * W + x) * C, qb = (static_cast<int64_t>(sy1) * W + x) * C;
         if (MIMO_CHECK(qa >= 0 && qa + (C == 4 ? 16 : 12) <= frame_bytes &&
                            f * D.frame_stride + qa + (C == 4 ? 16 : 12) <= D.limit,
