@@ -206,6 +206,14 @@ def test_shrunk_batch_warp_staged_matches_oracle(dtype):
             assert_bf16_close(pv, ref, order)
 
 
+def test_shrink_of_exactly_the_warp_staged_threshold():
+    # c2's RGBA images under a 200,000-pixel budget: 480x640 -> 384x512, a shrink of exactly 1.25 on both
+    # axes (4 H = 5 H', the dispatch's equality case), compositing onto white on the warp-staged kernel
+    w = workloads.workload("c2")
+    assert oracle.smart_resize(480, 640, max_pixels=200_000) == (384, 512)
+    check_against_oracle(w["images"], w["mean"], w["std"], max_pixels=200_000)
+
+
 def test_shrunk_batch_in_the_large_parameter_block():
     # more than 32 images: the launch carries the 512-image parameter block (the other instantiation)
     imgs = shrunk_batch(73, 40, 40_000, lo=250, hi=420)
