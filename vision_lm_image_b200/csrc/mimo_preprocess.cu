@@ -763,6 +763,10 @@ __global__ void __launch_bounds__(kThreads, 5) preprocess_kernel(const __grid_co
 // identically. There is no shared memory and no barrier. The row taps come
 // from the exact quotient, once per block row, and stay in registers. Each
 // row quad is one 16-byte load (RGBA) or three 4-byte loads (RGB).
+// bf16 rows take another mapping (direct_bf16x8): each half of the CTA takes
+// every other block, and a thread owns 8 consecutive pixels of one output row,
+// so each channel leaves in one 16-byte store per temporal slot instead of two
+// 8-byte ones, and the per-block work is spread over twice the pixels.
 // ---------------------------------------------------------------------------
 
 // The 4-pixel quad a thread reads from one source row. Every width on this
@@ -816,8 +820,212 @@ __device__ __forceinline__ void convert4(const uint32_t (&w)[4], int C, float4 (
     v[2] = make_float4(B0.x, B0.y, B1.x, B1.y);
 }
 
+// The direct kernel's bf16 rows: each half of the CTA (128 threads) takes
+// every other block of the CTA's range, and a thread owns 8 consecutive pixels
+// of one output row of its block, so each channel's 8 bf16 values leave in one
+// 16-byte store per temporal slot. Per pixel the arithmetic is that of the
+// fp32 path below, quad by quad, then the same round to bf16.
+template <bool kVideoLaunch, class Params>
+__device__ __forceinline__ void direct_bf16x8(const Params &P) {
+    const int tid = threadIdx.x;
+    const int grp = tid >> 7, g = tid & 127;
+    const int w4 = g >> 5, lane = tid & 31;
+    const int64_t B = P.block_start[P.n];
+    const int begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * B / gridDim.x);
+    const int end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * B / gridDim.x);
+    const int first = begin + grp;
+    if (first >= end) return;
+
+    // this thread's place in every block: warp w4 of the half covers output rows 8 (w4 & 1) .. +7 of
+    // patch row mh = w4 >> 1; for each mw, 16 lanes write 256 contiguous bytes of an output row
+    const int mh = w4 >> 1;
+    const int py = ((w4 & 1) << 3) | (lane >> 2);
+    const int mw = (lane >> 1) & 1;
+    const int q2 = lane & 1;
+    const int dy = (mh << 4) | py;
+    const int dx0 = (mw << 4) | (q2 << 3);
+    const int col = py * 16 + q2 * 8;
+
+    int ii = find_image(P, first);
+    int t, bh, bw, tt;
+    {
+        const ImageDesc &D = P.img[ii];
+        const int gq = D.Wr / kBlock;
+        int local = first - P.block_start[ii] + (ii == 0 ? P.unit0 : 0);
+        const bool vid = (D.flags & kVideo) != 0;
+        tt = vid ? (local & 1) : 0;
+        if (vid) local >>= 1;
+        const int units = (D.Hr / kBlock) * gq;
+        t = local / units;
+        local -= t * units;
+        bh = local / gq;
+        bw = local - bh * gq;
+    }
+    // one block on: the other temporal slot of a video's unit, else one column on, then the next block
+    // row, then the next temporal patch (a video) or image
+    auto advance = [&]() {
+        const ImageDesc &Dn = P.img[ii];
+        const int g_w = Dn.Wr / kBlock, g_h = Dn.Hr / kBlock;
+        if constexpr (kVideoLaunch) {
+            if (tt == 0) {
+                tt = 1;
+            } else {
+                tt = 0;
+                if (++bw == g_w) {
+                    bw = 0;
+                    if (++bh == g_h) {
+                        bh = 0;
+                        ++t;
+                    }
+                }
+            }
+        } else {
+            if (++bw == g_w) {
+                bw = 0;
+                if (++bh == g_h) {
+                    bh = 0;
+                    ++ii;
+                }
+            }
+        }
+    };
+    int tap_ii = -1, tap_bh = -1;
+    int32_t sy0 = 0, sy1 = 0;
+    float ly = 0.0f;
+    for (int blk = first; blk < end; blk += 2) {
+        const ImageDesc &D = P.img[ii];
+        const int32_t H = D.H, W = D.W, Hr = D.Hr, flags = D.flags;
+        const int C = (flags >> kChannelShift) & 0xFF;
+        const bool yident = (flags & kIdentityRows) != 0;
+        if (ii != tap_ii || bh != tap_bh) {
+            const int64_t den = 2 * static_cast<int64_t>(Hr);
+            const double inv_den = 1.0 / static_cast<double>(den);
+            const int64_t Y = static_cast<int64_t>(bh) * kBlock + dy;
+            const int64_t num = (2 * Y + 1) * H - Hr;
+            int64_t qq = static_cast<int64_t>(floor(static_cast<double>(num) * inv_den));
+            int64_t r = num - qq * den;
+            while (r < 0) {
+                --qq;
+                r += den;
+            }
+            while (r >= den) {
+                ++qq;
+                r -= den;
+            }
+            const bool clamp = qq < 0;
+            sy0 = clamp ? 0 : static_cast<int32_t>(qq);
+            sy1 = (static_cast<int64_t>(sy0) + 1 < H) ? sy0 + 1 : H - 1;
+            ly = clamp ? 0.0f : static_cast<float>(r) * static_cast<float>(inv_den);
+            tap_ii = ii;
+            tap_bh = bh;
+        }
+        const bool video = kVideoLaunch;
+        const int64_t f = video ? min(2 * t + tt, D.frames - 1) : 0;
+        const uint8_t *img = P.src + D.src_off + f * D.frame_stride;
+        [[maybe_unused]] const int64_t frame_bytes = static_cast<int64_t>(H) * W * C;
+        const float2 ly2 = f2(ly, ly), nly2 = f2(-ly, -ly);
+        uint32_t pk[3][4];  // channel c: bf16 pairs of pixels (0,1), (2,3), (4,5), (6,7)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int64_t x = static_cast<int64_t>(bw) * kBlock + dx0 + 4 * h;
+            uint32_t wa[4] = {0u, 0u, 0u, 0u}, wb[4] = {0u, 0u, 0u, 0u};
+            float4 va[3], vb[3];
+            const int64_t qa = (static_cast<int64_t>(sy0) * W + x) * C, qb = (static_cast<int64_t>(sy1) * W + x) * C;
+            if (MIMO_CHECK(qa >= 0 && qa + (C == 4 ? 16 : 12) <= frame_bytes &&
+                               f * D.frame_stride + qa + (C == 4 ? 16 : 12) <= D.limit,
+                           kChkSrcLoad))
+                load_quad(img + qa, C, wa);
+            if (!yident) {
+                if (MIMO_CHECK(qb >= 0 && qb + (C == 4 ? 16 : 12) <= frame_bytes &&
+                                   f * D.frame_stride + qb + (C == 4 ? 16 : 12) <= D.limit,
+                               kChkSrcLoad))
+                    load_quad(img + qb, C, wb);
+                convert4(wb, C, vb);
+            }
+            convert4(wa, C, va);
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+                float2 v01 = f2(va[c].x, va[c].y), v23 = f2(va[c].z, va[c].w);
+                if (!yident) {
+                    v01 = fma2(ly2, f2(vb[c].x, vb[c].y), fma2(nly2, v01, v01));
+                    v23 = fma2(ly2, f2(vb[c].z, vb[c].w), fma2(nly2, v23, v23));
+                }
+                const float2 k2 = f2(P.k[c], P.k[c]), b2 = f2(P.b[c], P.b[c]);
+                const float2 n01 = fma2(v01, k2, b2);
+                const float2 n23 = fma2(v23, k2, b2);
+                const __nv_bfloat162 lo2 = __floats2bfloat162_rn(n01.x, n01.y);
+                const __nv_bfloat162 hi2 = __floats2bfloat162_rn(n23.x, n23.y);
+                pk[c][2 * h] = *reinterpret_cast<const uint32_t *>(&lo2);
+                pk[c][2 * h + 1] = *reinterpret_cast<const uint32_t *>(&hi2);
+            }
+        }
+        const int gw2 = D.Wr / kBlock, gh2 = Hr / kBlock;
+        const int64_t t_units = static_cast<int64_t>(t) * gh2 * gw2;
+        const int64_t unit =
+            t_units + (P.order ? static_cast<int64_t>(bw) * gh2 + bh : static_cast<int64_t>(bh) * gw2 + bw);
+        const int64_t row = D.row0 + 4 * unit + (mh * 2 + mw);
+        const int slot0 = video ? 256 * tt : 0;
+        if (MIMO_CHECK(row >= P.chk_row_lo && row < P.chk_row_hi, kChkRowStore)) {
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + row * kRowWidth + c * 512 + col + slot0;
+                const uint4 u = make_uint4(pk[c][0], pk[c][1], pk[c][2], pk[c][3]);
+                if (P.keep_rows) {
+                    uint64_t pol;
+                    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+                    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(o), "r"(u.x),
+                                 "r"(u.y), "r"(u.z), "r"(u.w), "l"(pol)
+                                 : "memory");
+                    if (!video)
+                        asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(o + 256),
+                                     "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w), "l"(pol)
+                                     : "memory");
+                } else {
+                    __stcs(reinterpret_cast<uint4 *>(o), u);
+                    if (!video) __stcs(reinterpret_cast<uint4 *>(o + 256), u);
+                }
+            }
+        }
+        if (g < 3 && (!video || tt == 0)) {
+            const int64_t src_unit = t_units + static_cast<int64_t>(bh) * gw2 + bw;  // merge order
+            const int64_t dst_unit = t_units + static_cast<int64_t>(bw) * gh2 + bh;  // column order
+            if (g == 0 && P.perm != nullptr) {
+                const int32_t s0 = static_cast<int32_t>(D.row0 + 4 * src_unit);
+                if (MIMO_CHECK(D.row0 + 4 * dst_unit >= 0 && D.row0 + 4 * dst_unit + 4 <= P.chk_table_rows,
+                               kChkTableStore))
+                    __stcs(reinterpret_cast<int4 *>(P.perm + D.row0 + 4 * dst_unit),
+                           make_int4(s0, s0 + 1, s0 + 2, s0 + 3));
+            } else if (g == 1 && P.pos != nullptr) {
+                const int32_t hh = 2 * bh, ww = 2 * bw;
+                int4 *d = reinterpret_cast<int4 *>(P.pos + 2 * (D.row0 + 4 * unit));
+                if (MIMO_CHECK(D.row0 + 4 * unit >= P.chk_row_lo && D.row0 + 4 * unit + 4 <= P.chk_row_hi,
+                               kChkTableStore)) {
+                    __stcs(d, make_int4(hh, ww, hh, ww + 1));
+                    __stcs(d + 1, make_int4(hh + 1, ww, hh + 1, ww + 1));
+                }
+            } else if (g == 2 && P.win != nullptr) {
+                const int64_t u0 = D.row0 / 4;
+                if (MIMO_CHECK(u0 + dst_unit >= 0 && 4 * (u0 + dst_unit) + 4 <= P.chk_table_rows, kChkTableStore))
+                    P.win[u0 + dst_unit] = static_cast<int32_t>(u0 + src_unit);
+            }
+        }
+        if (blk + 2 < end) {
+            advance();
+            advance();
+        }
+    }
+}
+
+// bf16 rows need 64 registers for their two quads (4 CTAs per SM); fp32 rows
+// keep 48 (a video) or 40 (images).
 template <bool kBF16, bool kVideoLaunch, class Params>
-__global__ void __launch_bounds__(kThreads, kVideoLaunch ? 5 : 6) direct_kernel(const __grid_constant__ Params P) {
+__global__ void __launch_bounds__(kThreads, kBF16 ? 4 : (kVideoLaunch ? 5 : 6)) direct_kernel(
+    const __grid_constant__ Params P) {
+    if constexpr (kBF16) {
+        direct_bf16x8<kVideoLaunch>(P);
+        return;
+    }
+    // fp32 rows: 4 pixels per thread
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int64_t B = P.block_start[P.n];
