@@ -823,8 +823,9 @@ __device__ __forceinline__ void convert4(const uint32_t (&w)[4], int C, float4 (
 // The direct kernel's bf16 rows: each half of the CTA (128 threads) takes
 // every other block of the CTA's range, and a thread owns 8 consecutive pixels
 // of one output row of its block, so each channel's 8 bf16 values leave in one
-// 16-byte store per temporal slot. Per pixel the arithmetic is that of the
-// fp32 path below, quad by quad, then the same round to bf16.
+// 16-byte store per temporal slot, and its two source rows arrive in a few wide
+// loads issued together. Per pixel the arithmetic is that of the fp32 path
+// below, quad by quad, then the same round to bf16.
 template <bool kVideoLaunch, class Params>
 __device__ __forceinline__ void direct_bf16x8(const Params &P) {
     const int tid = threadIdx.x;
@@ -925,23 +926,72 @@ __device__ __forceinline__ void direct_bf16x8(const Params &P) {
         [[maybe_unused]] const int64_t frame_bytes = static_cast<int64_t>(H) * W * C;
         const float2 ly2 = f2(ly, ly), nly2 = f2(-ly, -ly);
         uint32_t pk[3][4];  // channel c: bf16 pairs of pixels (0,1), (2,3), (4,5), (6,7)
+        // the loads of both quads of both rows go out before any conversion. RGBA: the 8 pixels of a row
+        // are 32 bytes at a 16-byte boundary, two 16-byte loads. RGB: 24 bytes at an 8-byte boundary
+        // (W a multiple of 32, the first column of 8, the frame 16-byte aligned), three 8-byte loads
+        uint2 ra[3] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u)};
+        uint2 rb[3] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u)};
+        uint4 qa4[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+        uint4 qb4[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+        if (C == 4) {
+            const int64_t x0 = static_cast<int64_t>(bw) * kBlock + dx0;
+            const int64_t pa = (static_cast<int64_t>(sy0) * W + x0) * 4, pb = (static_cast<int64_t>(sy1) * W + x0) * 4;
+            if (MIMO_CHECK(pa >= 0 && pa + 32 <= frame_bytes && f * D.frame_stride + pa + 32 <= D.limit &&
+                               (reinterpret_cast<uintptr_t>(img + pa) & 15u) == 0,
+                           kChkSrcLoad)) {
+                qa4[0] = __ldg(reinterpret_cast<const uint4 *>(img + pa));
+                qa4[1] = __ldg(reinterpret_cast<const uint4 *>(img + pa) + 1);
+            }
+            if (!yident && MIMO_CHECK(pb >= 0 && pb + 32 <= frame_bytes && f * D.frame_stride + pb + 32 <= D.limit &&
+                                          (reinterpret_cast<uintptr_t>(img + pb) & 15u) == 0,
+                                      kChkSrcLoad)) {
+                qb4[0] = __ldg(reinterpret_cast<const uint4 *>(img + pb));
+                qb4[1] = __ldg(reinterpret_cast<const uint4 *>(img + pb) + 1);
+            }
+        } else {
+            const int64_t x0 = static_cast<int64_t>(bw) * kBlock + dx0;
+            const int64_t pa = (static_cast<int64_t>(sy0) * W + x0) * 3, pb = (static_cast<int64_t>(sy1) * W + x0) * 3;
+            if (MIMO_CHECK(pa >= 0 && pa + 24 <= frame_bytes && f * D.frame_stride + pa + 24 <= D.limit &&
+                               (reinterpret_cast<uintptr_t>(img + pa) & 7u) == 0,
+                           kChkSrcLoad)) {
+                const uint2 *q = reinterpret_cast<const uint2 *>(img + pa);
+                ra[0] = __ldg(q);
+                ra[1] = __ldg(q + 1);
+                ra[2] = __ldg(q + 2);
+            }
+            if (!yident && MIMO_CHECK(pb >= 0 && pb + 24 <= frame_bytes && f * D.frame_stride + pb + 24 <= D.limit &&
+                                          (reinterpret_cast<uintptr_t>(img + pb) & 7u) == 0,
+                                      kChkSrcLoad)) {
+                const uint2 *q = reinterpret_cast<const uint2 *>(img + pb);
+                rb[0] = __ldg(q);
+                rb[1] = __ldg(q + 1);
+                rb[2] = __ldg(q + 2);
+            }
+        }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const int64_t x = static_cast<int64_t>(bw) * kBlock + dx0 + 4 * h;
             uint32_t wa[4] = {0u, 0u, 0u, 0u}, wb[4] = {0u, 0u, 0u, 0u};
             float4 va[3], vb[3];
-            const int64_t qa = (static_cast<int64_t>(sy0) * W + x) * C, qb = (static_cast<int64_t>(sy1) * W + x) * C;
-            if (MIMO_CHECK(qa >= 0 && qa + (C == 4 ? 16 : 12) <= frame_bytes &&
-                               f * D.frame_stride + qa + (C == 4 ? 16 : 12) <= D.limit,
-                           kChkSrcLoad))
-                load_quad(img + qa, C, wa);
-            if (!yident) {
-                if (MIMO_CHECK(qb >= 0 && qb + (C == 4 ? 16 : 12) <= frame_bytes &&
-                                   f * D.frame_stride + qb + (C == 4 ? 16 : 12) <= D.limit,
-                               kChkSrcLoad))
-                    load_quad(img + qb, C, wb);
-                convert4(wb, C, vb);
+            if (C == 3) {
+                // words 3h .. 3h+2 of the row's six
+                wa[0] = h ? ra[1].y : ra[0].x;
+                wa[1] = h ? ra[2].x : ra[0].y;
+                wa[2] = h ? ra[2].y : ra[1].x;
+                wb[0] = h ? rb[1].y : rb[0].x;
+                wb[1] = h ? rb[2].x : rb[0].y;
+                wb[2] = h ? rb[2].y : rb[1].x;
+            } else {
+                const uint4 a4 = h ? qa4[1] : qa4[0], b4 = h ? qb4[1] : qb4[0];
+                wa[0] = a4.x;
+                wa[1] = a4.y;
+                wa[2] = a4.z;
+                wa[3] = a4.w;
+                wb[0] = b4.x;
+                wb[1] = b4.y;
+                wb[2] = b4.z;
+                wb[3] = b4.w;
             }
+            if (!yident) convert4(wb, C, vb);
             convert4(wa, C, va);
 #pragma unroll
             for (int c = 0; c < 3; ++c) {
